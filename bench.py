@@ -1,0 +1,404 @@
+#!/usr/bin/env python
+"""Benchmark of the NVFP4 dense SwiGLU FFN on B200.
+
+One step = one FFN layer forward (fused gate+up projection with the SiLU*mul
+epilogue, then the down projection) over one batch of the workload's
+synthetic input, through the library's C ABI.  Default workload: prefill,
+m=4096 rows, hidden 5120, inter 17408, bf16 activations (W4A16); the value is
+whole-job TFLOP/s (2 * m * 3 * hidden * inter flops per step).  The same run
+also times the m=1 decode layer (weight GB/s) and the fixed-format W4A4 layer,
+reported as sub-objects.
+
+Usage: python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+       [--workload prefill|decode|smallm|w4a4] [--m M] [--no-extra] [--no-cpu]
+Under torchrun each rank runs its own replica (the FFN has no cross-GPU step
+here): the timed region is bracketed by a barrier and a device synchronise,
+the time is the max over ranks, and the value sums all ranks' work.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "NVFP4 FFN µs/layer & TFLOP/s (m=4096); weight GB/s (m=1) vs roofline"
+L2_BYTES = 126 * 1024 * 1024
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+WORKLOADS = {
+    # name: (synth recipe, m, hidden, inter, activation format)
+    "prefill": ("prefill", 4096, 5120, 17408, "bf16"),
+    "decode": ("decode", 1, 5120, 17408, "bf16"),
+    "smallm": ("smallm", 64, 5120, 17408, "bf16"),
+    "w4a4": ("w4a4", 512, 4096, 12288, "nvfp4_fixed"),
+}
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return {k: float(d[k]) for k in FALLBACK_PEAKS}, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def ffn_flops(m, H, I):
+    return 2.0 * m * 3 * H * I
+
+
+def nvfp4_bytes(n, k):
+    return n * k / 2 + n * k / 16
+
+
+# --------------------------------------------------------------- clocks
+
+class Clocks:
+    """nvidia-smi sampling of SM clocks and throttle reasons while running."""
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.tmp = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.Q}", "--format=csv,noheader,nounits",
+                 "-lms", "50"], stdout=self.tmp, stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.tmp.flush()
+        self.tmp.seek(0)
+        rows = [r.split(",") for r in self.tmp.read().strip().splitlines() if r.strip()]
+        os.unlink(self.tmp.name)
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for r in rows:
+            try:
+                sm.append(float(r[1]))
+                mx.append(float(r[2]))
+            except (ValueError, IndexError):
+                continue
+            for nm, v in zip(names, r[5:9]):
+                if v.strip().lower() == "active":
+                    reasons.add(nm)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# --------------------------------------------------------------- our arm
+
+class Workload:
+    def __init__(self, native, name, m=None):
+        import torch
+        from nvfp4_quantized_dense_w4a16_b200 import synth
+        recipe, m0, H, I, fmt = WORKLOADS[name]
+        self.name, self.m, self.H, self.I, self.fmt = name, (m or m0), H, I, fmt
+        inp = synth.make_inputs(recipe, m=self.m)
+        dev = lambda b: torch.from_numpy(np.ascontiguousarray(b).view(np.int16)).view(torch.bfloat16).cuda()
+        hs = []
+        for bits in (inp.w_gate, inp.w_up, inp.w_down):
+            w = dev(bits)
+            c, s, g = native.ffn_nvfp4_quantize_weights(w)
+            hs.append(native.ffn_nvfp4_weight_create(c, s, g))
+            del w, c, s, g
+        self.gate_up = native.ffn_nvfp4_weight_create_gate_up(hs[0], hs[1])
+        self.down = hs[2]
+        del hs[:2]
+        self.x = dev(inp.x)
+        self.x_bits = inp.x
+        self.out = torch.empty((self.m, H), dtype=torch.bfloat16, device="cuda")
+        self.ws = torch.empty((max(16, native.ffn_nvfp4_workspace_size(self.m, H, I, fmt)),),
+                              dtype=torch.uint8, device="cuda")
+        self.native = native
+        torch.cuda.synchronize()
+        # reads per step exceed L2 for prefill-size batches; otherwise flush
+        self.weight_bytes = nvfp4_bytes(2 * I, H) + nvfp4_bytes(H, I)
+        self.flush_l2 = self.weight_bytes + self.m * (H + I) * 4 < 2 * L2_BYTES
+
+    def step(self):
+        self.native.ffn_nvfp4_forward(self.x, self.gate_up, self.down, self.fmt, out=self.out,
+                                      workspace=self.ws)
+
+    def kernel_units(self, kname):
+        """(bound, algorithmic flops or bytes per launch) of a kernel of this layer."""
+        m, H, I = self.m, self.H, self.I
+        if "quantize_activations" in kname:
+            return "hbm", None
+        if "gate_up" in kname:
+            flops, byts = 2.0 * m * 2 * I * H, nvfp4_bytes(2 * I, H) + m * H * 2 + m * I * 2
+        else:
+            flops, byts = 2.0 * m * H * I, nvfp4_bytes(H, I) + m * I * 2 + m * H * 2
+        # tensor-bound when the arithmetic intensity exceeds the ridge point
+        return ("tensor", flops) if flops / byts > 250 else ("hbm", byts)
+
+
+def run_ours(args, rank, world, dist):
+    import torch
+    from nvfp4_quantized_dense_w4a16_b200 import build as B
+    B.build()
+    from nvfp4_quantized_dense_w4a16_b200 import native as N
+
+    peaks, peak_src = load_peaks()
+    dev_index = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(dev_index)
+    wl = Workload(N, args.workload, args.m)
+    flush = torch.empty(2 * L2_BYTES // 4, dtype=torch.float32, device="cuda") if wl.flush_l2 else None
+
+    def barrier():
+        if dist is not None:
+            dist.barrier()
+        torch.cuda.synchronize()
+
+    clocks = Clocks(dev_index)
+    clocks.start()
+    for _ in range(args.warmup):
+        wl.step()
+    barrier()
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    stops = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    N.ffn_nvfp4_profile_begin()
+    for i in range(args.steps):
+        if flush is not None:
+            flush.zero_()
+        starts[i].record()
+        wl.step()
+        stops[i].record()
+    barrier()
+    prof = N.ffn_nvfp4_profile_end()
+    clk = clocks.stop()
+    ms = sum(a.elapsed_time(b) for a, b in zip(starts, stops))
+    if dist is not None:
+        t = torch.tensor([ms], dtype=torch.float64, device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    ms_step = ms / args.steps
+    flops = ffn_flops(wl.m, wl.H, wl.I)
+    value = world * flops * args.steps / (ms * 1e-3) / 1e12
+
+    # dominant kernel and its roofline
+    roof = None
+    if prof:
+        kname, (launches, kms) = max(prof.items(), key=lambda kv: kv[1][1])
+        bound, units = wl.kernel_units(kname)
+        avg_s = kms / launches * 1e-3
+        if bound == "tensor":
+            peak = peaks["bf16_tflops"]
+            achieved = units / avg_s / 1e12
+            unit = "TFLOP/s"
+        else:
+            peak = peaks["hbm_gbs"]
+            achieved = units / avg_s / 1e9
+            unit = "GB/s"
+        roof = {"kernel": kname, "bound": bound, "achieved": round(achieved, 2), "peak": peak,
+                "peak_source": peak_src, "unit": unit, "frac": round(achieved / peak, 4),
+                "traffic": None, "avg_launch_us": round(avg_s * 1e6, 2), "launches": launches}
+    kernels = {k: {"launches": l, "total_ms": round(t, 4), "share": round(t / max(1e-9, sum(v[1] for v in prof.values())), 4)}
+               for k, (l, t) in prof.items()}
+    gpu_launches = sum(v[0] for v in prof.values())
+
+    # end to end through the public API with pinned host buffers
+    x_host = torch.from_numpy(np.ascontiguousarray(wl.x_bits).view(np.int16)).view(torch.bfloat16).pin_memory()
+    out_host = torch.empty((wl.m, wl.H), dtype=torch.bfloat16).pin_memory()
+    x_dev = torch.empty_like(wl.x)
+    e2e_steps = max(3, min(args.steps, 50))
+    for _ in range(2):
+        x_dev.copy_(x_host, non_blocking=True)
+        N.ffn_nvfp4_forward(x_dev, wl.gate_up, wl.down, wl.fmt, out=wl.out, workspace=wl.ws)
+        out_host.copy_(wl.out, non_blocking=True)
+    barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(e2e_steps):
+        x_dev.copy_(x_host, non_blocking=True)
+        N.ffn_nvfp4_forward(x_dev, wl.gate_up, wl.down, wl.fmt, out=wl.out, workspace=wl.ws)
+        out_host.copy_(wl.out, non_blocking=True)
+    e1.record()
+    barrier()
+    e2e_ms = e0.elapsed_time(e1)
+    if dist is not None:
+        t = torch.tensor([e2e_ms], dtype=torch.float64, device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+    e2e = {"value": round(world * flops * e2e_steps / (e2e_ms * 1e-3) / 1e12, 3), "unit": "TFLOP/s",
+           "h2d_bytes_per_step": wl.m * wl.H * 2, "d2h_bytes_per_step": wl.m * wl.H * 2,
+           "ms_per_step": round(e2e_ms / e2e_steps, 4)}
+
+    extra = {}
+    if not args.no_extra and args.workload == "prefill":
+        del wl, x_dev
+        torch.cuda.empty_cache()
+        extra["decode_m1"] = secondary(N, "decode", 1, peaks, steps=max(args.steps, 20))
+        extra["w4a4_m512"] = secondary(N, "w4a4", 512, peaks, steps=max(args.steps // 2, 5))
+        torch.cuda.empty_cache()
+    return {
+        "value": round(value, 3), "ms_per_step": round(ms_step, 4), "roofline": roof,
+        "kernels": kernels, "gpu_launches": gpu_launches, "clocks": clk, "e2e": e2e,
+        "workload": args.workload, "m": args.m or WORKLOADS[args.workload][1], "extra": extra,
+        "l2": "flushed between timed steps" if flush is not None else "inputs larger than L2",
+    }
+
+
+def secondary(N, name, m, peaks, steps):
+    """Time another layer shape: per-step µs, weight GB/s and TFLOP/s."""
+    import torch
+    wl = Workload(N, name, m)
+    flush = torch.empty(2 * L2_BYTES // 4, dtype=torch.float32, device="cuda")
+    for _ in range(3):
+        wl.step()
+    torch.cuda.synchronize()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    N.ffn_nvfp4_profile_begin()
+    for a, b in ev:
+        flush.zero_()
+        a.record()
+        wl.step()
+        b.record()
+    torch.cuda.synchronize()
+    prof = N.ffn_nvfp4_profile_end()
+    ms = sum(a.elapsed_time(b) for a, b in ev) / steps
+    res = {"m": m, "hidden": wl.H, "inter": wl.I, "format": wl.fmt, "us_per_layer": round(ms * 1e3, 2),
+           "weight_gbs": round(wl.weight_bytes / (ms * 1e-3) / 1e9, 1),
+           "tflops": round(ffn_flops(m, wl.H, wl.I) / (ms * 1e-3) / 1e12, 3),
+           "hbm_roofline_frac": round(wl.weight_bytes / (ms * 1e-3) / 1e9 / peaks["hbm_gbs"], 4),
+           "kernels": {k: {"launches": l, "avg_us": round(t / l * 1e3, 2)} for k, (l, t) in prof.items()}}
+    del wl
+    return res
+
+
+# --------------------------------------------------------------- CPU oracle
+
+def oracle_sample(name, rows, reps, warmup=0):
+    """Time the CPU oracle on `rows` rows of the workload (after quantising the
+    weights with the oracle).  Returns (seconds per rep, flops per rep, threads)."""
+    from nvfp4_quantized_dense_w4a16_b200 import synth
+    from oracle import nvfp4_ffn as O
+    recipe, m0, H, I, fmt = WORKLOADS[name]
+    inp = synth.make_inputs(recipe, m=max(rows, 1))
+    q = [O.quantize_weight(synth.bf16_bits_to_f32(b)) for b in (inp.w_gate, inp.w_up, inp.w_down)]
+    x = synth.bf16_bits_to_f32(inp.x[:rows]).astype(np.float64)
+    f = O.ffn_w4a16 if fmt == "bf16" else O.ffn_w4a4
+    for _ in range(warmup):
+        f(x, *q)
+    times = []
+    for _ in range(reps):
+        t0 = time.perf_counter()
+        f(x, *q)
+        times.append(time.perf_counter() - t0)
+    try:
+        from threadpoolctl import threadpool_info
+        threads = max([p.get("num_threads", 1) for p in threadpool_info()] or [1])
+    except Exception:
+        threads = os.cpu_count() or 1
+    return times, ffn_flops(rows, H, I), threads
+
+
+def cpu_baseline(name, rows=1, reps=1):
+    times, fl, threads = oracle_sample(name, rows, reps)
+    s = statistics.mean(times)
+    return {"value": round(fl / s / 1e12, 6), "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
+            "sample": f"{rows} row(s) of the {name} workload through the fp64 numpy oracle "
+                      f"(weights pre-quantised by the oracle), mean of {reps} run(s), {s:.2f} s each"}
+
+
+def run_reference(args):
+    rows = 1
+    times, fl, threads = oracle_sample(args.workload, rows, args.steps, warmup=min(args.warmup, 1))
+    s = sum(times)
+    value = fl * args.steps / s / 1e12
+    recipe, m0, H, I, fmt = WORKLOADS[args.workload]
+    line = {
+        "impl": "reference", "metric": METRIC, "value": round(value, 6), "unit": "TFLOP/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(s / args.steps * 1e3, 3), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": args.workload, "m": args.m or m0, "hidden": H, "inter": I,
+                   "act_format": fmt, "sample_rows_per_step": rows},
+        "cpu_baseline": {"value": round(value, 6), "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
+                         "sample": f"{rows} row per step of the {args.workload} workload (fp64 numpy oracle)"},
+        "e2e": {"value": round(value, 6), "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", choices=sorted(WORKLOADS), default="prefill")
+    ap.add_argument("--m", type=int, default=None)
+    ap.add_argument("--no-extra", action="store_true")
+    ap.add_argument("--no-cpu", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+
+    if args.impl == "reference":
+        if rank == 0:
+            run_reference(args)
+        return
+
+    dist = None
+    if world > 1:
+        import datetime
+        import torch
+        import torch.distributed as dist
+        torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", "0")))
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
+    res = run_ours(args, rank, world, dist)
+    if dist is not None:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank != 0:
+        return
+    recipe, m0, H, I, fmt = WORKLOADS[args.workload]
+    cpu = None
+    if world == 1 and not args.no_cpu:
+        cpu = cpu_baseline(args.workload)
+    line = {
+        "metric": METRIC, "value": res["value"], "unit": "TFLOP/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": res["ms_per_step"],
+        "us_per_layer": round(res["ms_per_step"] * 1e3, 2),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16 x nvfp4 (fp32 accumulate)" if fmt == "bf16" else "nvfp4 x nvfp4 (fp32 accumulate)",
+        "data": "synthetic (seeded numpy draws; random-init weights)",
+        "config": {"workload": args.workload, "m": res["m"], "hidden": H, "inter": I, "act_format": fmt,
+                   "parallelism": f"replicas x{world}", "l2": res["l2"]},
+        "roofline": res["roofline"], "cpu_baseline": cpu, "e2e": res["e2e"],
+        "gpu_launches": res["gpu_launches"], "kernels": res["kernels"], "clocks": res["clocks"],
+    }
+    line.update(res["extra"])
+    print(json.dumps(line), flush=True)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,194 @@
+/*
+ * ffn_nvfp4.h -- C ABI of the NVFP4 dense SwiGLU FFN for NVIDIA B200 (sm_100a).
+ *
+ * The library computes one LLM serving layer,
+ *
+ *     out = down( silu( gate(x) ) * up(x) )
+ *
+ * over NVFP4 weights: FP4 E2M1 codes, one FP8 E4M3 scale per 16 consecutive
+ * elements along K, and one FP32 scale per tensor.  Activations are bf16
+ * (W4A16), or, in the fixed activation format, are themselves quantised per
+ * row to NVFP4 before every projection (W4A4) so that a row's output bits do
+ * not depend on how many rows share the call.
+ *
+ * Where each operation comes from (pages of the metrale engine's source):
+ *  - the FFN dataflow (gate and up into bf16 buffers, silu_mul in place, down
+ *    from the activated buffer): "metrale_model_layers/layers/
+ *    dense_ffn_fixed.rs", DenseFfnLayer::forward_fixed, and
+ *    "metrale_model_layers/layers/dense_ffn_prefill.rs", prefill_q2;
+ *  - the fixed activation format and its row-count invariance: the module
+ *    comment of "metrale_model_layers/layers/dense_ffn_fixed.rs";
+ *  - one NVFP4 projection for m rows (the W4A16 GEMM family and its m
+ *    dispatch): "metrale_model_layers/layers/dense_ffn_prefill.rs",
+ *    DenseFfnLayer::w4a16_prefill_gemm;
+ *  - the fused [2*inter, hidden] gate+up weight whose halves are the gate and
+ *    up weights: "metrale_model_layers/layers/dense_ffn_overlays.rs",
+ *    set_fp8_gate_up_fused;
+ *  - errors instead of silent fallbacks: the bail!/ensure! results of the
+ *    same pages.
+ * The NVFP4 encoding is the public one (OCP MX v1.0 FP4 E2M1 elements, OCP
+ * OFP8 E4M3 block scales); the conventions for the scales are stated at
+ * ffn_nvfp4_quantize_weights and ffn_nvfp4_quantize_activations.
+ *
+ * Conventions for every entry point
+ *  - All tensor pointers are DEVICE pointers on the current CUDA device unless
+ *    a parameter says otherwise; the caller owns them.  Work is enqueued on
+ *    `stream` (a cudaStream_t passed as void*; NULL = the legacy default
+ *    stream).  No entry point synchronises the stream, and the compute entry
+ *    points (quantize_*, forward, linear) allocate no memory.
+ *  - Row-major layouts: a [rows, cols] tensor has cols contiguous.
+ *    bf16 tensors are IEEE bfloat16 bit patterns.
+ *  - NVFP4 tensors of logical shape [rows, k]: `codes` is uint8 [rows, k/2],
+ *    byte j holding element 2j in its low nibble and 2j+1 in its high nibble
+ *    (nibble: bit 3 sign, bits 0-2 magnitude index into {0,.5,1,1.5,2,3,4,6});
+ *    `block_scales` is uint8 [rows, k/16], one E4M3 byte per 16 elements.
+ *  - Pointers must be 16-byte aligned; k must be a multiple of 32.
+ *  - On any error nothing is launched and an ffn_status other than FFN_OK is
+ *    returned; asynchronous CUDA errors of earlier work surface as
+ *    FFN_ERR_CUDA from the next call or at the caller's stream synchronise.
+ *    No entry point aborts the process.
+ */
+#ifndef FFN_NVFP4_H
+#define FFN_NVFP4_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define FFN_NVFP4_ABI_VERSION 1
+
+typedef enum ffn_status {
+  FFN_OK = 0,
+  FFN_ERR_INVALID_ARG = 1, /* null pointer, negative size, bad enum value   */
+  FFN_ERR_SHAPE = 2,       /* dims not multiples of 32, handle dims mismatch */
+  FFN_ERR_ALIGNMENT = 3,   /* a pointer is not 16-byte aligned              */
+  FFN_ERR_UNSUPPORTED = 4, /* a valid request this build does not serve     */
+  FFN_ERR_CUDA = 5,        /* a CUDA runtime call or launch failed          */
+  FFN_ERR_OOM = 6,         /* device allocation failed (handle creation)    */
+  FFN_ERR_WORKSPACE = 7    /* workspace missing or smaller than required    */
+} ffn_status;
+
+typedef enum ffn_act_format {
+  FFN_ACT_BF16 = 0,        /* W4A16: bf16 activations                       */
+  FFN_ACT_NVFP4_FIXED = 1  /* W4A4: activations quantised per row to NVFP4  */
+} ffn_act_format;
+
+/* Opaque NVFP4 weight: owns device copies of the codes, the block scales and
+ * the tensor scale(s), plus the re-tiled copies the kernels read.  Immutable
+ * after creation; may be shared by concurrent calls on several streams. */
+typedef struct ffn_nvfp4_weight ffn_nvfp4_weight;
+
+/* Human-readable name of a status code (static storage). */
+const char* ffn_status_string(ffn_status s);
+
+/* FFN_NVFP4_ABI_VERSION of the built library. */
+int ffn_nvfp4_abi_version(void);
+
+/* Quantise a bf16 weight W[n, k] to NVFP4.
+ *   w_bf16        [n, k] bf16 (input)
+ *   codes         uint8 [n, k/2]  (output)
+ *   block_scales  uint8 [n, k/16] (output, E4M3)
+ *   global_scale  one float (output, device)
+ * Arithmetic (all fp32, round-to-nearest-even): amax = max|W|;
+ * gs = amax / 2688 (2688 = 6 * 448; gs = 1 if amax == 0); per 16-element block
+ * t = (block amax / gs) / 6, s = E4M3(t) with saturation to 448,
+ * sdec = E4M3value(s) * gs, code = E2M1(w / sdec) rounding to nearest with
+ * ties to the even magnitude index, saturating at 6 and keeping the sign bit;
+ * a block whose s (or sdec) is zero gets code 0 throughout.  The result is
+ * deterministic and bit-reproducible.  Inputs must be finite.
+ * Launches three kernels; no host synchronisation. */
+ffn_status ffn_nvfp4_quantize_weights(const void* w_bf16, int64_t n, int64_t k,
+                                      void* codes, void* block_scales,
+                                      float* global_scale, void* stream);
+
+/* Quantise bf16 activations X[m, k] per row to NVFP4, as the fixed format does
+ * before each projection: per 16-element block s = E4M3(block amax / 6) (fp32,
+ * nearest even, saturating), code = E2M1(x / E4M3value(s)), no tensor scale;
+ * all-zero block when s == 0.  codes uint8 [m, k/2], block_scales uint8
+ * [m, k/16].  Exposed so callers can check the activation codes bit for bit. */
+ffn_status ffn_nvfp4_quantize_activations(const void* x_bf16, int64_t m, int64_t k,
+                                          void* codes, void* block_scales,
+                                          void* stream);
+
+/* Build a weight handle from NVFP4 tensors of logical shape [n, k] (codes,
+ * block_scales as above, global_scale one device float).  Copies the data
+ * (the caller keeps ownership of its buffers) and builds the kernel layouts.
+ * Allocates device memory; enqueues copies on `stream`; the handle is usable
+ * by later work on `stream` (other streams: synchronise first).
+ * Errors: FFN_ERR_SHAPE unless n > 0 and k is a positive multiple of 32. */
+ffn_status ffn_nvfp4_weight_create(const void* codes, const void* block_scales,
+                                   const float* global_scale, int64_t n, int64_t k,
+                                   void* stream, ffn_nvfp4_weight** out);
+
+/* Fused gate+up handle of logical shape [2*inter, hidden]: rows [0, inter)
+ * are `gate`, rows [inter, 2*inter) are `up`, byte for byte, each keeping its
+ * own tensor scale.  `gate` and `up` must share (n, k) and stay owned by the
+ * caller (they may be destroyed afterwards). */
+ffn_status ffn_nvfp4_weight_create_gate_up(const ffn_nvfp4_weight* gate,
+                                           const ffn_nvfp4_weight* up, void* stream,
+                                           ffn_nvfp4_weight** out);
+
+/* Release a handle and its device memory (synchronises the device first, so
+ * no queued work still reads it).  NULL is accepted. */
+ffn_status ffn_nvfp4_weight_destroy(ffn_nvfp4_weight* w);
+
+/* Logical dims of a handle; *is_gate_up = 1 for a fused gate+up handle. */
+ffn_status ffn_nvfp4_weight_dims(const ffn_nvfp4_weight* w, int64_t* n, int64_t* k,
+                                 int* is_gate_up);
+
+/* Workspace bytes ffn_nvfp4_forward needs for (m, hidden, inter, format). */
+ffn_status ffn_nvfp4_workspace_size(int64_t m, int64_t hidden, int64_t inter,
+                                    ffn_act_format format, size_t* bytes);
+
+/* The FFN layer for m rows.
+ *   x        [m, hidden] bf16
+ *   gate_up  fused handle [2*inter, hidden] (ffn_nvfp4_weight_create_gate_up)
+ *   down     handle [hidden, inter]
+ *   out      [m, hidden] bf16; only rows 0..m-1 are written
+ *   workspace device scratch of >= ffn_nvfp4_workspace_size bytes; holds the
+ *            bf16 intermediate h = silu(g) * u and, in the fixed format, the
+ *            quantised activations; contents are undefined afterwards.
+ * Numerics: g = bf16(gs_g * sum x*w_g), u likewise, h = bf16(silu(g) * u),
+ * out = bf16(gs_d * sum h*w_d), with fp32 accumulation.  In FFN_ACT_NVFP4_FIXED
+ * x and h are quantised per row (as ffn_nvfp4_quantize_activations) before
+ * their projections, and the kernels and reduction order do not depend on m,
+ * so each output row is bit-identical whatever m is.
+ * m == 0 is a no-op.  Allocates nothing and does not synchronise. */
+ffn_status ffn_nvfp4_forward(const void* x, int64_t m, int64_t hidden, int64_t inter,
+                             const ffn_nvfp4_weight* gate_up, const ffn_nvfp4_weight* down,
+                             ffn_act_format format, void* out, void* workspace,
+                             size_t workspace_bytes, void* stream);
+
+/* One projection y[m, n] = bf16(gs * sum_k x[m, k] * w[n, k]) for a plain
+ * (not gate+up) handle of shape [n, k]; in FFN_ACT_NVFP4_FIXED x is quantised
+ * per row first.  Workspace: ffn_nvfp4_linear_workspace_size bytes. */
+ffn_status ffn_nvfp4_linear_workspace_size(int64_t m, int64_t n, int64_t k,
+                                           ffn_act_format format, size_t* bytes);
+ffn_status ffn_nvfp4_linear(const void* x, int64_t m, const ffn_nvfp4_weight* w,
+                            ffn_act_format format, void* y, void* workspace,
+                            size_t workspace_bytes, void* stream);
+
+/* Per-kernel timing (opt-in tracing).  After ffn_nvfp4_profile_begin, every
+ * kernel launch the library makes from the calling thread is bracketed by a
+ * pair of CUDA events recorded on the launch's stream.  ffn_nvfp4_profile_end
+ * stops recording, synchronises the device, and aggregates the durations per
+ * kernel into out[0..*count) (name: static string; capacity entries at most,
+ * FFN_ERR_INVALID_ARG if more distinct kernels ran).  Recording adds event
+ * records to the streams but no device work; it creates CUDA events (host
+ * resources) on first use and reuses them afterwards. */
+typedef struct ffn_kernel_time {
+  const char* name;
+  int launches;
+  double total_ms;
+} ffn_kernel_time;
+ffn_status ffn_nvfp4_profile_begin(void);
+ffn_status ffn_nvfp4_profile_end(ffn_kernel_time* out, int capacity, int* count);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FFN_NVFP4_H */

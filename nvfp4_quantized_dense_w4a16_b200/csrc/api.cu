@@ -1,0 +1,308 @@
+// C ABI of the NVFP4 SwiGLU FFN: argument checks, weight handles, workspace
+// carving and the per-call kernel dispatch.  See include/ffn_nvfp4.h.
+#include <new>
+
+#include "ffn_nvfp4.h"
+#include "internal.h"
+
+using ffn::Epilogue;
+using ffn::WeightView;
+
+struct ffn_nvfp4_weight {
+  int64_t n = 0, k = 0;
+  int gate_up = 0;
+  int device = 0;
+  uint8_t* codes = nullptr;   // [n, k/2] canonical
+  uint8_t* scales = nullptr;  // [n, k/16] canonical
+  float* gs = nullptr;        // 1 float, or 2 (gate, up) for a fused handle
+  WeightView view() const { return WeightView{codes, scales, gs, n, k}; }
+};
+
+namespace {
+
+inline cudaStream_t as_stream(void* s) { return reinterpret_cast<cudaStream_t>(s); }
+
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+inline ffn_status cuda_status(cudaError_t e) { return e == cudaSuccess ? FFN_OK : FFN_ERR_CUDA; }
+
+inline size_t round_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+// Pick up errors of earlier asynchronous work before enqueuing more.
+inline ffn_status precheck() {
+  const cudaError_t e = cudaPeekAtLastError();
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    return FFN_ERR_CUDA;
+  }
+  return FFN_OK;
+}
+
+bool valid_k(int64_t k) { return k > 0 && k % 32 == 0; }
+
+// Workspace layout of ffn_nvfp4_forward / ffn_nvfp4_linear (each region
+// 256-byte aligned): [h bf16 m*inter] [xq codes m*hidden/2] [xq scales
+// m*hidden/16] [hq codes m*inter/2] [hq scales m*inter/16].
+struct Carve {
+  size_t h = 0, xq_c = 0, xq_s = 0, hq_c = 0, hq_s = 0, total = 0;
+};
+
+Carve carve_ffn(int64_t m, int64_t hidden, int64_t inter, ffn_act_format f) {
+  Carve c;
+  size_t off = 0;
+  c.h = off;
+  off += round_up((size_t)m * inter * 2, 256);
+  if (f == FFN_ACT_NVFP4_FIXED) {
+    c.xq_c = off; off += round_up((size_t)m * hidden / 2, 256);
+    c.xq_s = off; off += round_up((size_t)m * hidden / 16, 256);
+    c.hq_c = off; off += round_up((size_t)m * inter / 2, 256);
+    c.hq_s = off; off += round_up((size_t)m * inter / 16, 256);
+  }
+  c.total = off;
+  return c;
+}
+
+Carve carve_linear(int64_t m, int64_t k, ffn_act_format f) {
+  Carve c;
+  size_t off = 0;
+  if (f == FFN_ACT_NVFP4_FIXED) {
+    c.xq_c = off; off += round_up((size_t)m * k / 2, 256);
+    c.xq_s = off; off += round_up((size_t)m * k / 16, 256);
+  }
+  c.total = off;
+  return c;
+}
+
+template <class T>
+ffn_status alloc(T** p, size_t bytes) {
+  if (cudaMalloc(reinterpret_cast<void**>(p), bytes) != cudaSuccess) {
+    cudaGetLastError();
+    *p = nullptr;
+    return FFN_ERR_OOM;
+  }
+  return FFN_OK;
+}
+
+void free_weight(ffn_nvfp4_weight* w) {
+  if (!w) return;
+  cudaFree(w->codes);
+  cudaFree(w->scales);
+  cudaFree(w->gs);
+  delete w;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* ffn_status_string(ffn_status s) {
+  switch (s) {
+    case FFN_OK: return "FFN_OK";
+    case FFN_ERR_INVALID_ARG: return "FFN_ERR_INVALID_ARG";
+    case FFN_ERR_SHAPE: return "FFN_ERR_SHAPE";
+    case FFN_ERR_ALIGNMENT: return "FFN_ERR_ALIGNMENT";
+    case FFN_ERR_UNSUPPORTED: return "FFN_ERR_UNSUPPORTED";
+    case FFN_ERR_CUDA: return "FFN_ERR_CUDA";
+    case FFN_ERR_OOM: return "FFN_ERR_OOM";
+    case FFN_ERR_WORKSPACE: return "FFN_ERR_WORKSPACE";
+  }
+  return "FFN_ERR_UNKNOWN";
+}
+
+int ffn_nvfp4_abi_version(void) { return FFN_NVFP4_ABI_VERSION; }
+
+ffn_status ffn_nvfp4_quantize_weights(const void* w_bf16, int64_t n, int64_t k, void* codes,
+                                      void* block_scales, float* global_scale, void* stream) {
+  if (!w_bf16 || !codes || !block_scales || !global_scale) return FFN_ERR_INVALID_ARG;
+  if (n <= 0 || !valid_k(k)) return FFN_ERR_SHAPE;
+  if (!aligned16(w_bf16) || !aligned16(codes) || !aligned16(block_scales) ||
+      (reinterpret_cast<uintptr_t>(global_scale) & 3u))
+    return FFN_ERR_ALIGNMENT;
+  if (ffn_status st = precheck()) return st;
+  return cuda_status(ffn::launch_quantize_weights(w_bf16, n, k, codes, block_scales,
+                                                  global_scale, as_stream(stream)));
+}
+
+ffn_status ffn_nvfp4_quantize_activations(const void* x_bf16, int64_t m, int64_t k, void* codes,
+                                          void* block_scales, void* stream) {
+  if (m < 0) return FFN_ERR_INVALID_ARG;
+  if (!valid_k(k)) return FFN_ERR_SHAPE;
+  if (m == 0) return FFN_OK;
+  if (!x_bf16 || !codes || !block_scales) return FFN_ERR_INVALID_ARG;
+  if (!aligned16(x_bf16) || !aligned16(codes) || !aligned16(block_scales))
+    return FFN_ERR_ALIGNMENT;
+  if (ffn_status st = precheck()) return st;
+  return cuda_status(
+      ffn::launch_quantize_activations(x_bf16, m, k, codes, block_scales, as_stream(stream)));
+}
+
+ffn_status ffn_nvfp4_weight_create(const void* codes, const void* block_scales,
+                                   const float* global_scale, int64_t n, int64_t k,
+                                   void* stream, ffn_nvfp4_weight** out) {
+  if (!out) return FFN_ERR_INVALID_ARG;
+  *out = nullptr;
+  if (!codes || !block_scales || !global_scale) return FFN_ERR_INVALID_ARG;
+  if (n <= 0 || !valid_k(k)) return FFN_ERR_SHAPE;
+  if (!aligned16(codes) || !aligned16(block_scales)) return FFN_ERR_ALIGNMENT;
+  if (ffn_status st = precheck()) return st;
+  auto* w = new (std::nothrow) ffn_nvfp4_weight;
+  if (!w) return FFN_ERR_OOM;
+  w->n = n;
+  w->k = k;
+  cudaGetDevice(&w->device);
+  const cudaStream_t s = as_stream(stream);
+  ffn_status st = FFN_OK;
+  if ((st = alloc(&w->codes, (size_t)n * k / 2)) || (st = alloc(&w->scales, (size_t)n * k / 16)) ||
+      (st = alloc(&w->gs, 2 * sizeof(float)))) {
+    free_weight(w);
+    return st;
+  }
+  cudaError_t e = cudaMemcpyAsync(w->codes, codes, (size_t)n * k / 2, cudaMemcpyDeviceToDevice, s);
+  if (e == cudaSuccess)
+    e = cudaMemcpyAsync(w->scales, block_scales, (size_t)n * k / 16, cudaMemcpyDeviceToDevice, s);
+  if (e == cudaSuccess)
+    e = cudaMemcpyAsync(w->gs, global_scale, sizeof(float), cudaMemcpyDeviceToDevice, s);
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    free_weight(w);
+    return FFN_ERR_CUDA;
+  }
+  *out = w;
+  return FFN_OK;
+}
+
+ffn_status ffn_nvfp4_weight_create_gate_up(const ffn_nvfp4_weight* gate,
+                                           const ffn_nvfp4_weight* up, void* stream,
+                                           ffn_nvfp4_weight** out) {
+  if (!out) return FFN_ERR_INVALID_ARG;
+  *out = nullptr;
+  if (!gate || !up) return FFN_ERR_INVALID_ARG;
+  if (gate->gate_up || up->gate_up) return FFN_ERR_INVALID_ARG;
+  if (gate->n != up->n || gate->k != up->k) return FFN_ERR_SHAPE;
+  if (ffn_status st = precheck()) return st;
+  const int64_t I = gate->n, H = gate->k;
+  auto* w = new (std::nothrow) ffn_nvfp4_weight;
+  if (!w) return FFN_ERR_OOM;
+  w->n = 2 * I;
+  w->k = H;
+  w->gate_up = 1;
+  cudaGetDevice(&w->device);
+  const cudaStream_t s = as_stream(stream);
+  ffn_status st = FFN_OK;
+  const size_t cb = (size_t)I * H / 2, sb = (size_t)I * H / 16;
+  if ((st = alloc(&w->codes, 2 * cb)) || (st = alloc(&w->scales, 2 * sb)) ||
+      (st = alloc(&w->gs, 2 * sizeof(float)))) {
+    free_weight(w);
+    return st;
+  }
+  cudaError_t e = cudaMemcpyAsync(w->codes, gate->codes, cb, cudaMemcpyDeviceToDevice, s);
+  if (e == cudaSuccess) e = cudaMemcpyAsync(w->codes + cb, up->codes, cb, cudaMemcpyDeviceToDevice, s);
+  if (e == cudaSuccess) e = cudaMemcpyAsync(w->scales, gate->scales, sb, cudaMemcpyDeviceToDevice, s);
+  if (e == cudaSuccess) e = cudaMemcpyAsync(w->scales + sb, up->scales, sb, cudaMemcpyDeviceToDevice, s);
+  if (e == cudaSuccess) e = cudaMemcpyAsync(w->gs, gate->gs, sizeof(float), cudaMemcpyDeviceToDevice, s);
+  if (e == cudaSuccess) e = cudaMemcpyAsync(w->gs + 1, up->gs, sizeof(float), cudaMemcpyDeviceToDevice, s);
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    free_weight(w);
+    return FFN_ERR_CUDA;
+  }
+  *out = w;
+  return FFN_OK;
+}
+
+ffn_status ffn_nvfp4_weight_destroy(ffn_nvfp4_weight* w) {
+  if (!w) return FFN_OK;
+  const cudaError_t e = cudaDeviceSynchronize();
+  free_weight(w);
+  return cuda_status(e);
+}
+
+ffn_status ffn_nvfp4_weight_dims(const ffn_nvfp4_weight* w, int64_t* n, int64_t* k,
+                                 int* is_gate_up) {
+  if (!w) return FFN_ERR_INVALID_ARG;
+  if (n) *n = w->n;
+  if (k) *k = w->k;
+  if (is_gate_up) *is_gate_up = w->gate_up;
+  return FFN_OK;
+}
+
+ffn_status ffn_nvfp4_workspace_size(int64_t m, int64_t hidden, int64_t inter,
+                                    ffn_act_format format, size_t* bytes) {
+  if (!bytes || m < 0) return FFN_ERR_INVALID_ARG;
+  if (format != FFN_ACT_BF16 && format != FFN_ACT_NVFP4_FIXED) return FFN_ERR_INVALID_ARG;
+  if (!valid_k(hidden) || !valid_k(inter)) return FFN_ERR_SHAPE;
+  *bytes = carve_ffn(m, hidden, inter, format).total;
+  return FFN_OK;
+}
+
+ffn_status ffn_nvfp4_forward(const void* x, int64_t m, int64_t hidden, int64_t inter,
+                             const ffn_nvfp4_weight* gate_up, const ffn_nvfp4_weight* down,
+                             ffn_act_format format, void* out, void* workspace,
+                             size_t workspace_bytes, void* stream) {
+  if (m < 0 || !gate_up || !down) return FFN_ERR_INVALID_ARG;
+  if (format != FFN_ACT_BF16 && format != FFN_ACT_NVFP4_FIXED) return FFN_ERR_INVALID_ARG;
+  if (!valid_k(hidden) || !valid_k(inter)) return FFN_ERR_SHAPE;
+  if (!gate_up->gate_up || down->gate_up) return FFN_ERR_INVALID_ARG;
+  if (gate_up->n != 2 * inter || gate_up->k != hidden || down->n != hidden || down->k != inter)
+    return FFN_ERR_SHAPE;
+  if (m == 0) return FFN_OK;
+  if (!x || !out) return FFN_ERR_INVALID_ARG;
+  const Carve c = carve_ffn(m, hidden, inter, format);
+  if (!workspace || workspace_bytes < c.total) return FFN_ERR_WORKSPACE;
+  if (!aligned16(x) || !aligned16(out) || !aligned16(workspace)) return FFN_ERR_ALIGNMENT;
+  if (ffn_status st = precheck()) return st;
+  const cudaStream_t s = as_stream(stream);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  void* h = ws + c.h;
+  cudaError_t e;
+  if (format == FFN_ACT_BF16) {
+    e = ffn::launch_gemv_w4a16(x, m, gate_up->view(), Epilogue::kSiluMul, h, s);
+    if (e == cudaSuccess) e = ffn::launch_gemv_w4a16(h, m, down->view(), Epilogue::kStore, out, s);
+  } else {
+    uint8_t *xq = ws + c.xq_c, *xs = ws + c.xq_s, *hq = ws + c.hq_c, *hs = ws + c.hq_s;
+    e = ffn::launch_quantize_activations(x, m, hidden, xq, xs, s);
+    if (e == cudaSuccess)
+      e = ffn::launch_gemv_w4a4(xq, xs, m, gate_up->view(), Epilogue::kSiluMul, h, s);
+    if (e == cudaSuccess) e = ffn::launch_quantize_activations(h, m, inter, hq, hs, s);
+    if (e == cudaSuccess)
+      e = ffn::launch_gemv_w4a4(hq, hs, m, down->view(), Epilogue::kStore, out, s);
+  }
+  return cuda_status(e);
+}
+
+ffn_status ffn_nvfp4_linear_workspace_size(int64_t m, int64_t n, int64_t k,
+                                           ffn_act_format format, size_t* bytes) {
+  if (!bytes || m < 0 || n <= 0) return FFN_ERR_INVALID_ARG;
+  if (format != FFN_ACT_BF16 && format != FFN_ACT_NVFP4_FIXED) return FFN_ERR_INVALID_ARG;
+  if (!valid_k(k)) return FFN_ERR_SHAPE;
+  *bytes = carve_linear(m, k, format).total;
+  return FFN_OK;
+}
+
+ffn_status ffn_nvfp4_linear(const void* x, int64_t m, const ffn_nvfp4_weight* w,
+                            ffn_act_format format, void* y, void* workspace,
+                            size_t workspace_bytes, void* stream) {
+  if (m < 0 || !w) return FFN_ERR_INVALID_ARG;
+  if (format != FFN_ACT_BF16 && format != FFN_ACT_NVFP4_FIXED) return FFN_ERR_INVALID_ARG;
+  if (w->gate_up) return FFN_ERR_UNSUPPORTED;
+  if (m == 0) return FFN_OK;
+  if (!x || !y) return FFN_ERR_INVALID_ARG;
+  const Carve c = carve_linear(m, w->k, format);
+  if (c.total && (!workspace || workspace_bytes < c.total)) return FFN_ERR_WORKSPACE;
+  if (!aligned16(x) || !aligned16(y) || (c.total && !aligned16(workspace)))
+    return FFN_ERR_ALIGNMENT;
+  if (ffn_status st = precheck()) return st;
+  const cudaStream_t s = as_stream(stream);
+  cudaError_t e;
+  if (format == FFN_ACT_BF16) {
+    e = ffn::launch_gemv_w4a16(x, m, w->view(), Epilogue::kStore, y, s);
+  } else {
+    uint8_t* ws = static_cast<uint8_t*>(workspace);
+    e = ffn::launch_quantize_activations(x, m, w->k, ws + c.xq_c, ws + c.xq_s, s);
+    if (e == cudaSuccess)
+      e = ffn::launch_gemv_w4a4(ws + c.xq_c, ws + c.xq_s, m, w->view(), Epilogue::kStore, y, s);
+  }
+  return cuda_status(e);
+}
+
+}  // extern "C"

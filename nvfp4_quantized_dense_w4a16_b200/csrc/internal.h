@@ -1,0 +1,35 @@
+// Host-side declarations shared by the library's translation units.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace ffn {
+
+// Operand of one projection: canonical NVFP4 layout of a [n, k] weight.
+// For a fused gate+up weight, rows [0, n/2) are gate and [n/2, n) are up and
+// gs points at two floats (gate, up).
+struct WeightView {
+  const uint8_t* codes;   // [n, k/2]
+  const uint8_t* scales;  // [n, k/16]
+  const float* gs;        // 1 or 2 device floats
+  int64_t n, k;
+};
+
+enum class Epilogue : int {
+  kStore = 0,   // y[r, j] = bf16(gs * acc)
+  kSiluMul = 1  // h[r, j] = bf16(silu(bf16(gs_g*acc_g)) * bf16(gs_u*acc_u)), j < n/2
+};
+
+cudaError_t launch_quantize_weights(const void* w, int64_t n, int64_t k, void* codes,
+                                    void* scales, float* gs, cudaStream_t s);
+cudaError_t launch_quantize_activations(const void* x, int64_t m, int64_t k, void* codes,
+                                        void* scales, cudaStream_t s);
+
+// CUDA-core projections (any m; used for small m and as the general path).
+cudaError_t launch_gemv_w4a16(const void* x, int64_t m, const WeightView& w, Epilogue ep,
+                              void* y, cudaStream_t s);
+cudaError_t launch_gemv_w4a4(const uint8_t* xcodes, const uint8_t* xscales, int64_t m,
+                             const WeightView& w, Epilogue ep, void* y, cudaStream_t s);
+
+}  // namespace ffn

@@ -1,0 +1,263 @@
+"""ctypes binding of ``libffn_nvfp4.so`` (include/ffn_nvfp4.h).
+
+Argument marshalling only: every function takes torch tensors, checks their
+device, dtype, shape and contiguity, and passes raw pointers, sizes and the
+current CUDA stream to the C ABI of the same name.  All compute happens in the
+library's CUDA kernels; there is no CPU fallback, and importing this module
+fails loudly when the library has not been built.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import re
+
+import torch
+
+PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(PKG, "libffn_nvfp4.so")
+HEADER = os.path.join(os.path.dirname(PKG), "include", "ffn_nvfp4.h")
+
+FFN_ACT_BF16 = 0
+FFN_ACT_NVFP4_FIXED = 1
+_FORMATS = {"bf16": FFN_ACT_BF16, "w4a16": FFN_ACT_BF16,
+            "nvfp4_fixed": FFN_ACT_NVFP4_FIXED, "w4a4": FFN_ACT_NVFP4_FIXED}
+
+
+class FfnError(RuntimeError):
+    def __init__(self, fn: str, status: int, name: str):
+        super().__init__(f"{fn} failed: {name} ({status})")
+        self.status = status
+        self.status_name = name
+
+
+class KernelTime(ctypes.Structure):
+    _fields_ = [("name", ctypes.c_char_p), ("launches", ctypes.c_int), ("total_ms", ctypes.c_double)]
+
+
+def _load() -> ctypes.CDLL:
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(
+            f"{LIB_PATH} is missing: build it with `python -m nvfp4_quantized_dense_w4a16_b200.build` "
+            "(the NVFP4 FFN has no CPU implementation)")
+    lib = ctypes.CDLL(LIB_PATH)
+    vp, i64, sz = ctypes.c_void_p, ctypes.c_int64, ctypes.c_size_t
+    P = ctypes.POINTER
+    sig = {
+        "ffn_status_string": (ctypes.c_char_p, [ctypes.c_int]),
+        "ffn_nvfp4_abi_version": (ctypes.c_int, []),
+        "ffn_nvfp4_quantize_weights": (ctypes.c_int, [vp, i64, i64, vp, vp, vp, vp]),
+        "ffn_nvfp4_quantize_activations": (ctypes.c_int, [vp, i64, i64, vp, vp, vp]),
+        "ffn_nvfp4_weight_create": (ctypes.c_int, [vp, vp, vp, i64, i64, vp, P(vp)]),
+        "ffn_nvfp4_weight_create_gate_up": (ctypes.c_int, [vp, vp, vp, P(vp)]),
+        "ffn_nvfp4_weight_destroy": (ctypes.c_int, [vp]),
+        "ffn_nvfp4_weight_dims": (ctypes.c_int, [vp, P(i64), P(i64), P(ctypes.c_int)]),
+        "ffn_nvfp4_workspace_size": (ctypes.c_int, [i64, i64, i64, ctypes.c_int, P(sz)]),
+        "ffn_nvfp4_forward": (ctypes.c_int, [vp, i64, i64, i64, vp, vp, ctypes.c_int, vp, vp, sz, vp]),
+        "ffn_nvfp4_linear_workspace_size": (ctypes.c_int, [i64, i64, i64, ctypes.c_int, P(sz)]),
+        "ffn_nvfp4_linear": (ctypes.c_int, [vp, i64, vp, ctypes.c_int, vp, vp, sz, vp]),
+        "ffn_nvfp4_profile_begin": (ctypes.c_int, []),
+        "ffn_nvfp4_profile_end": (ctypes.c_int, [P(KernelTime), ctypes.c_int, P(ctypes.c_int)]),
+    }
+    for name, (res, args) in sig.items():
+        f = getattr(lib, name)
+        f.restype = res
+        f.argtypes = args
+    return lib
+
+
+lib = _load()
+
+
+def declared_symbols(header: str = HEADER) -> list[str]:
+    """Function names declared in the public header."""
+    text = open(header).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(ffn_[a-z0-9_]+)\s*\(", text)))
+
+
+def status_string(status: int) -> str:
+    return lib.ffn_status_string(status).decode()
+
+
+def _check(fn: str, status: int):
+    if status != 0:
+        raise FfnError(fn, status, status_string(status))
+
+
+def _fmt(fmt) -> int:
+    if isinstance(fmt, int):
+        return fmt
+    return _FORMATS[fmt]
+
+
+def _stream(stream=None) -> int:
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return s.cuda_stream
+
+
+def _ptr(t: torch.Tensor | None):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _need(t: torch.Tensor, name: str, dtype: torch.dtype, shape=None):
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor (the library has no CPU path)")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
+
+
+def ffn_nvfp4_abi_version() -> int:
+    return lib.ffn_nvfp4_abi_version()
+
+
+def ffn_nvfp4_quantize_weights(w: torch.Tensor, codes=None, block_scales=None, global_scale=None,
+                               stream=None):
+    """bf16 [n, k] -> (codes uint8 [n, k/2], block_scales uint8 [n, k/16], gs float32 [1])."""
+    _need(w, "w", torch.bfloat16)
+    n, k = w.shape
+    dev = w.device
+    codes = torch.empty((n, k // 2), dtype=torch.uint8, device=dev) if codes is None else codes
+    block_scales = torch.empty((n, k // 16), dtype=torch.uint8, device=dev) if block_scales is None else block_scales
+    global_scale = torch.empty((1,), dtype=torch.float32, device=dev) if global_scale is None else global_scale
+    _need(codes, "codes", torch.uint8, (n, k // 2))
+    _need(block_scales, "block_scales", torch.uint8, (n, k // 16))
+    _need(global_scale, "global_scale", torch.float32, (1,))
+    _check("ffn_nvfp4_quantize_weights", lib.ffn_nvfp4_quantize_weights(
+        _ptr(w), n, k, _ptr(codes), _ptr(block_scales), _ptr(global_scale), _stream(stream)))
+    return codes, block_scales, global_scale
+
+
+def ffn_nvfp4_quantize_activations(x: torch.Tensor, codes=None, block_scales=None, stream=None):
+    """bf16 [m, k] -> (codes uint8 [m, k/2], block_scales uint8 [m, k/16])."""
+    _need(x, "x", torch.bfloat16)
+    m, k = x.shape
+    codes = torch.empty((m, k // 2), dtype=torch.uint8, device=x.device) if codes is None else codes
+    block_scales = torch.empty((m, k // 16), dtype=torch.uint8, device=x.device) if block_scales is None else block_scales
+    _need(codes, "codes", torch.uint8, (m, k // 2))
+    _need(block_scales, "block_scales", torch.uint8, (m, k // 16))
+    _check("ffn_nvfp4_quantize_activations", lib.ffn_nvfp4_quantize_activations(
+        _ptr(x), m, k, _ptr(codes), _ptr(block_scales), _stream(stream)))
+    return codes, block_scales
+
+
+class Weight:
+    """Owning wrapper of an ``ffn_nvfp4_weight*`` handle."""
+
+    def __init__(self, handle: ctypes.c_void_p):
+        self._h = handle
+        n, k, gu = ctypes.c_int64(), ctypes.c_int64(), ctypes.c_int()
+        _check("ffn_nvfp4_weight_dims", lib.ffn_nvfp4_weight_dims(
+            self._h, ctypes.byref(n), ctypes.byref(k), ctypes.byref(gu)))
+        self.n, self.k, self.is_gate_up = n.value, k.value, bool(gu.value)
+
+    @property
+    def handle(self):
+        return self._h
+
+    def close(self):
+        if self._h:
+            _check("ffn_nvfp4_weight_destroy", lib.ffn_nvfp4_weight_destroy(self._h))
+            self._h = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+
+def ffn_nvfp4_weight_create(codes: torch.Tensor, block_scales: torch.Tensor,
+                            global_scale: torch.Tensor, stream=None) -> Weight:
+    _need(codes, "codes", torch.uint8)
+    n, half_k = codes.shape
+    k = 2 * half_k
+    _need(block_scales, "block_scales", torch.uint8, (n, k // 16))
+    _need(global_scale, "global_scale", torch.float32, (1,))
+    h = ctypes.c_void_p()
+    _check("ffn_nvfp4_weight_create", lib.ffn_nvfp4_weight_create(
+        _ptr(codes), _ptr(block_scales), _ptr(global_scale), n, k, _stream(stream), ctypes.byref(h)))
+    return Weight(h)
+
+
+def ffn_nvfp4_weight_create_gate_up(gate: Weight, up: Weight, stream=None) -> Weight:
+    h = ctypes.c_void_p()
+    _check("ffn_nvfp4_weight_create_gate_up", lib.ffn_nvfp4_weight_create_gate_up(
+        gate.handle, up.handle, _stream(stream), ctypes.byref(h)))
+    return Weight(h)
+
+
+def ffn_nvfp4_workspace_size(m: int, hidden: int, inter: int, fmt="bf16") -> int:
+    out = ctypes.c_size_t()
+    _check("ffn_nvfp4_workspace_size", lib.ffn_nvfp4_workspace_size(m, hidden, inter, _fmt(fmt), ctypes.byref(out)))
+    return out.value
+
+
+def ffn_nvfp4_linear_workspace_size(m: int, n: int, k: int, fmt="bf16") -> int:
+    out = ctypes.c_size_t()
+    _check("ffn_nvfp4_linear_workspace_size", lib.ffn_nvfp4_linear_workspace_size(m, n, k, _fmt(fmt), ctypes.byref(out)))
+    return out.value
+
+
+def _workspace(nbytes: int, device, workspace):
+    if workspace is None:
+        workspace = torch.empty((max(nbytes, 16),), dtype=torch.uint8, device=device)
+    _need(workspace, "workspace", torch.uint8)
+    if workspace.numel() < nbytes:
+        raise ValueError(f"workspace needs {nbytes} bytes, got {workspace.numel()}")
+    return workspace
+
+
+def ffn_nvfp4_forward(x: torch.Tensor, gate_up: Weight, down: Weight, fmt="bf16", out=None,
+                      workspace=None, stream=None) -> torch.Tensor:
+    """out[m, hidden] = down(silu(gate(x)) * up(x)) through the C ABI."""
+    _need(x, "x", torch.bfloat16)
+    m, hidden = x.shape
+    inter = down.k
+    if gate_up.k != hidden:
+        raise ValueError(f"x has {hidden} columns, gate_up expects {gate_up.k}")
+    out = torch.empty((m, hidden), dtype=torch.bfloat16, device=x.device) if out is None else out
+    _need(out, "out", torch.bfloat16, (m, hidden))
+    nbytes = ffn_nvfp4_workspace_size(m, hidden, inter, fmt)
+    workspace = _workspace(nbytes, x.device, workspace)
+    _check("ffn_nvfp4_forward", lib.ffn_nvfp4_forward(
+        _ptr(x), m, hidden, inter, gate_up.handle, down.handle, _fmt(fmt), _ptr(out),
+        _ptr(workspace), workspace.numel(), _stream(stream)))
+    return out
+
+
+def ffn_nvfp4_linear(x: torch.Tensor, w: Weight, fmt="bf16", y=None, workspace=None,
+                     stream=None) -> torch.Tensor:
+    """y[m, n] = bf16(gs * x @ w^T) (x quantised per row first in the fixed format)."""
+    _need(x, "x", torch.bfloat16)
+    m, k = x.shape
+    if k != w.k:
+        raise ValueError(f"x has {k} columns, the weight expects {w.k}")
+    y = torch.empty((m, w.n), dtype=torch.bfloat16, device=x.device) if y is None else y
+    _need(y, "y", torch.bfloat16, (m, w.n))
+    nbytes = ffn_nvfp4_linear_workspace_size(m, w.n, k, fmt)
+    workspace = _workspace(nbytes, x.device, workspace)
+    _check("ffn_nvfp4_linear", lib.ffn_nvfp4_linear(
+        _ptr(x), m, w.handle, _fmt(fmt), _ptr(y), _ptr(workspace), workspace.numel(),
+        _stream(stream)))
+    return y
+
+
+def ffn_nvfp4_profile_begin():
+    """Start timing every kernel the library launches from this thread."""
+    _check("ffn_nvfp4_profile_begin", lib.ffn_nvfp4_profile_begin())
+
+
+def ffn_nvfp4_profile_end() -> dict:
+    """Stop timing; {kernel name: (launches, total ms)} (synchronises the device)."""
+    cap = 64
+    arr = (KernelTime * cap)()
+    n = ctypes.c_int()
+    _check("ffn_nvfp4_profile_end", lib.ffn_nvfp4_profile_end(arr, cap, ctypes.byref(n)))
+    return {arr[i].name.decode(): (arr[i].launches, arr[i].total_ms) for i in range(n.value)}
