@@ -206,11 +206,11 @@ def ffn_nvfp4_linear_workspace_size(m: int, n: int, k: int, fmt="bf16") -> int:
 
 
 def _workspace(nbytes: int, device, workspace):
+    """A fresh workspace of the required size, or the caller's (whose size the
+    C ABI checks, returning FFN_ERR_WORKSPACE when it is too small)."""
     if workspace is None:
         workspace = torch.empty((max(nbytes, 16),), dtype=torch.uint8, device=device)
     _need(workspace, "workspace", torch.uint8)
-    if workspace.numel() < nbytes:
-        raise ValueError(f"workspace needs {nbytes} bytes, got {workspace.numel()}")
     return workspace
 
 
