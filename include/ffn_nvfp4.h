@@ -171,6 +171,14 @@ ffn_status ffn_nvfp4_linear(const void* x, int64_t m, const ffn_nvfp4_weight* w,
                             ffn_act_format format, void* y, void* workspace,
                             size_t workspace_bytes, void* stream);
 
+/* Device-side error bits.  Kernels that wait on asynchronous copies or on
+ * tensor-core completion give up after about two seconds instead of hanging,
+ * free their tensor memory, skip their stores and OR a bit into a device-wide
+ * error word (1: producer, 2: MMA issuer, 4: dequant, 8: epilogue, 16: drain
+ * timeout).  Synchronises the device, writes the word to *flags and, if
+ * clear != 0, resets it to zero.  0 means every kernel completed normally. */
+ffn_status ffn_nvfp4_device_error(int* flags, int clear);
+
 /* Per-kernel timing (opt-in tracing).  After ffn_nvfp4_profile_begin, every
  * kernel launch the library makes from the calling thread is bracketed by a
  * pair of CUDA events recorded on the launch's stream.  ffn_nvfp4_profile_end

@@ -1,5 +1,8 @@
 // C ABI of the NVFP4 SwiGLU FFN: argument checks, weight handles, workspace
 // carving and the per-call kernel dispatch.  See include/ffn_nvfp4.h.
+#include <stdlib.h>
+#include <string.h>
+
 #include <new>
 
 #include "ffn_nvfp4.h"
@@ -15,7 +18,9 @@ struct ffn_nvfp4_weight {
   uint8_t* codes = nullptr;   // [n, k/2] canonical
   uint8_t* scales = nullptr;  // [n, k/16] canonical
   float* gs = nullptr;        // 1 float, or 2 (gate, up) for a fused handle
+  uint8_t* tiled = nullptr;   // tensor-core layout (see tc_gemm.cu)
   WeightView view() const { return WeightView{codes, scales, gs, n, k}; }
+  ffn::TcWeight tc() const { return ffn::TcWeight{tiled, gs, n, k}; }
 };
 
 namespace {
@@ -40,11 +45,40 @@ inline ffn_status precheck() {
 
 bool valid_k(int64_t k) { return k > 0 && k % 32 == 0; }
 
+int num_sms() {
+  int dev = 0, n = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) {
+    cudaGetLastError();
+    return 148;  // B200
+  }
+  return n;
+}
+
+// Projection kernel family for m rows: the tensor-core GEMM, or the CUDA-core
+// GEMV.  FFN_NVFP4_W4A16_PATH=gemv|tc overrides (read once) for measurements.
+enum class Path { kTc, kGemv };
+
+Path w4a16_path(int64_t m) {
+  static int forced = [] {
+    const char* v = getenv("FFN_NVFP4_W4A16_PATH");
+    if (!v) return 0;
+    if (!strcmp(v, "gemv")) return 1;
+    if (!strcmp(v, "tc")) return 2;
+    return 0;
+  }();
+  if (forced == 1) return Path::kGemv;
+  if (forced == 2) return Path::kTc;
+  (void)m;
+  return Path::kTc;
+}
+
 // Workspace layout of ffn_nvfp4_forward / ffn_nvfp4_linear (each region
 // 256-byte aligned): [h bf16 m*inter] [xq codes m*hidden/2] [xq scales
 // m*hidden/16] [hq codes m*inter/2] [hq scales m*inter/16].
 struct Carve {
-  size_t h = 0, xq_c = 0, xq_s = 0, hq_c = 0, hq_s = 0, total = 0;
+  size_t h = 0, xq_c = 0, xq_s = 0, hq_c = 0, hq_s = 0, part = 0, total = 0;
+  ffn::TcPlan gate_up, down;
 };
 
 Carve carve_ffn(int64_t m, int64_t hidden, int64_t inter, ffn_act_format f) {
@@ -52,6 +86,15 @@ Carve carve_ffn(int64_t m, int64_t hidden, int64_t inter, ffn_act_format f) {
   size_t off = 0;
   c.h = off;
   off += round_up((size_t)m * inter * 2, 256);
+  if (f == FFN_ACT_BF16 && m > 0 && w4a16_path(m) == Path::kTc) {
+    const int sms = num_sms();
+    c.gate_up = ffn::plan_tc(m, 2 * inter, hidden, true, sms);
+    c.down = ffn::plan_tc(m, hidden, inter, false, sms);
+    const size_t pb = c.gate_up.partial_bytes > c.down.partial_bytes ? c.gate_up.partial_bytes
+                                                                    : c.down.partial_bytes;
+    c.part = off;
+    off += round_up(pb, 256);
+  }
   if (f == FFN_ACT_NVFP4_FIXED) {
     c.xq_c = off; off += round_up((size_t)m * hidden / 2, 256);
     c.xq_s = off; off += round_up((size_t)m * hidden / 16, 256);
@@ -62,9 +105,14 @@ Carve carve_ffn(int64_t m, int64_t hidden, int64_t inter, ffn_act_format f) {
   return c;
 }
 
-Carve carve_linear(int64_t m, int64_t k, ffn_act_format f) {
+Carve carve_linear(int64_t m, int64_t n, int64_t k, ffn_act_format f) {
   Carve c;
   size_t off = 0;
+  if (f == FFN_ACT_BF16 && m > 0 && w4a16_path(m) == Path::kTc) {
+    c.down = ffn::plan_tc(m, n, k, false, num_sms());
+    c.part = off;
+    off += round_up(c.down.partial_bytes, 256);
+  }
   if (f == FFN_ACT_NVFP4_FIXED) {
     c.xq_c = off; off += round_up((size_t)m * k / 2, 256);
     c.xq_s = off; off += round_up((size_t)m * k / 16, 256);
@@ -88,6 +136,7 @@ void free_weight(ffn_nvfp4_weight* w) {
   cudaFree(w->codes);
   cudaFree(w->scales);
   cudaFree(w->gs);
+  cudaFree(w->tiled);
   delete w;
 }
 
@@ -162,6 +211,13 @@ ffn_status ffn_nvfp4_weight_create(const void* codes, const void* block_scales,
     e = cudaMemcpyAsync(w->scales, block_scales, (size_t)n * k / 16, cudaMemcpyDeviceToDevice, s);
   if (e == cudaSuccess)
     e = cudaMemcpyAsync(w->gs, global_scale, sizeof(float), cudaMemcpyDeviceToDevice, s);
+  if (e == cudaSuccess) {
+    if ((st = alloc(&w->tiled, (size_t)ffn::tc_tiled_bytes(n, k, false)))) {
+      free_weight(w);
+      return st;
+    }
+    e = ffn::launch_tile_weight(w->codes, w->scales, n, k, false, w->tiled, s);
+  }
   if (e != cudaSuccess) {
     cudaGetLastError();
     free_weight(w);
@@ -201,6 +257,13 @@ ffn_status ffn_nvfp4_weight_create_gate_up(const ffn_nvfp4_weight* gate,
   if (e == cudaSuccess) e = cudaMemcpyAsync(w->scales + sb, up->scales, sb, cudaMemcpyDeviceToDevice, s);
   if (e == cudaSuccess) e = cudaMemcpyAsync(w->gs, gate->gs, sizeof(float), cudaMemcpyDeviceToDevice, s);
   if (e == cudaSuccess) e = cudaMemcpyAsync(w->gs + 1, up->gs, sizeof(float), cudaMemcpyDeviceToDevice, s);
+  if (e == cudaSuccess) {
+    if ((st = alloc(&w->tiled, (size_t)ffn::tc_tiled_bytes(2 * I, H, true)))) {
+      free_weight(w);
+      return st;
+    }
+    e = ffn::launch_tile_weight(w->codes, w->scales, 2 * I, H, true, w->tiled, s);
+  }
   if (e != cudaSuccess) {
     cudaGetLastError();
     free_weight(w);
@@ -255,7 +318,11 @@ ffn_status ffn_nvfp4_forward(const void* x, int64_t m, int64_t hidden, int64_t i
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   void* h = ws + c.h;
   cudaError_t e;
-  if (format == FFN_ACT_BF16) {
+  if (format == FFN_ACT_BF16 && w4a16_path(m) == Path::kTc) {
+    void* part = ws + c.part;
+    e = ffn::launch_tc_w4a16(x, m, gate_up->tc(), true, c.gate_up, h, part, s);
+    if (e == cudaSuccess) e = ffn::launch_tc_w4a16(h, m, down->tc(), false, c.down, out, part, s);
+  } else if (format == FFN_ACT_BF16) {
     e = ffn::launch_gemv_w4a16(x, m, gate_up->view(), Epilogue::kSiluMul, h, s);
     if (e == cudaSuccess) e = ffn::launch_gemv_w4a16(h, m, down->view(), Epilogue::kStore, out, s);
   } else {
@@ -270,12 +337,21 @@ ffn_status ffn_nvfp4_forward(const void* x, int64_t m, int64_t hidden, int64_t i
   return cuda_status(e);
 }
 
+ffn_status ffn_nvfp4_device_error(int* flags, int clear) {
+  if (!flags) return FFN_ERR_INVALID_ARG;
+  if (cudaDeviceSynchronize() != cudaSuccess) {
+    cudaGetLastError();
+    return FFN_ERR_CUDA;
+  }
+  return cuda_status(ffn::read_device_error(flags, clear != 0));
+}
+
 ffn_status ffn_nvfp4_linear_workspace_size(int64_t m, int64_t n, int64_t k,
                                            ffn_act_format format, size_t* bytes) {
   if (!bytes || m < 0 || n <= 0) return FFN_ERR_INVALID_ARG;
   if (format != FFN_ACT_BF16 && format != FFN_ACT_NVFP4_FIXED) return FFN_ERR_INVALID_ARG;
   if (!valid_k(k)) return FFN_ERR_SHAPE;
-  *bytes = carve_linear(m, k, format).total;
+  *bytes = carve_linear(m, n, k, format).total;
   return FFN_OK;
 }
 
@@ -287,14 +363,16 @@ ffn_status ffn_nvfp4_linear(const void* x, int64_t m, const ffn_nvfp4_weight* w,
   if (w->gate_up) return FFN_ERR_UNSUPPORTED;
   if (m == 0) return FFN_OK;
   if (!x || !y) return FFN_ERR_INVALID_ARG;
-  const Carve c = carve_linear(m, w->k, format);
+  const Carve c = carve_linear(m, w->n, w->k, format);
   if (c.total && (!workspace || workspace_bytes < c.total)) return FFN_ERR_WORKSPACE;
   if (!aligned16(x) || !aligned16(y) || (c.total && !aligned16(workspace)))
     return FFN_ERR_ALIGNMENT;
   if (ffn_status st = precheck()) return st;
   const cudaStream_t s = as_stream(stream);
   cudaError_t e;
-  if (format == FFN_ACT_BF16) {
+  if (format == FFN_ACT_BF16 && w4a16_path(m) == Path::kTc) {
+    e = ffn::launch_tc_w4a16(x, m, w->tc(), false, c.down, y, static_cast<uint8_t*>(workspace) + c.part, s);
+  } else if (format == FFN_ACT_BF16) {
     e = ffn::launch_gemv_w4a16(x, m, w->view(), Epilogue::kStore, y, s);
   } else {
     uint8_t* ws = static_cast<uint8_t*>(workspace);

@@ -21,6 +21,28 @@ enum class Epilogue : int {
   kSiluMul = 1  // h[r, j] = bf16(silu(bf16(gs_g*acc_g)) * bf16(gs_u*acc_u)), j < n/2
 };
 
+// Tensor-core (tcgen05) projection over the pre-tiled weight layout.
+struct TcWeight {
+  const uint8_t* tiled;  // [tiles][ceil(k/64)][4608]
+  const float* gs;       // 1 or 2 device floats
+  int64_t n, k;          // logical dims (n = 2*inter for a fused gate+up weight)
+};
+
+struct TcPlan {
+  int bn = 0;            // activation rows per tile (MMA N)
+  int xtiles = 0, wtiles = 0, kc = 0, kc_per_split = 0, splits = 1, n_pad = 0;
+  size_t partial_bytes = 0;  // fp32 split-K partials needed in the workspace
+};
+
+TcPlan plan_tc(int64_t m, int64_t n, int64_t k, bool gate_up, int num_sms);
+int64_t tc_tiled_bytes(int64_t n, int64_t k, bool gate_up);
+cudaError_t launch_tile_weight(const uint8_t* codes, const uint8_t* scales, int64_t n, int64_t k,
+                               bool gate_up, uint8_t* out, cudaStream_t s);
+cudaError_t launch_tc_w4a16(const void* x, int64_t m, const TcWeight& w, bool silu_mul,
+                            const TcPlan& p, void* y, void* partials, cudaStream_t s);
+// Device-wide error bits set by kernels whose bounded waits gave up.
+cudaError_t read_device_error(int* flags, bool clear);
+
 cudaError_t launch_quantize_weights(const void* w, int64_t n, int64_t k, void* codes,
                                     void* scales, float* gs, cudaStream_t s);
 cudaError_t launch_quantize_activations(const void* x, int64_t m, int64_t k, void* codes,

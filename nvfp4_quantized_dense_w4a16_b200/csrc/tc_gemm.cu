@@ -1,0 +1,511 @@
+// tcgen05 (5th-generation tensor core) NVFP4-weight x bf16-activation GEMM
+// for sm_100a: one projection D[n, r] = sum_k W[n, k] * X[r, k] of the FFN
+// ("metrale_model_layers/layers/dense_ffn_prefill.rs", w4a16_prefill_gemm:
+// the NVFP4 projection GEMM the layer runs for m rows).
+//
+// Design (one CTA per 128-weight-row tile x BN activation rows x K range):
+//  * weights are streamed in a pre-tiled layout (per 128-row tile and
+//    64-element K chunk: 128 x 16 B low codes, 128 x 16 B high codes,
+//    128 x 4 B E4M3 scales = 4608 B) by one bulk async copy per stage;
+//  * activations X [m, K] bf16 arrive by 2-D TMA with the 128-byte swizzle
+//    (box 64 x BN), the layout the MMA reads directly;
+//  * four dequant warps turn each thread's row of codes into exact bf16
+//    values (E2M1 value * E4M3 block scale: at most 6 significant bits) with
+//    byte-permute table lookups and write them straight into tensor memory,
+//    where they are the MMA's A operand (M = 128 weight rows) -- so the
+//    dequantised weights never occupy shared-memory bandwidth;
+//  * one thread issues tcgen05.mma kind::f16 (A from TMEM, B = X tile from
+//    shared memory, fp32 accumulator in TMEM, N = BN);
+//  * the four dequant warps then read the accumulator back (tcgen05.ld) and
+//    run the epilogue: y = bf16(gs * acc); or for the fused gate+up weight
+//    (64 gate rows then the matching 64 up rows per tile) the SiLU*mul
+//    h = bf16(silu(bf16(gs_g*g)) * bf16(gs_u*u)); or fp32 split-K partials.
+// Pipelines are mbarrier-driven; every wait is bounded and, on timeout, sets
+// a device error bit and lets the CTA free its TMEM and exit.
+#include <cudaTypedefs.h>
+
+#include <mutex>
+
+#include "common.cuh"
+#include "internal.h"
+#include "profile.h"
+#include "sm100.cuh"
+
+namespace ffn {
+
+__device__ int g_ffn_device_error = 0;
+
+using namespace sm100;
+
+namespace {
+
+constexpr int kChunkK = 64;        // K elements per stage
+constexpr int kTileRows = 128;     // weight rows per tile = TMEM lanes
+constexpr int kChunkBytes = 4608;  // 128 x (16 + 16 + 4) bytes
+
+enum : int { kEpiStore = 0, kEpiSiluMul = 1, kEpiPartial = 2 };
+
+template <int BN, int STAGES>
+struct TcCfg {
+  static constexpr int kXStageBytes = BN * 128;
+  static constexpr int kAColBase = BN < 32 ? 32 : BN;  // TMEM column of A stage 0
+  static constexpr int kTmemNeed = kAColBase + 32 * STAGES;
+  static constexpr int kTmemCols = kTmemNeed <= 64 ? 64 : kTmemNeed <= 128 ? 128 : kTmemNeed <= 256 ? 256 : 512;
+  static constexpr int kEpiBytes = 16384;
+  static constexpr int kSmemW = STAGES * kXStageBytes;
+  static constexpr int kSmemEpi = kSmemW + STAGES * kChunkBytes;
+  static constexpr int kSmemBar = kSmemEpi + kEpiBytes;
+  static constexpr int kSmemBytes = kSmemBar + (3 * STAGES + 1) * 8 + 16;
+  static constexpr int kSmemAlloc = kSmemBytes + 1024;  // slack for 1024-byte alignment
+  static_assert(kTmemNeed <= 512, "TMEM budget");
+  static_assert(kSmemAlloc <= 232448, "shared memory budget");
+  static_assert(BN % 16 == 0 && BN >= 16 && BN <= 256, "MMA N");
+};
+
+struct TcArgs {
+  const uint8_t* wt;   // tiled weight [tiles][kc_total][4608]
+  const float* gs;     // tensor scale(s)
+  void* out;           // bf16 [m, ldo] or fp32 partials [splits][m][n_pad]
+  int m, n_out, ldo, kc_total, kc_per_split, n_pad;
+};
+
+__device__ __forceinline__ uint32_t bmul2(uint32_t a, uint32_t b) {
+  __nv_bfloat162 r = __hmul2(*reinterpret_cast<__nv_bfloat162*>(&a),
+                             *reinterpret_cast<__nv_bfloat162*>(&b));
+  return *reinterpret_cast<uint32_t*>(&r);
+}
+
+// E4M3 byte -> (s, s) as bf16x2 (exact: 4 significant bits, exponent 2^-9..2^8).
+__device__ __forceinline__ uint32_t scale_pair(uint32_t s8) {
+  const uint32_t b = __float_as_uint(e4m3_decode(s8)) >> 16;
+  return b | (b << 16);
+}
+
+// Eight E2M1 codes (nibble i = element i) times the block scale pair ->
+// four bf16x2 words (element 2j in the low half of word j).  The bf16 bytes of
+// the magnitudes {0, .5, 1, 1.5, 2, 3, 4, 6} are looked up with byte permutes:
+// high bytes {00,3F,3F,3F,40,40,40,40}, low bytes {00,00,80,C0,00,40,80,C0};
+// the sign (nibble bit 3) is moved to bit 7 of the high byte.
+__device__ __forceinline__ void dequant8(uint32_t c, uint32_t s2, uint32_t* o) {
+  const uint32_t mags = c & 0x77777777u;
+  const uint32_t m47 = mags >> 16;
+  const uint32_t c4 = c << 4;
+  uint32_t hi03 = __byte_perm(0x3F3F3F00u, 0x40404040u, mags);
+  uint32_t lo03 = __byte_perm(0xC0800000u, 0xC0804000u, mags);
+  uint32_t hi47 = __byte_perm(0x3F3F3F00u, 0x40404040u, m47);
+  uint32_t lo47 = __byte_perm(0xC0800000u, 0xC0804000u, m47);
+  hi03 |= __byte_perm(c4, c, 0x5140) & 0x80808080u;
+  hi47 |= __byte_perm(c4, c, 0x7362) & 0x80808080u;
+  o[0] = bmul2(__byte_perm(lo03, hi03, 0x5140), s2);
+  o[1] = bmul2(__byte_perm(lo03, hi03, 0x7362), s2);
+  o[2] = bmul2(__byte_perm(lo47, hi47, 0x5140), s2);
+  o[3] = bmul2(__byte_perm(lo47, hi47, 0x7362), s2);
+}
+
+// One thread's 64-element chunk of its weight row -> 32 bf16x2 TMEM columns.
+__device__ __forceinline__ void dequant64(const uint4 lo, const uint4 hi, uint32_t sc,
+                                          uint32_t (&v)[32]) {
+  const uint32_t s0 = scale_pair(sc & 0xffu), s1 = scale_pair((sc >> 8) & 0xffu);
+  const uint32_t s2 = scale_pair((sc >> 16) & 0xffu), s3 = scale_pair(sc >> 24);
+  dequant8(lo.x, s0, v + 0);
+  dequant8(lo.y, s0, v + 4);
+  dequant8(lo.z, s1, v + 8);
+  dequant8(lo.w, s1, v + 12);
+  dequant8(hi.x, s2, v + 16);
+  dequant8(hi.y, s2, v + 20);
+  dequant8(hi.z, s3, v + 24);
+  dequant8(hi.w, s3, v + 28);
+}
+
+// Bounded wait that ignores the abort flag (used to drain in-flight work).
+__device__ __forceinline__ bool wait_drain(uint64_t* bar, uint32_t parity) {
+  const long long t0 = clock64();
+  while (!mbar_try_wait(bar, parity)) {
+    if (clock64() - t0 > kWaitLimitCycles) {
+      atomicOr(&g_ffn_device_error, 16);
+      return false;
+    }
+  }
+  return true;
+}
+
+template <int BN, int STAGES, int EPI>
+__global__ void __launch_bounds__(256, (BN <= 64 ? 2 : 1))
+tc_w4a16_kernel(const __grid_constant__ CUtensorMap xmap, const TcArgs a) {
+  using C = TcCfg<BN, STAGES>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  uint8_t* xs = smem;
+  uint8_t* wsm = smem + C::kSmemW;
+  uint8_t* epi = smem + C::kSmemEpi;
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::kSmemBar);
+  uint64_t* empty = full + STAGES;
+  uint64_t* afull = empty + STAGES;
+  uint64_t* accum = afull + STAGES;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(accum + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  int* err = &g_ffn_device_error;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int xtile = blockIdx.x, wtile = blockIdx.y;
+  const int kc0 = blockIdx.z * a.kc_per_split;
+  const int nk = min(a.kc_total, kc0 + a.kc_per_split) - kc0;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+      mbar_init(&afull[s], 4);
+    }
+    mbar_init(accum, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 2) {
+    tmem_alloc(tmem_slot, C::kTmemCols);
+    tmem_relinquish();
+  }
+  if (warp == 0 && lane == 0) tma_prefetch_desc(&xmap);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    // ---------------------------------------------------------- producer
+    if (lane == 0) {
+      const uint8_t* wsrc = a.wt + ((size_t)wtile * a.kc_total + kc0) * kChunkBytes;
+      int issued = 0;
+      for (int i = 0; i < nk; ++i) {
+        const int s = i % STAGES;
+        if (i >= STAGES && !mbar_wait(&empty[s], ((i / STAGES) - 1) & 1, abort_flag, err, 1)) break;
+        mbar_arrive_expect_tx(&full[s], kChunkBytes + C::kXStageBytes);
+        bulk_load(wsm + s * kChunkBytes, wsrc + (size_t)i * kChunkBytes, kChunkBytes, &full[s]);
+        tma_load_2d(xs + s * C::kXStageBytes, &xmap, (kc0 + i) * kChunkK, xtile * BN, &full[s]);
+        ++issued;
+      }
+      // no copy into this CTA's shared memory may outlive it
+      for (int i = max(0, issued - STAGES); i < issued; ++i) wait_drain(&full[i % STAGES], (i / STAGES) & 1);
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------- MMA issuer
+    if (lane == 0) {
+      const uint32_t idesc = idesc_bf16_f32(kTileRows, BN);
+      for (int i = 0; i < nk; ++i) {
+        const int s = i % STAGES;
+        if (!mbar_wait(&afull[s], (i / STAGES) & 1, abort_flag, err, 2)) break;
+        tc_fence_after();
+        const uint32_t a_base = tmem + C::kAColBase + 32 * s;
+        const uint64_t b_base = smem_desc_sw128(smem_u32(xs + s * C::kXStageBytes));
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk)
+          mma_bf16_ts(tmem, a_base + 8 * kk, b_base + 2 * kk, idesc, (i | kk) != 0 ? 1u : 0u);
+        mma_commit(&empty[s]);
+      }
+      mma_commit(accum);  // fires once every MMA issued above has completed
+    }
+  } else if (warp >= 4) {
+    // ------------------------------------------- dequant, then epilogue
+    const int q = warp & 3;
+    const int row = 32 * q + lane;                // tile row == TMEM lane
+    const uint32_t lane_addr = (uint32_t)(32 * q) << 16;
+    for (int i = 0; i < nk; ++i) {
+      const int s = i % STAGES;
+      const bool ok = mbar_wait(&full[s], (i / STAGES) & 1, abort_flag, err, 4);
+      if (!__all_sync(0xffffffffu, ok)) break;  // keep the warp converged for tcgen05.st
+      const uint8_t* w = wsm + s * kChunkBytes;
+      const uint4 lo = *reinterpret_cast<const uint4*>(w + 16 * row);
+      const uint4 hi = *reinterpret_cast<const uint4*>(w + 2048 + 16 * row);
+      const uint32_t sc = *reinterpret_cast<const uint32_t*>(w + 4096 + 4 * row);
+      uint32_t v[32];
+      dequant64(lo, hi, sc, v);
+      tmem_st32(tmem + lane_addr + C::kAColBase + 32 * s, v);
+      tmem_st_wait();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&afull[s]);
+    }
+    const bool done = __all_sync(0xffffffffu, wait_drain(accum, 0));
+    tc_fence_after();
+    if (done && !*abort_flag) {
+      const int rbase = xtile * BN;
+      const int nchunks = (BN + 31) / 32;
+      const int et = threadIdx.x - 128;  // 0..127 within the epilogue warps
+      for (int c = 0; c < nchunks; ++c) {
+        const int r0 = rbase + 32 * c;
+        if (r0 >= a.m) break;
+        const int jmax = min(32, BN - 32 * c);
+        uint32_t v[32];
+        tmem_ld32(tmem + lane_addr + 32 * c, v);
+        tmem_ld_wait();
+        if (EPI == kEpiPartial) {
+          float* P = static_cast<float*>(a.out) + (size_t)blockIdx.z * a.m * a.n_pad;
+          const int col = kTileRows * wtile + row;
+#pragma unroll
+          for (int j = 0; j < 32; ++j)
+            if (j < jmax && r0 + j < a.m) P[(size_t)(r0 + j) * a.n_pad + col] = __uint_as_float(v[j]);
+        } else if (EPI == kEpiStore) {
+          uint16_t* T = reinterpret_cast<uint16_t*>(epi);  // [32][128] bf16
+          const float gs = a.gs[0];
+#pragma unroll
+          for (int j = 0; j < 32; ++j) T[j * 128 + row] = f32_to_bf16_bits(gs * __uint_as_float(v[j]));
+          named_bar_sync(1, 128);
+          const int n0 = kTileRows * wtile;
+          for (int idx = et; idx < 32 * 16; idx += 128) {
+            const int j = idx >> 4, ch = idx & 15;
+            const int r = r0 + j, n = n0 + 8 * ch;
+            if (j < jmax && r < a.m && n < a.n_out)
+              *reinterpret_cast<uint4*>(static_cast<uint16_t*>(a.out) + (size_t)r * a.ldo + n) =
+                  *reinterpret_cast<const uint4*>(T + j * 128 + 8 * ch);
+          }
+          named_bar_sync(1, 128);
+        } else {  // kEpiSiluMul: rows 0-63 gate, 64-127 the matching up rows
+          float* U = reinterpret_cast<float*>(epi);                  // [32][64] fp32
+          uint16_t* Hs = reinterpret_cast<uint16_t*>(epi + 8192);    // [32][64] bf16
+          if (q >= 2) {
+            const float gsu = a.gs[1];
+#pragma unroll
+            for (int j = 0; j < 32; ++j) U[j * 64 + (row - 64)] = bf16_round(gsu * __uint_as_float(v[j]));
+          }
+          named_bar_sync(1, 128);
+          if (q < 2) {
+            const float gsg = a.gs[0];
+#pragma unroll
+            for (int j = 0; j < 32; ++j) {
+              const float g = bf16_round(gsg * __uint_as_float(v[j]));
+              Hs[j * 64 + row] = f32_to_bf16_bits(silu_f32(g) * U[j * 64 + row]);
+            }
+          }
+          named_bar_sync(1, 128);
+          const int n0 = 64 * wtile;
+          for (int idx = et; idx < 32 * 8; idx += 128) {
+            const int j = idx >> 3, ch = idx & 7;
+            const int r = r0 + j, n = n0 + 8 * ch;
+            if (j < jmax && r < a.m && n < a.n_out)
+              *reinterpret_cast<uint4*>(static_cast<uint16_t*>(a.out) + (size_t)r * a.ldo + n) =
+                  *reinterpret_cast<const uint4*>(Hs + j * 64 + 8 * ch);
+          }
+          named_bar_sync(1, 128);
+        }
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 2) {
+    tc_fence_after();
+    tmem_dealloc(tmem, C::kTmemCols);
+  }
+}
+
+// Split-K reduction in a fixed order (z = 0, 1, ...), then the epilogue.
+template <bool kGateUp>
+__global__ void splitk_reduce_kernel(const float* __restrict__ P, int splits, int m, int n_pad,
+                                     int n_out, const float* __restrict__ gs,
+                                     uint16_t* __restrict__ out, int ldo) {
+  const int64_t idx = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;
+  if (idx >= (int64_t)m * n_out) return;
+  const int r = (int)(idx / n_out), n = (int)(idx % n_out);
+  const size_t plane = (size_t)m * n_pad;
+  if (kGateUp) {
+    const int gcol = kTileRows * (n / 64) + (n % 64), ucol = gcol + 64;
+    float g = 0.0f, u = 0.0f;
+    for (int z = 0; z < splits; ++z) {
+      g += P[z * plane + (size_t)r * n_pad + gcol];
+      u += P[z * plane + (size_t)r * n_pad + ucol];
+    }
+    const float gb = bf16_round(gs[0] * g), ub = bf16_round(gs[1] * u);
+    out[(size_t)r * ldo + n] = f32_to_bf16_bits(silu_f32(gb) * ub);
+  } else {
+    float acc = 0.0f;
+    for (int z = 0; z < splits; ++z) acc += P[z * plane + (size_t)r * n_pad + n];
+    out[(size_t)r * ldo + n] = f32_to_bf16_bits(gs[0] * acc);
+  }
+}
+
+// Re-tile a canonical NVFP4 weight (codes [n, k/2], scales [n, k/16]) into the
+// per-(128-row tile, 64-element chunk) layout the kernel streams.  For a fused
+// gate+up weight (half = inter), tile t holds gate rows [64t, 64t+64) followed
+// by the up rows with the same indices.  Padding rows / K tails are zero.
+__global__ void tile_weight_kernel(const uint8_t* __restrict__ codes,
+                                   const uint8_t* __restrict__ scales, int64_t nrows, int64_t k,
+                                   int64_t half, int ntiles, int kc, uint8_t* __restrict__ out) {
+  const int64_t idx = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;
+  if (idx >= (int64_t)ntiles * kc * kTileRows) return;
+  const int r = (int)(idx % kTileRows);
+  const int64_t tj = idx / kTileRows;
+  const int j = (int)(tj % kc);
+  const int t = (int)(tj / kc);
+  int64_t src;
+  bool valid;
+  if (half > 0) {
+    const int64_t i = 64 * (int64_t)t + (r & 63);
+    src = r < 64 ? i : half + i;
+    valid = i < half;
+  } else {
+    src = (int64_t)kTileRows * t + r;
+    valid = src < nrows;
+  }
+  uint4 lo = make_uint4(0, 0, 0, 0), hi = lo;
+  uint32_t sc = 0;
+  if (valid) {
+    const int64_t cb = k / 2, sb = k / 16;
+    const uint8_t* crow = codes + src * cb;
+    const uint8_t* srow = scales + src * sb;
+    const int64_t off = 32 * (int64_t)j;
+    if (off + 16 <= cb) lo = *reinterpret_cast<const uint4*>(crow + off);
+    if (off + 32 <= cb) hi = *reinterpret_cast<const uint4*>(crow + off + 16);
+    for (int b = 0; b < 4; ++b)
+      if (4 * (int64_t)j + b < sb) sc |= (uint32_t)srow[4 * j + b] << (8 * b);
+  }
+  uint8_t* base = out + ((int64_t)t * kc + j) * kChunkBytes;
+  *reinterpret_cast<uint4*>(base + 16 * r) = lo;
+  *reinterpret_cast<uint4*>(base + 2048 + 16 * r) = hi;
+  *reinterpret_cast<uint32_t*>(base + 4096 + 4 * r) = sc;
+}
+
+// ----------------------------------------------------------------- host side
+
+PFN_cuTensorMapEncodeTiled_v12000 get_encode() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+// 2-D map over X [m, k] bf16 with a 64 x box_rows box and the 128-byte swizzle.
+bool make_x_map(CUtensorMap* map, const void* x, int64_t m, int64_t k, int box_rows) {
+  auto enc = get_encode();
+  if (!enc) return false;
+  cuuint64_t dims[2] = {(cuuint64_t)k, (cuuint64_t)m};
+  cuuint64_t strides[1] = {(cuuint64_t)k * 2};
+  cuuint32_t box[2] = {(cuuint32_t)kChunkK, (cuuint32_t)box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(x), dims, strides, box,
+             estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int BN, int STAGES, int EPI>
+cudaError_t launch_cfg(const CUtensorMap& map, const TcArgs& a, dim3 grid, cudaStream_t s) {
+  using C = TcCfg<BN, STAGES>;
+  auto kern = tc_w4a16_kernel<BN, STAGES, EPI>;
+  static bool attr_set = false;  // per instantiation; idempotent if raced
+  if (!attr_set) {
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemAlloc);
+    if (e != cudaSuccess) return e;
+    attr_set = true;
+  }
+  kern<<<grid, 256, C::kSmemAlloc, s>>>(map, a);
+  return cudaGetLastError();
+}
+
+template <int EPI>
+cudaError_t launch_bn(int bn, const CUtensorMap& map, const TcArgs& a, dim3 grid, cudaStream_t s) {
+  switch (bn) {
+    case 16: return launch_cfg<16, 7, EPI>(map, a, grid, s);
+    case 32: return launch_cfg<32, 7, EPI>(map, a, grid, s);
+    case 64: return launch_cfg<64, 6, EPI>(map, a, grid, s);
+    case 128: return launch_cfg<128, 6, EPI>(map, a, grid, s);
+    default: return launch_cfg<256, 5, EPI>(map, a, grid, s);
+  }
+}
+
+}  // namespace
+
+int tc_tile_bytes_per_row_chunk() { return kChunkBytes; }
+
+int64_t tc_tiled_bytes(int64_t n, int64_t k, bool gate_up) {
+  const int64_t tiles = gate_up ? (n / 2 + 63) / 64 : (n + kTileRows - 1) / kTileRows;
+  const int64_t kc = (k + kChunkK - 1) / kChunkK;
+  return tiles * kc * kChunkBytes;
+}
+
+cudaError_t launch_tile_weight(const uint8_t* codes, const uint8_t* scales, int64_t n, int64_t k,
+                               bool gate_up, uint8_t* out, cudaStream_t s) {
+  const int64_t half = gate_up ? n / 2 : 0;
+  const int ntiles = (int)(gate_up ? (half + 63) / 64 : (n + kTileRows - 1) / kTileRows);
+  const int kc = (int)((k + kChunkK - 1) / kChunkK);
+  const int64_t total = (int64_t)ntiles * kc * kTileRows;
+  tile_weight_kernel<<<(unsigned)((total + 255) / 256), 256, 0, s>>>(codes, scales, n, k, half, ntiles,
+                                                                   kc, out);
+  return cudaGetLastError();
+}
+
+TcPlan plan_tc(int64_t m, int64_t n, int64_t k, bool gate_up, int num_sms) {
+  TcPlan p;
+  p.bn = m <= 16 ? 16 : m <= 32 ? 32 : m <= 64 ? 64 : m <= 128 ? 128 : 256;
+  p.xtiles = (int)((m + p.bn - 1) / p.bn);
+  p.wtiles = (int)(gate_up ? (n / 2 + 63) / 64 : (n + kTileRows - 1) / kTileRows);
+  p.kc = (int)((k + kChunkK - 1) / kChunkK);
+  p.n_pad = p.wtiles * kTileRows;
+  const int ctas_per_sm = p.bn <= 64 ? 2 : 1;
+  const int64_t slots = (int64_t)num_sms * ctas_per_sm;
+  const int64_t ctas = (int64_t)p.xtiles * p.wtiles;
+  int splits = 1;
+  if (ctas < slots) {
+    splits = (int)(slots / ctas);
+    const int max_splits = p.kc / 8 > 1 ? p.kc / 8 : 1;  // keep >= 8 chunks per split
+    if (splits > max_splits) splits = max_splits;
+  }
+  p.kc_per_split = (p.kc + splits - 1) / splits;
+  p.splits = (p.kc + p.kc_per_split - 1) / p.kc_per_split;
+  p.partial_bytes = p.splits > 1 ? (size_t)p.splits * m * p.n_pad * sizeof(float) : 0;
+  return p;
+}
+
+cudaError_t launch_tc_w4a16(const void* x, int64_t m, const TcWeight& w, bool silu_mul,
+                            const TcPlan& p, void* y, void* partials, cudaStream_t s) {
+  CUtensorMap map;
+  if (!make_x_map(&map, x, m, w.k, p.bn)) return cudaErrorInvalidValue;
+  TcArgs a;
+  a.wt = w.tiled;
+  a.gs = w.gs;
+  a.m = (int)m;
+  a.n_out = (int)(silu_mul ? w.n / 2 : w.n);
+  a.ldo = a.n_out;
+  a.kc_total = p.kc;
+  a.kc_per_split = p.kc_per_split;
+  a.n_pad = p.n_pad;
+  const dim3 grid(p.xtiles, p.wtiles, p.splits);
+  cudaError_t e;
+  if (p.splits > 1) {
+    a.out = partials;
+    {
+      ProfScope prof(s, silu_mul ? "tc_w4a16_gate_up_partial" : "tc_w4a16_partial");
+      e = launch_bn<kEpiPartial>(p.bn, map, a, grid, s);
+    }
+    if (e != cudaSuccess) return e;
+    const int64_t total = m * a.n_out;
+    ProfScope prof(s, silu_mul ? "splitk_reduce_silu_mul" : "splitk_reduce");
+    if (silu_mul)
+      splitk_reduce_kernel<true><<<(unsigned)((total + 255) / 256), 256, 0, s>>>(
+          (const float*)partials, p.splits, (int)m, p.n_pad, a.n_out, w.gs, (uint16_t*)y, a.ldo);
+    else
+      splitk_reduce_kernel<false><<<(unsigned)((total + 255) / 256), 256, 0, s>>>(
+          (const float*)partials, p.splits, (int)m, p.n_pad, a.n_out, w.gs, (uint16_t*)y, a.ldo);
+    return cudaGetLastError();
+  }
+  a.out = y;
+  ProfScope prof(s, silu_mul ? "tc_w4a16_gate_up_silu" : "tc_w4a16");
+  return silu_mul ? launch_bn<kEpiSiluMul>(p.bn, map, a, grid, s)
+                  : launch_bn<kEpiStore>(p.bn, map, a, grid, s);
+}
+
+cudaError_t read_device_error(int* flags, bool clear) {
+  cudaError_t e = cudaMemcpyFromSymbol(flags, g_ffn_device_error, sizeof(int));
+  if (e == cudaSuccess && clear) {
+    const int zero = 0;
+    e = cudaMemcpyToSymbol(g_ffn_device_error, &zero, sizeof(int));
+  }
+  return e;
+}
+
+}  // namespace ffn

@@ -57,6 +57,7 @@ def _load() -> ctypes.CDLL:
         "ffn_nvfp4_linear_workspace_size": (ctypes.c_int, [i64, i64, i64, ctypes.c_int, P(sz)]),
         "ffn_nvfp4_linear": (ctypes.c_int, [vp, i64, vp, ctypes.c_int, vp, vp, sz, vp]),
         "ffn_nvfp4_profile_begin": (ctypes.c_int, []),
+        "ffn_nvfp4_device_error": (ctypes.c_int, [P(ctypes.c_int), ctypes.c_int]),
         "ffn_nvfp4_profile_end": (ctypes.c_int, [P(KernelTime), ctypes.c_int, P(ctypes.c_int)]),
     }
     for name, (res, args) in sig.items():
@@ -220,8 +221,6 @@ def ffn_nvfp4_forward(x: torch.Tensor, gate_up: Weight, down: Weight, fmt="bf16"
     _need(x, "x", torch.bfloat16)
     m, hidden = x.shape
     inter = down.k
-    if gate_up.k != hidden:
-        raise ValueError(f"x has {hidden} columns, gate_up expects {gate_up.k}")
     out = torch.empty((m, hidden), dtype=torch.bfloat16, device=x.device) if out is None else out
     _need(out, "out", torch.bfloat16, (m, hidden))
     nbytes = ffn_nvfp4_workspace_size(m, hidden, inter, fmt)
@@ -261,3 +260,10 @@ def ffn_nvfp4_profile_end() -> dict:
     n = ctypes.c_int()
     _check("ffn_nvfp4_profile_end", lib.ffn_nvfp4_profile_end(arr, cap, ctypes.byref(n)))
     return {arr[i].name.decode(): (arr[i].launches, arr[i].total_ms) for i in range(n.value)}
+
+
+def ffn_nvfp4_device_error(clear: bool = True) -> int:
+    """Device-side error bits of kernels whose bounded waits gave up (0 = none)."""
+    v = ctypes.c_int()
+    _check("ffn_nvfp4_device_error", lib.ffn_nvfp4_device_error(ctypes.byref(v), int(clear)))
+    return v.value

@@ -178,3 +178,37 @@ def test_errors_are_reported_not_raised_on_device(native, tiny):
     assert e.value.status_name == "FFN_ERR_ALIGNMENT"
     # the context is still usable
     assert_close(bf16_to_f64(tiny.forward("bf16")), tiny.oracle("bf16"))
+
+
+@pytest.mark.parametrize("m,H,I", [(33, 1056, 800), (300, 512, 96), (257, 256, 2048), (1, 4096, 1056)])
+def test_ffn_tile_edges(native, m, H, I):
+    # K % 64 == 32 (1056), inter % 64 == 32 (800, 96: partial gate+up tiles),
+    # several 256-row activation tiles with a ragged last one, deep split-K.
+    inp = synth.make_inputs("smallm", m=m, hidden=H, inter=I, seed=40 + m)
+    case = FfnCase(native, inp)
+    assert_close(bf16_to_f64(case.forward("bf16")), case.oracle("bf16"), f"m={m} H={H} I={I}")
+    assert native.ffn_nvfp4_device_error() == 0
+
+
+def test_gemv_path_matches_oracle_in_subprocess(native):
+    # the CUDA-core projection family, selected per process by environment
+    import os
+    import subprocess
+    import sys
+    code = (
+        "import sys; sys.path.insert(0, 'tests'); sys.path.insert(0, '.');"
+        "from gpu_helpers import FfnCase, assert_close, bf16_to_f64;"
+        "from nvfp4_quantized_dense_w4a16_b200 import native as N, synth;"
+        "c = FfnCase(N, synth.make_inputs('smallm', m=5, hidden=512, inter=1536, seed=3));"
+        "assert_close(bf16_to_f64(c.forward('bf16')), c.oracle('bf16'));"
+        "print('gemv-ok')")
+    env = dict(os.environ, FFN_NVFP4_W4A16_PATH="gemv")
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    r = subprocess.run([sys.executable, "-c", code], cwd=root, env=env, capture_output=True, text=True,
+                       timeout=600)
+    assert r.returncode == 0 and "gemv-ok" in r.stdout, r.stdout + r.stderr
+
+
+def test_device_error_word_is_clear(native, tiny):
+    tiny.forward("bf16")
+    assert native.ffn_nvfp4_device_error(clear=False) == 0
