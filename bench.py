@@ -44,6 +44,22 @@ WORKLOADS = {
 }
 
 
+def max_over_ranks(value: float, dist, device) -> float:
+    """Max of a per-rank scalar (a time) over all ranks; identity without a group."""
+    if dist is None:
+        return value
+    import torch
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def aggregate_throughput(units_per_step: float, steps: int, max_ms: float, world: int) -> float:
+    """Whole-job throughput: every rank did `steps` steps of `units_per_step`
+    units; the job took the slowest rank's time."""
+    return world * units_per_step * steps / (max_ms * 1e-3)
+
+
 def load_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -192,14 +208,10 @@ def run_ours(args, rank, world, dist):
     barrier()
     prof = N.ffn_nvfp4_profile_end()
     clk = clocks.stop()
-    ms = sum(a.elapsed_time(b) for a, b in zip(starts, stops))
-    if dist is not None:
-        t = torch.tensor([ms], dtype=torch.float64, device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = max_over_ranks(sum(a.elapsed_time(b) for a, b in zip(starts, stops)), dist, "cuda")
     ms_step = ms / args.steps
     flops = ffn_flops(wl.m, wl.H, wl.I)
-    value = world * flops * args.steps / (ms * 1e-3) / 1e12
+    value = aggregate_throughput(flops, args.steps, ms, world) / 1e12
 
     # dominant kernel and its roofline
     roof = None
@@ -240,12 +252,8 @@ def run_ours(args, rank, world, dist):
         out_host.copy_(wl.out, non_blocking=True)
     e1.record()
     barrier()
-    e2e_ms = e0.elapsed_time(e1)
-    if dist is not None:
-        t = torch.tensor([e2e_ms], dtype=torch.float64, device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
-    e2e = {"value": round(world * flops * e2e_steps / (e2e_ms * 1e-3) / 1e12, 3), "unit": "TFLOP/s",
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1), dist, "cuda")
+    e2e = {"value": round(aggregate_throughput(flops, e2e_steps, e2e_ms, world) / 1e12, 3), "unit": "TFLOP/s",
            "h2d_bytes_per_step": wl.m * wl.H * 2, "d2h_bytes_per_step": wl.m * wl.H * 2,
            "ms_per_step": round(e2e_ms / e2e_steps, 4)}
 
