@@ -171,6 +171,26 @@ ffn_status ffn_nvfp4_linear(const void* x, int64_t m, const ffn_nvfp4_weight* w,
                             ffn_act_format format, void* y, void* workspace,
                             size_t workspace_bytes, void* stream);
 
+/* Allocation-free variant of ffn_nvfp4_linear for bf16 activations (W4A16),
+ * for callers that cannot allocate device memory on the call path: for
+ * example a plugin whose host framework owns every device allocation and
+ * passes it no workspace, or serving code that must not call cudaMalloc once
+ * running (cudaMalloc can synchronise the whole device).  The source pages
+ * have no counterpart; this entry point exists only for such callers.
+ *   x [m, k] bf16, w a plain (not gate+up) handle of shape [n, k],
+ *   y [m, n] bf16 = bf16(gs * x @ w^T), the same kernels as ffn_nvfp4_linear.
+ * The split-K partial sums live in one fixed 16 MiB device array that every
+ * GPU loading the library holds until the process exits; a shape whose
+ * partials would need more returns FFN_ERR_WORKSPACE (nothing launched).  It
+ * calls no cudaMalloc, cudaFree or allocating library routine.  The first
+ * call on each device looks up that device's address of the array (with the
+ * device current), so make that first call before any stream capture.  All
+ * calls share the array: calls that overlap on the GPU (other streams, other
+ * threads) race and must be serialised by the caller.  Every partial a call
+ * reads is written earlier in the same call, so nothing needs clearing. */
+ffn_status ffn_nvfp4_linear_noalloc(const void* x, int64_t m, const ffn_nvfp4_weight* w,
+                                    void* y, void* stream);
+
 /* Device-side error bits.  Kernels that wait on asynchronous copies or on
  * tensor-core completion give up after about two seconds instead of hanging,
  * free their tensor memory, skip their stores and OR a bit into a device-wide

@@ -142,6 +142,11 @@ void free_weight(ffn_nvfp4_weight* w) {
 
 }  // namespace
 
+void ffn::handle_tc_view(const ffn_nvfp4_weight* w, ffn::TcWeight* out, bool* gate_up) {
+  *out = w->tc();
+  *gate_up = w->gate_up != 0;
+}
+
 extern "C" {
 
 const char* ffn_status_string(ffn_status s) {

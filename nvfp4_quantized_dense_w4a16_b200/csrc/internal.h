@@ -4,6 +4,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include "ffn_nvfp4.h"
+
 namespace ffn {
 
 // Operand of one projection: canonical NVFP4 layout of a [n, k] weight.
@@ -40,6 +42,9 @@ cudaError_t launch_tile_weight(const uint8_t* codes, const uint8_t* scales, int6
                                bool gate_up, uint8_t* out, cudaStream_t s);
 cudaError_t launch_tc_w4a16(const void* x, int64_t m, const TcWeight& w, bool silu_mul,
                             const TcPlan& p, void* y, void* partials, cudaStream_t s);
+// Tensor-core view of a handle (and whether it is a fused gate+up handle).
+void handle_tc_view(const ffn_nvfp4_weight* w, TcWeight* out, bool* gate_up);
+
 // Device-wide error bits set by kernels whose bounded waits gave up.
 cudaError_t read_device_error(int* flags, bool clear);
 

@@ -56,6 +56,7 @@ def _load() -> ctypes.CDLL:
         "ffn_nvfp4_forward": (ctypes.c_int, [vp, i64, i64, i64, vp, vp, ctypes.c_int, vp, vp, sz, vp]),
         "ffn_nvfp4_linear_workspace_size": (ctypes.c_int, [i64, i64, i64, ctypes.c_int, P(sz)]),
         "ffn_nvfp4_linear": (ctypes.c_int, [vp, i64, vp, ctypes.c_int, vp, vp, sz, vp]),
+        "ffn_nvfp4_linear_noalloc": (ctypes.c_int, [vp, i64, vp, vp, vp]),
         "ffn_nvfp4_profile_begin": (ctypes.c_int, []),
         "ffn_nvfp4_device_error": (ctypes.c_int, [P(ctypes.c_int), ctypes.c_int]),
         "ffn_nvfp4_profile_end": (ctypes.c_int, [P(KernelTime), ctypes.c_int, P(ctypes.c_int)]),
@@ -267,3 +268,17 @@ def ffn_nvfp4_device_error(clear: bool = True) -> int:
     v = ctypes.c_int()
     _check("ffn_nvfp4_device_error", lib.ffn_nvfp4_device_error(ctypes.byref(v), int(clear)))
     return v.value
+
+
+def ffn_nvfp4_linear_noalloc(x: torch.Tensor, w: Weight, y=None, stream=None) -> torch.Tensor:
+    """bf16 projection through the allocation-free entry point (fixed device
+    scratch inside the library; concurrent calls must be serialised)."""
+    _need(x, "x", torch.bfloat16)
+    m, k = x.shape
+    if k != w.k:
+        raise ValueError(f"x has {k} columns, the weight expects {w.k}")
+    y = torch.empty((m, w.n), dtype=torch.bfloat16, device=x.device) if y is None else y
+    _need(y, "y", torch.bfloat16, (m, w.n))
+    _check("ffn_nvfp4_linear_noalloc", lib.ffn_nvfp4_linear_noalloc(
+        _ptr(x), m, w.handle, _ptr(y), _stream(stream)))
+    return y
