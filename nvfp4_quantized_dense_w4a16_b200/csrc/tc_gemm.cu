@@ -45,21 +45,31 @@ constexpr int kChunkBytes = 4608;  // 128 x (16 + 16 + 4) bytes
 
 enum : int { kEpiStore = 0, kEpiSiluMul = 1, kEpiPartial = 2 };
 
-template <int BN, int STAGES>
+// Pipeline shape: activation ring of SX stages (released when the MMA that
+// read it completes), weight ring of SW stages (released as soon as the
+// dequant warps have read it), SA tensor-memory stages for the dequantised
+// weights, DQG dequant warpgroups (each dequantises 64 / DQG elements of every
+// row of a chunk).
+template <int BN, int SX, int SW, int SA, int DQG>
 struct TcCfg {
+  static constexpr int kThreads = 128 + 128 * DQG;
   static constexpr int kXStageBytes = BN * 128;
   static constexpr int kAColBase = BN < 32 ? 32 : BN;  // TMEM column of A stage 0
-  static constexpr int kTmemNeed = kAColBase + 32 * STAGES;
+  static constexpr int kTmemNeed = kAColBase + 32 * SA;
   static constexpr int kTmemCols = kTmemNeed <= 64 ? 64 : kTmemNeed <= 128 ? 128 : kTmemNeed <= 256 ? 256 : 512;
-  static constexpr int kEpiBytes = 16384;
-  static constexpr int kSmemW = STAGES * kXStageBytes;
-  static constexpr int kSmemEpi = kSmemW + STAGES * kChunkBytes;
-  static constexpr int kSmemBar = kSmemEpi + kEpiBytes;
-  static constexpr int kSmemBytes = kSmemBar + (3 * STAGES + 1) * 8 + 16;
+  static constexpr int kEpiBytes = 16384;  // per dequant warpgroup
+  static constexpr int kSmemW = SX * kXStageBytes;
+  static constexpr int kSmemEpi = kSmemW + SW * kChunkBytes;
+  static constexpr int kSmemBar = kSmemEpi + DQG * kEpiBytes;
+  static constexpr int kNumBars = 2 * SX + 2 * SW + 2 * SA + 1;
+  static constexpr int kSmemBytes = kSmemBar + kNumBars * 8 + 16;
   static constexpr int kSmemAlloc = kSmemBytes + 1024;  // slack for 1024-byte alignment
+  // two CTAs per SM when both fit (228 KB of shared memory, 512 TMEM columns)
+  static constexpr int kMinBlocks = (2 * (kSmemAlloc + 1024) <= 233472 && kTmemCols <= 256) ? 2 : 1;
   static_assert(kTmemNeed <= 512, "TMEM budget");
   static_assert(kSmemAlloc <= 232448, "shared memory budget");
   static_assert(BN % 16 == 0 && BN >= 16 && BN <= 256, "MMA N");
+  static_assert(DQG == 1 || DQG == 2, "dequant warpgroups");
 };
 
 struct TcArgs {
@@ -117,6 +127,21 @@ __device__ __forceinline__ void dequant64(const uint4 lo, const uint4 hi, uint32
   dequant8(hi.w, s3, v + 28);
 }
 
+// Half a chunk (32 elements: 16 bytes of codes, two block scales) -> 16 columns.
+__device__ __forceinline__ void dequant32(const uint4 c, uint32_t sc2, uint32_t (&v)[16]) {
+  const uint32_t s0 = scale_pair(sc2 & 0xffu), s1 = scale_pair((sc2 >> 8) & 0xffu);
+  dequant8(c.x, s0, v + 0);
+  dequant8(c.y, s0, v + 4);
+  dequant8(c.z, s1, v + 8);
+  dequant8(c.w, s1, v + 12);
+}
+
+// SiLU with the fast exponential and division (a few ulp in fp32; the result
+// is rounded to bf16 right after).
+__device__ __forceinline__ float silu_fast(float z) {
+  return z < -88.0f ? 0.0f * z : __fdividef(z, 1.0f + __expf(-z));
+}
+
 // Bounded wait that ignores the abort flag (used to drain in-flight work).
 __device__ __forceinline__ bool wait_drain(uint64_t* bar, uint32_t parity) {
   const long long t0 = clock64();
@@ -129,23 +154,28 @@ __device__ __forceinline__ bool wait_drain(uint64_t* bar, uint32_t parity) {
   return true;
 }
 
-template <int BN, int STAGES, int EPI>
-__global__ void __launch_bounds__(256, (BN <= 64 ? 2 : 1))
+template <int BN, int SX, int SW, int SA, int DQG, int EPI>
+__global__ void __launch_bounds__(TcCfg<BN, SX, SW, SA, DQG>::kThreads,
+                                  TcCfg<BN, SX, SW, SA, DQG>::kMinBlocks)
 tc_w4a16_kernel(const __grid_constant__ CUtensorMap xmap, const TcArgs a) {
-  using C = TcCfg<BN, STAGES>;
+  using C = TcCfg<BN, SX, SW, SA, DQG>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
   uint8_t* xs = smem;
   uint8_t* wsm = smem + C::kSmemW;
   uint8_t* epi = smem + C::kSmemEpi;
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::kSmemBar);
-  uint64_t* empty = full + STAGES;
-  uint64_t* afull = empty + STAGES;
-  uint64_t* accum = afull + STAGES;
+  uint64_t* xfull = reinterpret_cast<uint64_t*>(smem + C::kSmemBar);
+  uint64_t* xempty = xfull + SX;
+  uint64_t* wfull = xempty + SX;
+  uint64_t* wempty = wfull + SW;
+  uint64_t* afull = wempty + SW;
+  uint64_t* aempty = afull + SA;
+  uint64_t* accum = aempty + SA;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(accum + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   int* err = &g_ffn_device_error;
+  constexpr int kDqWarps = 4 * DQG;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int xtile = blockIdx.x, wtile = blockIdx.y;
@@ -153,10 +183,17 @@ tc_w4a16_kernel(const __grid_constant__ CUtensorMap xmap, const TcArgs a) {
   const int nk = min(a.kc_total, kc0 + a.kc_per_split) - kc0;
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < STAGES; ++s) {
-      mbar_init(&full[s], 1);
-      mbar_init(&empty[s], 1);
-      mbar_init(&afull[s], 4);
+    for (int s = 0; s < SX; ++s) {
+      mbar_init(&xfull[s], 1);
+      mbar_init(&xempty[s], 1);
+    }
+    for (int s = 0; s < SW; ++s) {
+      mbar_init(&wfull[s], 1);
+      mbar_init(&wempty[s], kDqWarps);
+    }
+    for (int s = 0; s < SA; ++s) {
+      mbar_init(&afull[s], kDqWarps);
+      mbar_init(&aempty[s], 1);
     }
     mbar_init(accum, 1);
     *abort_flag = 0;
@@ -166,73 +203,106 @@ tc_w4a16_kernel(const __grid_constant__ CUtensorMap xmap, const TcArgs a) {
     tmem_alloc(tmem_slot, C::kTmemCols);
     tmem_relinquish();
   }
-  if (warp == 0 && lane == 0) tma_prefetch_desc(&xmap);
+  if (warp == 3 && lane == 0) tma_prefetch_desc(&xmap);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
   if (warp == 0) {
-    // ---------------------------------------------------------- producer
+    // ------------------------------------------------- weight producer
     if (lane == 0) {
       const uint8_t* wsrc = a.wt + ((size_t)wtile * a.kc_total + kc0) * kChunkBytes;
       int issued = 0;
       for (int i = 0; i < nk; ++i) {
-        const int s = i % STAGES;
-        if (i >= STAGES && !mbar_wait(&empty[s], ((i / STAGES) - 1) & 1, abort_flag, err, 1)) break;
-        mbar_arrive_expect_tx(&full[s], kChunkBytes + C::kXStageBytes);
-        bulk_load(wsm + s * kChunkBytes, wsrc + (size_t)i * kChunkBytes, kChunkBytes, &full[s]);
-        tma_load_2d(xs + s * C::kXStageBytes, &xmap, (kc0 + i) * kChunkK, xtile * BN, &full[s]);
+        const int s = i % SW;
+        if (i >= SW && !mbar_wait(&wempty[s], ((i / SW) - 1) & 1, abort_flag, err, 1)) break;
+        mbar_arrive_expect_tx(&wfull[s], kChunkBytes);
+        bulk_load(wsm + s * kChunkBytes, wsrc + (size_t)i * kChunkBytes, kChunkBytes, &wfull[s]);
         ++issued;
       }
       // no copy into this CTA's shared memory may outlive it
-      for (int i = max(0, issued - STAGES); i < issued; ++i) wait_drain(&full[i % STAGES], (i / STAGES) & 1);
+      for (int i = max(0, issued - SW); i < issued; ++i) wait_drain(&wfull[i % SW], (i / SW) & 1);
+    }
+  } else if (warp == 3) {
+    // --------------------------------------------- activation producer
+    if (lane == 0) {
+      int issued = 0;
+      for (int i = 0; i < nk; ++i) {
+        const int s = i % SX;
+        if (i >= SX && !mbar_wait(&xempty[s], ((i / SX) - 1) & 1, abort_flag, err, 1)) break;
+        mbar_arrive_expect_tx(&xfull[s], C::kXStageBytes);
+        tma_load_2d(xs + s * C::kXStageBytes, &xmap, (kc0 + i) * kChunkK, xtile * BN, &xfull[s]);
+        ++issued;
+      }
+      for (int i = max(0, issued - SX); i < issued; ++i) wait_drain(&xfull[i % SX], (i / SX) & 1);
     }
   } else if (warp == 1) {
     // ------------------------------------------------------- MMA issuer
     if (lane == 0) {
       const uint32_t idesc = idesc_bf16_f32(kTileRows, BN);
       for (int i = 0; i < nk; ++i) {
-        const int s = i % STAGES;
-        if (!mbar_wait(&afull[s], (i / STAGES) & 1, abort_flag, err, 2)) break;
+        const int sa = i % SA, sx = i % SX;
+        if (!mbar_wait(&afull[sa], (i / SA) & 1, abort_flag, err, 2)) break;
+        if (!mbar_wait(&xfull[sx], (i / SX) & 1, abort_flag, err, 2)) break;
         tc_fence_after();
-        const uint32_t a_base = tmem + C::kAColBase + 32 * s;
-        const uint64_t b_base = smem_desc_sw128(smem_u32(xs + s * C::kXStageBytes));
+        const uint32_t a_base = tmem + C::kAColBase + 32 * sa;
+        const uint64_t b_base = smem_desc_sw128(smem_u32(xs + sx * C::kXStageBytes));
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk)
           mma_bf16_ts(tmem, a_base + 8 * kk, b_base + 2 * kk, idesc, (i | kk) != 0 ? 1u : 0u);
-        mma_commit(&empty[s]);
+        mma_commit(&aempty[sa]);
+        mma_commit(&xempty[sx]);
       }
       mma_commit(accum);  // fires once every MMA issued above has completed
     }
   } else if (warp >= 4) {
     // ------------------------------------------- dequant, then epilogue
-    const int q = warp & 3;
+    const int g = (warp - 4) >> 2;                // dequant warpgroup
+    const int q = warp & 3;                       // TMEM lane quarter
     const int row = 32 * q + lane;                // tile row == TMEM lane
     const uint32_t lane_addr = (uint32_t)(32 * q) << 16;
     for (int i = 0; i < nk; ++i) {
-      const int s = i % STAGES;
-      const bool ok = mbar_wait(&full[s], (i / STAGES) & 1, abort_flag, err, 4);
+      const int s = i % SW, sa = i % SA;
+      bool ok = mbar_wait(&wfull[s], (i / SW) & 1, abort_flag, err, 4);
       if (!__all_sync(0xffffffffu, ok)) break;  // keep the warp converged for tcgen05.st
       const uint8_t* w = wsm + s * kChunkBytes;
-      const uint4 lo = *reinterpret_cast<const uint4*>(w + 16 * row);
-      const uint4 hi = *reinterpret_cast<const uint4*>(w + 2048 + 16 * row);
-      const uint32_t sc = *reinterpret_cast<const uint32_t*>(w + 4096 + 4 * row);
-      uint32_t v[32];
-      dequant64(lo, hi, sc, v);
-      tmem_st32(tmem + lane_addr + C::kAColBase + 32 * s, v);
+      uint32_t v[64 / DQG / 2];
+      if constexpr (DQG == 1) {
+        const uint4 lo = *reinterpret_cast<const uint4*>(w + 16 * row);
+        const uint4 hi = *reinterpret_cast<const uint4*>(w + 2048 + 16 * row);
+        const uint32_t sc = *reinterpret_cast<const uint32_t*>(w + 4096 + 4 * row);
+        dequant64(lo, hi, sc, *reinterpret_cast<uint32_t(*)[32]>(v));
+      } else {
+        const uint4 c = *reinterpret_cast<const uint4*>(w + 2048 * g + 16 * row);
+        const uint32_t sc = *reinterpret_cast<const uint16_t*>(w + 4096 + 4 * row + 2 * g);
+        dequant32(c, sc, *reinterpret_cast<uint32_t(*)[16]>(v));
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&wempty[s]);   // the shared-memory slot may be refilled
+      if (i >= SA) {
+        ok = mbar_wait(&aempty[sa], ((i / SA) - 1) & 1, abort_flag, err, 4);
+        if (!__all_sync(0xffffffffu, ok)) break;
+        tc_fence_after();
+      }
+      const uint32_t taddr = tmem + lane_addr + C::kAColBase + 32 * sa + (64 / DQG / 2) * g;
+      if constexpr (DQG == 1)
+        tmem_st32(taddr, *reinterpret_cast<uint32_t(*)[32]>(v));
+      else
+        tmem_st16(taddr, *reinterpret_cast<uint32_t(*)[16]>(v));
       tmem_st_wait();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&afull[s]);
+      if (lane == 0) mbar_arrive(&afull[sa]);
     }
     const bool done = __all_sync(0xffffffffu, wait_drain(accum, 0));
     tc_fence_after();
     if (done && !*abort_flag) {
       const int rbase = xtile * BN;
       const int nchunks = (BN + 31) / 32;
-      const int et = threadIdx.x - 128;  // 0..127 within the epilogue warps
-      for (int c = 0; c < nchunks; ++c) {
+      const int et = threadIdx.x - 128 - 128 * g;  // 0..127 within this warpgroup
+      uint8_t* ebuf = epi + g * C::kEpiBytes;
+      for (int c = g; c < nchunks; c += DQG) {
         const int r0 = rbase + 32 * c;
         if (r0 >= a.m) break;
         const int jmax = min(32, BN - 32 * c);
@@ -246,11 +316,11 @@ tc_w4a16_kernel(const __grid_constant__ CUtensorMap xmap, const TcArgs a) {
           for (int j = 0; j < 32; ++j)
             if (j < jmax && r0 + j < a.m) P[(size_t)(r0 + j) * a.n_pad + col] = __uint_as_float(v[j]);
         } else if (EPI == kEpiStore) {
-          uint16_t* T = reinterpret_cast<uint16_t*>(epi);  // [32][128] bf16
+          uint16_t* T = reinterpret_cast<uint16_t*>(ebuf);  // [32][128] bf16
           const float gs = a.gs[0];
 #pragma unroll
           for (int j = 0; j < 32; ++j) T[j * 128 + row] = f32_to_bf16_bits(gs * __uint_as_float(v[j]));
-          named_bar_sync(1, 128);
+          named_bar_sync(1 + g, 128);
           const int n0 = kTileRows * wtile;
           for (int idx = et; idx < 32 * 16; idx += 128) {
             const int j = idx >> 4, ch = idx & 15;
@@ -259,25 +329,25 @@ tc_w4a16_kernel(const __grid_constant__ CUtensorMap xmap, const TcArgs a) {
               *reinterpret_cast<uint4*>(static_cast<uint16_t*>(a.out) + (size_t)r * a.ldo + n) =
                   *reinterpret_cast<const uint4*>(T + j * 128 + 8 * ch);
           }
-          named_bar_sync(1, 128);
+          named_bar_sync(1 + g, 128);
         } else {  // kEpiSiluMul: rows 0-63 gate, 64-127 the matching up rows
-          float* U = reinterpret_cast<float*>(epi);                  // [32][64] fp32
-          uint16_t* Hs = reinterpret_cast<uint16_t*>(epi + 8192);    // [32][64] bf16
+          float* U = reinterpret_cast<float*>(ebuf);                  // [32][64] fp32
+          uint16_t* Hs = reinterpret_cast<uint16_t*>(ebuf + 8192);    // [32][64] bf16
           if (q >= 2) {
             const float gsu = a.gs[1];
 #pragma unroll
             for (int j = 0; j < 32; ++j) U[j * 64 + (row - 64)] = bf16_round(gsu * __uint_as_float(v[j]));
           }
-          named_bar_sync(1, 128);
+          named_bar_sync(1 + g, 128);
           if (q < 2) {
             const float gsg = a.gs[0];
 #pragma unroll
             for (int j = 0; j < 32; ++j) {
-              const float g = bf16_round(gsg * __uint_as_float(v[j]));
-              Hs[j * 64 + row] = f32_to_bf16_bits(silu_f32(g) * U[j * 64 + row]);
+              const float gv = bf16_round(gsg * __uint_as_float(v[j]));
+              Hs[j * 64 + row] = f32_to_bf16_bits(silu_fast(gv) * U[j * 64 + row]);
             }
           }
-          named_bar_sync(1, 128);
+          named_bar_sync(1 + g, 128);
           const int n0 = 64 * wtile;
           for (int idx = et; idx < 32 * 8; idx += 128) {
             const int j = idx >> 3, ch = idx & 7;
@@ -286,7 +356,7 @@ tc_w4a16_kernel(const __grid_constant__ CUtensorMap xmap, const TcArgs a) {
               *reinterpret_cast<uint4*>(static_cast<uint16_t*>(a.out) + (size_t)r * a.ldo + n) =
                   *reinterpret_cast<const uint4*>(Hs + j * 64 + 8 * ch);
           }
-          named_bar_sync(1, 128);
+          named_bar_sync(1 + g, 128);
         }
       }
     }
@@ -316,7 +386,7 @@ __global__ void splitk_reduce_kernel(const float* __restrict__ P, int splits, in
       u += P[z * plane + (size_t)r * n_pad + ucol];
     }
     const float gb = bf16_round(gs[0] * g), ub = bf16_round(gs[1] * u);
-    out[(size_t)r * ldo + n] = f32_to_bf16_bits(silu_f32(gb) * ub);
+    out[(size_t)r * ldo + n] = f32_to_bf16_bits(silu_fast(gb) * ub);
   } else {
     float acc = 0.0f;
     for (int z = 0; z < splits; ++z) acc += P[z * plane + (size_t)r * n_pad + n];
@@ -393,28 +463,29 @@ bool make_x_map(CUtensorMap* map, const void* x, int64_t m, int64_t k, int box_r
              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int BN, int STAGES, int EPI>
+template <int BN, int SX, int SW, int SA, int DQG, int EPI>
 cudaError_t launch_cfg(const CUtensorMap& map, const TcArgs& a, dim3 grid, cudaStream_t s) {
-  using C = TcCfg<BN, STAGES>;
-  auto kern = tc_w4a16_kernel<BN, STAGES, EPI>;
+  using C = TcCfg<BN, SX, SW, SA, DQG>;
+  auto kern = tc_w4a16_kernel<BN, SX, SW, SA, DQG, EPI>;
   static bool attr_set = false;  // per instantiation; idempotent if raced
   if (!attr_set) {
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemAlloc);
     if (e != cudaSuccess) return e;
     attr_set = true;
   }
-  kern<<<grid, 256, C::kSmemAlloc, s>>>(map, a);
+  kern<<<grid, C::kThreads, C::kSmemAlloc, s>>>(map, a);
   return cudaGetLastError();
 }
 
 template <int EPI>
 cudaError_t launch_bn(int bn, const CUtensorMap& map, const TcArgs& a, dim3 grid, cudaStream_t s) {
   switch (bn) {
-    case 16: return launch_cfg<16, 7, EPI>(map, a, grid, s);
-    case 32: return launch_cfg<32, 7, EPI>(map, a, grid, s);
-    case 64: return launch_cfg<64, 6, EPI>(map, a, grid, s);
-    case 128: return launch_cfg<128, 6, EPI>(map, a, grid, s);
-    default: return launch_cfg<256, 5, EPI>(map, a, grid, s);
+    // BN, activation stages, weight stages, TMEM stages, dequant warpgroups
+    case 16: return launch_cfg<16, 6, 12, 4, 2, EPI>(map, a, grid, s);
+    case 32: return launch_cfg<32, 6, 12, 4, 2, EPI>(map, a, grid, s);
+    case 64: return launch_cfg<64, 4, 10, 4, 2, EPI>(map, a, grid, s);
+    case 128: return launch_cfg<128, 6, 10, 4, 2, EPI>(map, a, grid, s);
+    default: return launch_cfg<256, 4, 8, 4, 2, EPI>(map, a, grid, s);
   }
 }
 
