@@ -73,6 +73,17 @@ Path w4a16_path(int64_t m) {
   return Path::kTc;
 }
 
+// Fixed format: the block-scaled FP4 tensor-core kernel, or the CUDA-core one
+// (FFN_NVFP4_W4A4_PATH=gemv).  Either choice is made once per process and does
+// not depend on m, which the format's row invariance requires.
+Path w4a4_path() {
+  static const Path p = [] {
+    const char* v = getenv("FFN_NVFP4_W4A4_PATH");
+    return (v && !strcmp(v, "gemv")) ? Path::kGemv : Path::kTc;
+  }();
+  return p;
+}
+
 // Workspace layout of ffn_nvfp4_forward / ffn_nvfp4_linear (each region
 // 256-byte aligned): [h bf16 m*inter] [xq codes m*hidden/2] [xq scales
 // m*hidden/16] [hq codes m*inter/2] [hq scales m*inter/16].
@@ -80,6 +91,28 @@ struct Carve {
   size_t h = 0, xq_c = 0, xq_s = 0, hq_c = 0, hq_s = 0, part = 0, total = 0;
   ffn::TcPlan gate_up, down;
 };
+
+// Workspace of the fixed format on the tensor-core path: quantised x and h
+// codes, their 512-byte scale blocks, h, split-K partials.
+void carve_w4a4_tc(Carve& c, size_t& off, int64_t m, int64_t hidden, int64_t inter, bool ffn) {
+  const int sms = num_sms();
+  if (ffn) {
+    c.gate_up = ffn::plan_w4a4(m, 2 * inter, hidden, true, sms);
+    c.down = ffn::plan_w4a4(m, hidden, inter, false, sms);
+  } else {
+    c.down = ffn::plan_w4a4(m, hidden, inter, false, sms);  // (n, k) = (hidden, inter)
+  }
+  c.xq_c = off; off += round_up((size_t)m * (ffn ? hidden : inter) / 2, 256);
+  c.xq_s = off; off += round_up(ffn::w4a4_sf_block_bytes(m, ffn ? hidden : inter), 256);
+  if (ffn) {
+    c.hq_c = off; off += round_up((size_t)m * inter / 2, 256);
+    c.hq_s = off; off += round_up(ffn::w4a4_sf_block_bytes(m, inter), 256);
+  }
+  const size_t pb = c.gate_up.partial_bytes > c.down.partial_bytes ? c.gate_up.partial_bytes
+                                                                  : c.down.partial_bytes;
+  c.part = off;
+  off += round_up(pb, 256);
+}
 
 Carve carve_ffn(int64_t m, int64_t hidden, int64_t inter, ffn_act_format f) {
   Carve c;
@@ -95,7 +128,9 @@ Carve carve_ffn(int64_t m, int64_t hidden, int64_t inter, ffn_act_format f) {
     c.part = off;
     off += round_up(pb, 256);
   }
-  if (f == FFN_ACT_NVFP4_FIXED) {
+  if (f == FFN_ACT_NVFP4_FIXED && m > 0 && w4a4_path() == Path::kTc) {
+    carve_w4a4_tc(c, off, m, hidden, inter, true);
+  } else if (f == FFN_ACT_NVFP4_FIXED) {
     c.xq_c = off; off += round_up((size_t)m * hidden / 2, 256);
     c.xq_s = off; off += round_up((size_t)m * hidden / 16, 256);
     c.hq_c = off; off += round_up((size_t)m * inter / 2, 256);
@@ -113,7 +148,9 @@ Carve carve_linear(int64_t m, int64_t n, int64_t k, ffn_act_format f) {
     c.part = off;
     off += round_up(c.down.partial_bytes, 256);
   }
-  if (f == FFN_ACT_NVFP4_FIXED) {
+  if (f == FFN_ACT_NVFP4_FIXED && m > 0 && w4a4_path() == Path::kTc) {
+    carve_w4a4_tc(c, off, m, n, k, false);
+  } else if (f == FFN_ACT_NVFP4_FIXED) {
     c.xq_c = off; off += round_up((size_t)m * k / 2, 256);
     c.xq_s = off; off += round_up((size_t)m * k / 16, 256);
   }
@@ -330,6 +367,13 @@ ffn_status ffn_nvfp4_forward(const void* x, int64_t m, int64_t hidden, int64_t i
   } else if (format == FFN_ACT_BF16) {
     e = ffn::launch_gemv_w4a16(x, m, gate_up->view(), Epilogue::kSiluMul, h, s);
     if (e == cudaSuccess) e = ffn::launch_gemv_w4a16(h, m, down->view(), Epilogue::kStore, out, s);
+  } else if (w4a4_path() == Path::kTc) {
+    uint8_t *xq = ws + c.xq_c, *xs = ws + c.xq_s, *hq = ws + c.hq_c, *hs = ws + c.hq_s;
+    void* part = ws + c.part;
+    e = ffn::launch_quantize_activations_blocked(x, m, hidden, xq, xs, s);
+    if (e == cudaSuccess) e = ffn::launch_tc_w4a4(xq, xs, m, gate_up->tc(), true, c.gate_up, h, part, s);
+    if (e == cudaSuccess) e = ffn::launch_quantize_activations_blocked(h, m, inter, hq, hs, s);
+    if (e == cudaSuccess) e = ffn::launch_tc_w4a4(hq, hs, m, down->tc(), false, c.down, out, part, s);
   } else {
     uint8_t *xq = ws + c.xq_c, *xs = ws + c.xq_s, *hq = ws + c.hq_c, *hs = ws + c.hq_s;
     e = ffn::launch_quantize_activations(x, m, hidden, xq, xs, s);
@@ -379,6 +423,11 @@ ffn_status ffn_nvfp4_linear(const void* x, int64_t m, const ffn_nvfp4_weight* w,
     e = ffn::launch_tc_w4a16(x, m, w->tc(), false, c.down, y, static_cast<uint8_t*>(workspace) + c.part, s);
   } else if (format == FFN_ACT_BF16) {
     e = ffn::launch_gemv_w4a16(x, m, w->view(), Epilogue::kStore, y, s);
+  } else if (w4a4_path() == Path::kTc) {
+    uint8_t* ws = static_cast<uint8_t*>(workspace);
+    e = ffn::launch_quantize_activations_blocked(x, m, w->k, ws + c.xq_c, ws + c.xq_s, s);
+    if (e == cudaSuccess)
+      e = ffn::launch_tc_w4a4(ws + c.xq_c, ws + c.xq_s, m, w->tc(), false, c.down, y, ws + c.part, s);
   } else {
     uint8_t* ws = static_cast<uint8_t*>(workspace);
     e = ffn::launch_quantize_activations(x, m, w->k, ws + c.xq_c, ws + c.xq_s, s);

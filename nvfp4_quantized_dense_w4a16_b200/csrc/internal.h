@@ -42,6 +42,18 @@ cudaError_t launch_tile_weight(const uint8_t* codes, const uint8_t* scales, int6
                                bool gate_up, uint8_t* out, cudaStream_t s);
 cudaError_t launch_tc_w4a16(const void* x, int64_t m, const TcWeight& w, bool silu_mul,
                             const TcPlan& p, void* y, void* partials, cudaStream_t s);
+// Fixed-format (W4A4) projection on the block-scaled FP4 tensor core.  The
+// plan depends on (n, k) only (plus the number of 128-row activation tiles).
+TcPlan plan_w4a4(int64_t m, int64_t n, int64_t k, bool gate_up, int num_sms);
+size_t w4a4_sf_block_bytes(int64_t m, int64_t k);
+cudaError_t launch_tc_w4a4(const uint8_t* xcodes, const uint8_t* xsf_blocks, int64_t m,
+                           const TcWeight& w, bool silu_mul, const TcPlan& p, void* y,
+                           void* partials, cudaStream_t s);
+// Activation quantiser that also writes the scales as 512-byte blocks per
+// 128 rows and 64 elements (the W4A4 kernel's scale-factor layout).
+cudaError_t launch_quantize_activations_blocked(const void* x, int64_t m, int64_t k, void* codes,
+                                                void* sf_blocks, cudaStream_t s);
+
 // Tensor-core view of a handle (and whether it is a fused gate+up handle).
 void handle_tc_view(const ffn_nvfp4_weight* w, TcWeight* out, bool* gate_up);
 

@@ -106,6 +106,36 @@ __global__ void quantize_act_blocks_kernel(const uint16_t* __restrict__ x, int64
   scales[i] = (uint8_t)s8;
 }
 
+// As above, with the scale byte of (row r, 16-block kb) stored at
+// ((r / 128) * kc + kb / 4) * 512 + 16 * (r % 32) + 4 * ((r % 128) / 32) + kb % 4.
+__global__ void quantize_act_blocked_kernel(const uint16_t* __restrict__ x, int64_t nblocks,
+                                            int64_t kb_per_row, int kc,
+                                            uint8_t* __restrict__ codes,
+                                            uint8_t* __restrict__ sf_blocks) {
+  const int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;
+  if (i >= nblocks) return;
+  Block16 b;
+  load_block16(x + 16 * i, b);
+  const uint32_t s8 = e4m3_encode_satfinite(__fdiv_rn(b.amax, 6.0f));
+  const uint2 c = encode_block16(b, e4m3_decode(s8), s8 == 0);
+  reinterpret_cast<uint2*>(codes)[i] = c;
+  const int64_t r = i / kb_per_row, kb = i % kb_per_row;
+  const int rr = (int)(r & 127);
+  sf_blocks[((r >> 7) * kc + kb / 4) * 512 + 16 * (rr & 31) + 4 * (rr >> 5) + (kb & 3)] = (uint8_t)s8;
+}
+
+cudaError_t launch_quantize_activations_blocked(const void* x, int64_t m, int64_t k, void* codes,
+                                                void* sf_blocks, cudaStream_t s) {
+  const int64_t nblocks = m * k / 16;
+  if (nblocks == 0) return cudaSuccess;
+  const int threads = 256;
+  const int kc = (int)((k + 63) / 64);
+  ProfScope prof(s, "quantize_activations");
+  quantize_act_blocked_kernel<<<(unsigned)((nblocks + threads - 1) / threads), threads, 0, s>>>(
+      (const uint16_t*)x, nblocks, k / 16, kc, (uint8_t*)codes, (uint8_t*)sf_blocks);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_quantize_weights(const void* w, int64_t n, int64_t k, void* codes,
                                     void* scales, float* gs, cudaStream_t s) {
   const int64_t count = n * k;

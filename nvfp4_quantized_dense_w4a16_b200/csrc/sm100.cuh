@@ -167,6 +167,17 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&v)[32]) {
       : "memory");
 }
 
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&v)[16]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, "
+      "%11, %12, %13, %14, %15}, [%16];"
+      : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]),
+        "=r"(v[7]), "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]),
+        "=r"(v[14]), "=r"(v[15])
+      : "r"(taddr)
+      : "memory");
+}
+
 __device__ __forceinline__ void tmem_ld_wait() {
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
@@ -194,6 +205,50 @@ __device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t saddr) {
   d |= (uint64_t)1 << 46;                    // descriptor version for sm_100
   d |= (uint64_t)2 << 61;                    // layout: 128-byte swizzle
   return d;
+}
+
+// Shared-memory descriptor of a K-major operand without swizzle: 16-byte
+// rows, 8-row core matrices `sbo` bytes apart, the next 16-byte K unit `lbo`
+// bytes away (the tile base must be 16-byte aligned).
+__device__ __forceinline__ uint64_t smem_desc_interleave(uint32_t saddr, uint32_t lbo,
+                                                         uint32_t sbo) {
+  uint64_t d = 0;
+  d |= (uint64_t)((saddr & 0x3FFFFu) >> 4);
+  d |= (uint64_t)((lbo >> 4) & 0x3FFFu) << 16;
+  d |= (uint64_t)((sbo >> 4) & 0x3FFFu) << 32;
+  d |= (uint64_t)1 << 46;  // descriptor version for sm_100; layout 0 = no swizzle
+  return d;
+}
+
+// Instruction descriptor of kind::mxf4nvf4 (E2M1 A and B, both K-major,
+// UE4M3 scale factors, one per 16 elements, fp32 accumulation).
+__host__ __device__ constexpr uint32_t idesc_mxf4nvf4(int M, int N) {
+  return (1u << 7)                     // A format: E2M1
+         | (1u << 10)                  // B format: E2M1
+         | ((uint32_t)(N >> 3) << 17)  // N / 8
+         | (0u << 23)                  // scale factor format: UE4M3
+         | ((uint32_t)(M >> 4) << 24); // M / 16
+}
+
+// Block-scaled FP4 MMA (K = 64 per instruction): D (+)= (A * SFA) (B * SFB)^T
+// with A, B in shared memory and the scale factors in TMEM.
+__device__ __forceinline__ void mma_mxf4nvf4(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                             uint32_t idesc, uint32_t sfa_tmem, uint32_t sfb_tmem,
+                                             uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::mxf4nvf4.block_scale.scale_vec::4X [%0], %1, %2, %3, [%5], "
+      "[%6], p;\n\t}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(sfa_tmem), "r"(sfb_tmem)
+      : "memory");
+}
+
+// Copy a 32-row x 16-byte shared-memory block into 4 TMEM columns of lanes
+// 0-31, replicated into the other three lane quarters.
+__device__ __forceinline__ void tmem_cp_32x128b_x4(uint32_t taddr, uint64_t sdesc) {
+  asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc)
+               : "memory");
 }
 
 // D[tmem] (+)= A[tmem] * B[smem]^T, issued by one thread.

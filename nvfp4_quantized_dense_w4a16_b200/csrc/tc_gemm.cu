@@ -6,7 +6,11 @@
 // Design (one CTA per 128-weight-row tile x BN activation rows x K range):
 //  * weights are streamed in a pre-tiled layout (per 128-row tile and
 //    64-element K chunk: 128 x 16 B low codes, 128 x 16 B high codes,
-//    128 x 4 B E4M3 scales = 4608 B) by one bulk async copy per stage;
+//    128 x 4 B E4M3 scales = 4608 B) by one bulk async copy per stage; the
+//    codes are the canonical no-swizzle K-major operand layout of the
+//    block-scaled FP4 MMA and the scale bytes its 512-byte scale-factor block
+//    (row r at byte 16*(r%32) + 4*(r/32)), so the W4A4 kernel streams the
+//    same bytes;
 //  * activations X [m, K] bf16 arrive by 2-D TMA with the 128-byte swizzle
 //    (box 64 x BN), the layout the MMA reads directly;
 //  * four dequant warps turn each thread's row of codes into exact bf16
@@ -54,7 +58,10 @@ template <int BN, int SX, int SW, int SA, int DQG>
 struct TcCfg {
   static constexpr int kThreads = 128 + 128 * DQG;
   static constexpr int kXStageBytes = BN * 128;
-  static constexpr int kAColBase = BN < 32 ? 32 : BN;  // TMEM column of A stage 0
+  // Independent accumulators: narrow tiles rotate their K steps over several
+  // accumulators so that consecutive MMAs do not wait on each other's result.
+  static constexpr int kNacc = BN <= 32 ? 4 : BN <= 64 ? 2 : 1;
+  static constexpr int kAColBase = kNacc * BN < 32 ? 32 : kNacc * BN;  // TMEM column of A stage 0
   static constexpr int kTmemNeed = kAColBase + 32 * SA;
   static constexpr int kTmemCols = kTmemNeed <= 64 ? 64 : kTmemNeed <= 128 ? 128 : kTmemNeed <= 256 ? 256 : 512;
   static constexpr int kEpiBytes = 16384;  // per dequant warpgroup
@@ -154,6 +161,93 @@ __device__ __forceinline__ bool wait_drain(uint64_t* bar, uint32_t parity) {
   return true;
 }
 
+// Epilogue of one (128 weight rows) x (BN activation rows) accumulator tile
+// held in TMEM columns [0, BN): warpgroup g of NG takes every NG-th 32-column
+// chunk; thread (q, lane) owns tile row 32q + lane.  kEpiStore writes
+// y = bf16(gs * acc); kEpiSiluMul (rows 0-63 gate, 64-127 the matching up rows)
+// writes h = bf16(silu(bf16(gs_g * g)) * bf16(gs_u * u)); kEpiPartial writes
+// fp32 split-K partials.  Stores are staged through shared memory (ebuf,
+// 16 KB per warpgroup) so that global writes are 16-byte and row-contiguous.
+template <int BN, int EPI, int NG, int NACC = 1>
+__device__ __forceinline__ void epilogue_tile(const TcArgs& a, uint32_t tmem, int q, int lane,
+                                              int g, uint8_t* ebuf, int xtile, int wtile) {
+  const int row = 32 * q + lane;
+  const uint32_t lane_addr = (uint32_t)(32 * q) << 16;
+  const int rbase = xtile * BN;
+  const int nchunks = (BN + 31) / 32;
+  const int et = 32 * q + lane;  // 0..127 within this warpgroup
+  for (int c = g; c < nchunks; c += NG) {
+    const int r0 = rbase + 32 * c;
+    if (r0 >= a.m) break;
+    const int jmax = min(32, BN - 32 * c);
+    uint32_t v[32];
+    tmem_ld32(tmem + lane_addr + 32 * c, v);
+    tmem_ld_wait();
+    // accumulators 1..NACC-1 hold the other K steps: add them in a fixed order
+#pragma unroll
+    for (int acc = 1; acc < NACC; ++acc) {
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        uint32_t u[16];
+        tmem_ld16(tmem + lane_addr + acc * BN + 32 * c + 16 * h, u);
+        tmem_ld_wait();
+#pragma unroll
+        for (int j = 0; j < 16; ++j)
+          v[16 * h + j] = __float_as_uint(__uint_as_float(v[16 * h + j]) + __uint_as_float(u[j]));
+      }
+    }
+    if (EPI == kEpiPartial) {
+      float* P = static_cast<float*>(a.out) + (size_t)blockIdx.z * a.m * a.n_pad;
+      const int col = kTileRows * wtile + row;
+#pragma unroll
+      for (int j = 0; j < 32; ++j)
+        if (j < jmax && r0 + j < a.m) P[(size_t)(r0 + j) * a.n_pad + col] = __uint_as_float(v[j]);
+    } else if (EPI == kEpiStore) {
+      uint16_t* T = reinterpret_cast<uint16_t*>(ebuf);  // [32][128] bf16
+      const float gs = a.gs[0];
+#pragma unroll
+      for (int j = 0; j < 32; ++j) T[j * 128 + row] = f32_to_bf16_bits(gs * __uint_as_float(v[j]));
+      named_bar_sync(1 + g, 128);
+      const int n0 = kTileRows * wtile;
+      for (int idx = et; idx < 32 * 16; idx += 128) {
+        const int j = idx >> 4, ch = idx & 15;
+        const int r = r0 + j, n = n0 + 8 * ch;
+        if (j < jmax && r < a.m && n < a.n_out)
+          *reinterpret_cast<uint4*>(static_cast<uint16_t*>(a.out) + (size_t)r * a.ldo + n) =
+              *reinterpret_cast<const uint4*>(T + j * 128 + 8 * ch);
+      }
+      named_bar_sync(1 + g, 128);
+    } else {  // kEpiSiluMul
+      float* U = reinterpret_cast<float*>(ebuf);                  // [32][64] fp32
+      uint16_t* Hs = reinterpret_cast<uint16_t*>(ebuf + 8192);    // [32][64] bf16
+      if (q >= 2) {
+        const float gsu = a.gs[1];
+#pragma unroll
+        for (int j = 0; j < 32; ++j) U[j * 64 + (row - 64)] = bf16_round(gsu * __uint_as_float(v[j]));
+      }
+      named_bar_sync(1 + g, 128);
+      if (q < 2) {
+        const float gsg = a.gs[0];
+#pragma unroll
+        for (int j = 0; j < 32; ++j) {
+          const float gv = bf16_round(gsg * __uint_as_float(v[j]));
+          Hs[j * 64 + row] = f32_to_bf16_bits(silu_fast(gv) * U[j * 64 + row]);
+        }
+      }
+      named_bar_sync(1 + g, 128);
+      const int n0 = 64 * wtile;
+      for (int idx = et; idx < 32 * 8; idx += 128) {
+        const int j = idx >> 3, ch = idx & 7;
+        const int r = r0 + j, n = n0 + 8 * ch;
+        if (j < jmax && r < a.m && n < a.n_out)
+          *reinterpret_cast<uint4*>(static_cast<uint16_t*>(a.out) + (size_t)r * a.ldo + n) =
+              *reinterpret_cast<const uint4*>(Hs + j * 64 + 8 * ch);
+      }
+      named_bar_sync(1 + g, 128);
+    }
+  }
+}
+
 template <int BN, int SX, int SW, int SA, int DQG, int EPI>
 __global__ void __launch_bounds__(TcCfg<BN, SX, SW, SA, DQG>::kThreads,
                                   TcCfg<BN, SX, SW, SA, DQG>::kMinBlocks)
@@ -250,7 +344,8 @@ tc_w4a16_kernel(const __grid_constant__ CUtensorMap xmap, const TcArgs a) {
         const uint64_t b_base = smem_desc_sw128(smem_u32(xs + sx * C::kXStageBytes));
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk)
-          mma_bf16_ts(tmem, a_base + 8 * kk, b_base + 2 * kk, idesc, (i | kk) != 0 ? 1u : 0u);
+          mma_bf16_ts(tmem + (kk % C::kNacc) * BN, a_base + 8 * kk, b_base + 2 * kk, idesc,
+                      (i > 0 || kk >= C::kNacc) ? 1u : 0u);
         mma_commit(&aempty[sa]);
         mma_commit(&xempty[sx]);
       }
@@ -262,6 +357,12 @@ tc_w4a16_kernel(const __grid_constant__ CUtensorMap xmap, const TcArgs a) {
     const int q = warp & 3;                       // TMEM lane quarter
     const int row = 32 * q + lane;                // tile row == TMEM lane
     const uint32_t lane_addr = (uint32_t)(32 * q) << 16;
+    const int sf_off = 16 * lane + 4 * q;         // this row's 4 scale bytes (block layout)
+    // The store of chunk i is completed (wait::st, then the MMA is told) only
+    // after chunk i+1 has been dequantised, so the TMEM store latency overlaps
+    // the next chunk's arithmetic.
+    bool pending = false;
+    int pending_sa = 0;
     for (int i = 0; i < nk; ++i) {
       const int s = i % SW, sa = i % SA;
       bool ok = mbar_wait(&wfull[s], (i / SW) & 1, abort_flag, err, 4);
@@ -271,15 +372,22 @@ tc_w4a16_kernel(const __grid_constant__ CUtensorMap xmap, const TcArgs a) {
       if constexpr (DQG == 1) {
         const uint4 lo = *reinterpret_cast<const uint4*>(w + 16 * row);
         const uint4 hi = *reinterpret_cast<const uint4*>(w + 2048 + 16 * row);
-        const uint32_t sc = *reinterpret_cast<const uint32_t*>(w + 4096 + 4 * row);
+        const uint32_t sc = *reinterpret_cast<const uint32_t*>(w + 4096 + sf_off);
         dequant64(lo, hi, sc, *reinterpret_cast<uint32_t(*)[32]>(v));
       } else {
         const uint4 c = *reinterpret_cast<const uint4*>(w + 2048 * g + 16 * row);
-        const uint32_t sc = *reinterpret_cast<const uint16_t*>(w + 4096 + 4 * row + 2 * g);
+        const uint32_t sc = *reinterpret_cast<const uint16_t*>(w + 4096 + sf_off + 2 * g);
         dequant32(c, sc, *reinterpret_cast<uint32_t(*)[16]>(v));
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(&wempty[s]);   // the shared-memory slot may be refilled
+      if (pending) {
+        tmem_st_wait();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&afull[pending_sa]);
+        pending = false;
+      }
       if (i >= SA) {
         ok = mbar_wait(&aempty[sa], ((i / SA) - 1) & 1, abort_flag, err, 4);
         if (!__all_sync(0xffffffffu, ok)) break;
@@ -290,76 +398,160 @@ tc_w4a16_kernel(const __grid_constant__ CUtensorMap xmap, const TcArgs a) {
         tmem_st32(taddr, *reinterpret_cast<uint32_t(*)[32]>(v));
       else
         tmem_st16(taddr, *reinterpret_cast<uint32_t(*)[16]>(v));
+      pending = true;
+      pending_sa = sa;
+    }
+    if (pending) {
       tmem_st_wait();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&afull[sa]);
+      if (lane == 0) mbar_arrive(&afull[pending_sa]);
     }
     const bool done = __all_sync(0xffffffffu, wait_drain(accum, 0));
     tc_fence_after();
-    if (done && !*abort_flag) {
-      const int rbase = xtile * BN;
-      const int nchunks = (BN + 31) / 32;
-      const int et = threadIdx.x - 128 - 128 * g;  // 0..127 within this warpgroup
-      uint8_t* ebuf = epi + g * C::kEpiBytes;
-      for (int c = g; c < nchunks; c += DQG) {
-        const int r0 = rbase + 32 * c;
-        if (r0 >= a.m) break;
-        const int jmax = min(32, BN - 32 * c);
-        uint32_t v[32];
-        tmem_ld32(tmem + lane_addr + 32 * c, v);
-        tmem_ld_wait();
-        if (EPI == kEpiPartial) {
-          float* P = static_cast<float*>(a.out) + (size_t)blockIdx.z * a.m * a.n_pad;
-          const int col = kTileRows * wtile + row;
-#pragma unroll
-          for (int j = 0; j < 32; ++j)
-            if (j < jmax && r0 + j < a.m) P[(size_t)(r0 + j) * a.n_pad + col] = __uint_as_float(v[j]);
-        } else if (EPI == kEpiStore) {
-          uint16_t* T = reinterpret_cast<uint16_t*>(ebuf);  // [32][128] bf16
-          const float gs = a.gs[0];
-#pragma unroll
-          for (int j = 0; j < 32; ++j) T[j * 128 + row] = f32_to_bf16_bits(gs * __uint_as_float(v[j]));
-          named_bar_sync(1 + g, 128);
-          const int n0 = kTileRows * wtile;
-          for (int idx = et; idx < 32 * 16; idx += 128) {
-            const int j = idx >> 4, ch = idx & 15;
-            const int r = r0 + j, n = n0 + 8 * ch;
-            if (j < jmax && r < a.m && n < a.n_out)
-              *reinterpret_cast<uint4*>(static_cast<uint16_t*>(a.out) + (size_t)r * a.ldo + n) =
-                  *reinterpret_cast<const uint4*>(T + j * 128 + 8 * ch);
-          }
-          named_bar_sync(1 + g, 128);
-        } else {  // kEpiSiluMul: rows 0-63 gate, 64-127 the matching up rows
-          float* U = reinterpret_cast<float*>(ebuf);                  // [32][64] fp32
-          uint16_t* Hs = reinterpret_cast<uint16_t*>(ebuf + 8192);    // [32][64] bf16
-          if (q >= 2) {
-            const float gsu = a.gs[1];
-#pragma unroll
-            for (int j = 0; j < 32; ++j) U[j * 64 + (row - 64)] = bf16_round(gsu * __uint_as_float(v[j]));
-          }
-          named_bar_sync(1 + g, 128);
-          if (q < 2) {
-            const float gsg = a.gs[0];
-#pragma unroll
-            for (int j = 0; j < 32; ++j) {
-              const float gv = bf16_round(gsg * __uint_as_float(v[j]));
-              Hs[j * 64 + row] = f32_to_bf16_bits(silu_fast(gv) * U[j * 64 + row]);
-            }
-          }
-          named_bar_sync(1 + g, 128);
-          const int n0 = 64 * wtile;
-          for (int idx = et; idx < 32 * 8; idx += 128) {
-            const int j = idx >> 3, ch = idx & 7;
-            const int r = r0 + j, n = n0 + 8 * ch;
-            if (j < jmax && r < a.m && n < a.n_out)
-              *reinterpret_cast<uint4*>(static_cast<uint16_t*>(a.out) + (size_t)r * a.ldo + n) =
-                  *reinterpret_cast<const uint4*>(Hs + j * 64 + 8 * ch);
-          }
-          named_bar_sync(1 + g, 128);
-        }
-      }
+    if (done && !*abort_flag)
+      epilogue_tile<BN, EPI, DQG, C::kNacc>(a, tmem, q, lane, g, epi + g * C::kEpiBytes, xtile, wtile);
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 2) {
+    tc_fence_after();
+    tmem_dealloc(tmem, C::kTmemCols);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Fixed-format (W4A4) projection on the block-scaled FP4 tensor core
+// ("metrale_model_layers/layers/dense_ffn_fixed.rs", forward_fixed: the
+// nvfp4_proj_mx projections).  D[n, r] = sum_k (wq * sw)[n, k] (xq * sx)[r, k]
+// with kind::mxf4nvf4 (E2M1 x E2M1, UE4M3 scale per 16 elements, fp32 in TMEM).
+//  * A = weights: the same 4608-byte tiled chunks as above, read by one bulk
+//    copy per stage of kW4Chunks chunks; the codes are the no-swizzle K-major
+//    operand (16-byte rows, 8-row groups 128 B apart, second K half 2048 B
+//    away) and the chunk's 512-byte scale block is copied to TMEM as SFA;
+//  * B = quantised activations: codes [m, K/2] by 2-D TMA (128-byte rows of
+//    256 elements, 128-byte swizzle), scale blocks (one 512-byte block per
+//    128 rows and 64 elements, written by the activation quantiser) by bulk
+//    copy, copied to TMEM as SFB;
+//  * the tile shape (128 weight rows x 128 activation rows), the K split and
+//    the K order depend only on (n, K), never on m, and every output column
+//    of an MMA depends only on its own activation row, so a row's result is
+//    the same whatever m is.
+// ---------------------------------------------------------------------------
+constexpr int kW4BN = 128;        // activation rows per tile (fixed)
+constexpr int kW4Chunks = 4;      // 64-element chunks per stage
+constexpr int kW4Stages = 5;
+
+struct W4Cfg {
+  static constexpr int kWBytes = kW4Chunks * kChunkBytes;  // 18432
+  static constexpr int kXBytes = kW4BN * 128;              // 16384 (128 rows x 256 elements)
+  static constexpr int kSfbBytes = kW4Chunks * 512;        // 2048
+  static constexpr int kStageBytes = kWBytes + kXBytes + kSfbBytes;  // 36864 = 36 KB
+  static constexpr int kSmemEpi = kW4Stages * kStageBytes;
+  static constexpr int kSmemBar = kSmemEpi + 16384;
+  static constexpr int kSmemBytes = kSmemBar + (2 * kW4Stages + 1) * 8 + 16;
+  static constexpr int kSmemAlloc = kSmemBytes + 1024;
+  static constexpr int kSfaCol = kW4BN;                                  // TMEM columns
+  static constexpr int kSfbCol = kSfaCol + 4 * kW4Chunks * kW4Stages;
+  static constexpr int kTmemCols = 512;
+  static_assert(kSfbCol + 4 * kW4Chunks * kW4Stages <= kTmemCols, "TMEM budget");
+  static_assert(kStageBytes % 1024 == 0, "stage alignment");
+  static_assert(kSmemAlloc <= 232448, "shared memory budget");
+};
+
+struct W4Args {
+  TcArgs t;
+  const uint8_t* sfb;   // activation scale blocks [ceil(m/128)][kc][512]
+};
+
+template <int EPI>
+__global__ void __launch_bounds__(256, 1)
+tc_w4a4_kernel(const __grid_constant__ CUtensorMap xmap, const W4Args w4) {
+  using C = W4Cfg;
+  const TcArgs& a = w4.t;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  uint8_t* epi = smem + C::kSmemEpi;
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::kSmemBar);
+  uint64_t* empty = full + kW4Stages;
+  uint64_t* accum = empty + kW4Stages;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(accum + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  int* err = &g_ffn_device_error;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int xtile = blockIdx.x, wtile = blockIdx.y;
+  const int kc0 = blockIdx.z * a.kc_per_split;
+  const int nk = min(a.kc_total, kc0 + a.kc_per_split) - kc0;     // chunks of this CTA
+  const int nstage = (nk + kW4Chunks - 1) / kW4Chunks;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kW4Stages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
     }
+    mbar_init(accum, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 2) {
+    tmem_alloc(tmem_slot, C::kTmemCols);
+    tmem_relinquish();
+  }
+  if (warp == 0 && lane == 0) tma_prefetch_desc(&xmap);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      const uint8_t* wsrc = a.wt + ((size_t)wtile * a.kc_total + kc0) * kChunkBytes;
+      const uint8_t* ssrc = w4.sfb + ((size_t)xtile * a.kc_total + kc0) * 512;
+      int issued = 0;
+      for (int i = 0; i < nstage; ++i) {
+        const int s = i % kW4Stages;
+        const int nch = min(kW4Chunks, nk - kW4Chunks * i);
+        if (i >= kW4Stages && !mbar_wait(&empty[s], ((i / kW4Stages) - 1) & 1, abort_flag, err, 1)) break;
+        uint8_t* st = smem + s * C::kStageBytes;
+        mbar_arrive_expect_tx(&full[s], nch * (kChunkBytes + 512) + C::kXBytes);
+        bulk_load(st, wsrc + (size_t)kW4Chunks * i * kChunkBytes, nch * kChunkBytes, &full[s]);
+        tma_load_2d(st + C::kWBytes, &xmap, 32 * (kc0 + kW4Chunks * i), xtile * kW4BN, &full[s]);
+        bulk_load(st + C::kWBytes + C::kXBytes, ssrc + (size_t)kW4Chunks * i * 512, nch * 512, &full[s]);
+        ++issued;
+      }
+      for (int i = max(0, issued - kW4Stages); i < issued; ++i)
+        wait_drain(&full[i % kW4Stages], (i / kW4Stages) & 1);
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      const uint32_t idesc = idesc_mxf4nvf4(kTileRows, kW4BN);
+      for (int i = 0; i < nstage; ++i) {
+        const int s = i % kW4Stages;
+        const int nch = min(kW4Chunks, nk - kW4Chunks * i);
+        if (!mbar_wait(&full[s], (i / kW4Stages) & 1, abort_flag, err, 2)) break;
+        tc_fence_after();
+        const uint8_t* st = smem + s * C::kStageBytes;
+        const uint64_t b_base = smem_desc_sw128(smem_u32(st + C::kWBytes));
+        for (int c = 0; c < nch; ++c) {
+          const uint32_t slot = 4 * (s * kW4Chunks + c);
+          const uint8_t* wc = st + c * kChunkBytes;
+          tmem_cp_32x128b_x4(tmem + C::kSfaCol + slot, smem_desc_interleave(smem_u32(wc + 4096), 16, 128));
+          tmem_cp_32x128b_x4(tmem + C::kSfbCol + slot,
+                             smem_desc_interleave(smem_u32(st + C::kWBytes + C::kXBytes + 512 * c), 16, 128));
+          mma_mxf4nvf4(tmem, smem_desc_interleave(smem_u32(wc), 2048, 128), b_base + 2 * c, idesc,
+                       tmem + C::kSfaCol + slot, tmem + C::kSfbCol + slot, (i | c) != 0 ? 1u : 0u);
+        }
+        mma_commit(&empty[s]);
+      }
+      mma_commit(accum);
+    }
+  } else if (warp >= 4) {
+    const int q = warp & 3;
+    const bool done = __all_sync(0xffffffffu, wait_drain(accum, 0));
+    tc_fence_after();
+    if (done && !*abort_flag) epilogue_tile<kW4BN, EPI, 1>(a, tmem, q, lane, 0, epi, xtile, wtile);
   }
   tc_fence_before();
   __syncthreads();
@@ -432,7 +624,9 @@ __global__ void tile_weight_kernel(const uint8_t* __restrict__ codes,
   uint8_t* base = out + ((int64_t)t * kc + j) * kChunkBytes;
   *reinterpret_cast<uint4*>(base + 16 * r) = lo;
   *reinterpret_cast<uint4*>(base + 2048 + 16 * r) = hi;
-  *reinterpret_cast<uint32_t*>(base + 4096 + 4 * r) = sc;
+  // scale bytes in the 512-byte block arrangement of the block-scaled MMA's
+  // scale-factor copy: row r's four scales at 16 * (r % 32) + 4 * (r / 32)
+  *reinterpret_cast<uint32_t*>(base + 4096 + 16 * (r & 31) + 4 * (r >> 5)) = sc;
 }
 
 // ----------------------------------------------------------------- host side
@@ -568,6 +762,90 @@ cudaError_t launch_tc_w4a16(const void* x, int64_t m, const TcWeight& w, bool si
   ProfScope prof(s, silu_mul ? "tc_w4a16_gate_up_silu" : "tc_w4a16");
   return silu_mul ? launch_bn<kEpiSiluMul>(p.bn, map, a, grid, s)
                   : launch_bn<kEpiStore>(p.bn, map, a, grid, s);
+}
+
+TcPlan plan_w4a4(int64_t m, int64_t n, int64_t k, bool gate_up, int num_sms) {
+  // Everything but the number of activation tiles depends on (n, k) only.
+  TcPlan p;
+  p.bn = kW4BN;
+  p.xtiles = (int)((m + kW4BN - 1) / kW4BN);
+  p.wtiles = (int)(gate_up ? (n / 2 + 63) / 64 : (n + kTileRows - 1) / kTileRows);
+  p.kc = (int)((k + kChunkK - 1) / kChunkK);
+  p.n_pad = p.wtiles * kTileRows;
+  int splits = num_sms / p.wtiles;
+  const int max_splits = p.kc / (2 * kW4Chunks) > 1 ? p.kc / (2 * kW4Chunks) : 1;
+  if (splits > max_splits) splits = max_splits;
+  if (splits < 1) splits = 1;
+  p.kc_per_split = (p.kc + splits - 1) / splits;
+  p.kc_per_split = (p.kc_per_split + kW4Chunks - 1) / kW4Chunks * kW4Chunks;
+  p.splits = (p.kc + p.kc_per_split - 1) / p.kc_per_split;
+  p.partial_bytes = p.splits > 1 ? (size_t)p.splits * m * p.n_pad * sizeof(float) : 0;
+  return p;
+}
+
+size_t w4a4_sf_block_bytes(int64_t m, int64_t k) {
+  return (size_t)((m + kW4BN - 1) / kW4BN) * ((k + kChunkK - 1) / kChunkK) * 512;
+}
+
+cudaError_t launch_tc_w4a4(const uint8_t* xcodes, const uint8_t* xsf_blocks, int64_t m,
+                           const TcWeight& w, bool silu_mul, const TcPlan& p, void* y,
+                           void* partials, cudaStream_t s) {
+  auto enc = get_encode();
+  if (!enc) return cudaErrorInvalidValue;
+  CUtensorMap map;
+  {
+    cuuint64_t dims[2] = {(cuuint64_t)(w.k / 2), (cuuint64_t)m};
+    cuuint64_t strides[1] = {(cuuint64_t)(w.k / 2)};
+    cuuint32_t box[2] = {128, (cuuint32_t)kW4BN};
+    cuuint32_t estr[2] = {1, 1};
+    if (enc(&map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t*>(xcodes), dims, strides, box,
+            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return cudaErrorInvalidValue;
+  }
+  W4Args a;
+  a.t.wt = w.tiled;
+  a.t.gs = w.gs;
+  a.t.m = (int)m;
+  a.t.n_out = (int)(silu_mul ? w.n / 2 : w.n);
+  a.t.ldo = a.t.n_out;
+  a.t.kc_total = p.kc;
+  a.t.kc_per_split = p.kc_per_split;
+  a.t.n_pad = p.n_pad;
+  a.sfb = xsf_blocks;
+  const dim3 grid(p.xtiles, p.wtiles, p.splits);
+  static bool attr_set[3] = {false, false, false};
+  auto launch = [&](auto kern, int epi) -> cudaError_t {
+    if (!attr_set[epi]) {
+      cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, W4Cfg::kSmemAlloc);
+      if (e != cudaSuccess) return e;
+      attr_set[epi] = true;
+    }
+    kern<<<grid, 256, W4Cfg::kSmemAlloc, s>>>(map, a);
+    return cudaGetLastError();
+  };
+  cudaError_t e;
+  if (p.splits > 1) {
+    a.t.out = partials;
+    {
+      ProfScope prof(s, silu_mul ? "tc_w4a4_gate_up_partial" : "tc_w4a4_partial");
+      e = launch(tc_w4a4_kernel<kEpiPartial>, kEpiPartial);
+    }
+    if (e != cudaSuccess) return e;
+    const int64_t total = m * a.t.n_out;
+    ProfScope prof(s, silu_mul ? "splitk_reduce_silu_mul" : "splitk_reduce");
+    if (silu_mul)
+      splitk_reduce_kernel<true><<<(unsigned)((total + 255) / 256), 256, 0, s>>>(
+          (const float*)partials, p.splits, (int)m, p.n_pad, a.t.n_out, w.gs, (uint16_t*)y, a.t.ldo);
+    else
+      splitk_reduce_kernel<false><<<(unsigned)((total + 255) / 256), 256, 0, s>>>(
+          (const float*)partials, p.splits, (int)m, p.n_pad, a.t.n_out, w.gs, (uint16_t*)y, a.t.ldo);
+    return cudaGetLastError();
+  }
+  a.t.out = y;
+  ProfScope prof(s, silu_mul ? "tc_w4a4_gate_up_silu" : "tc_w4a4");
+  return silu_mul ? launch(tc_w4a4_kernel<kEpiSiluMul>, kEpiSiluMul)
+                  : launch(tc_w4a4_kernel<kEpiStore>, kEpiStore);
 }
 
 cudaError_t read_device_error(int* flags, bool clear) {

@@ -190,8 +190,9 @@ def test_ffn_tile_edges(native, m, H, I):
     assert native.ffn_nvfp4_device_error() == 0
 
 
-def test_gemv_path_matches_oracle_in_subprocess(native):
-    # the CUDA-core projection family, selected per process by environment
+@pytest.mark.parametrize("env,fmt", [("FFN_NVFP4_W4A16_PATH", "bf16"), ("FFN_NVFP4_W4A4_PATH", "nvfp4_fixed")])
+def test_cuda_core_paths_match_oracle_in_subprocess(native, env, fmt):
+    # the CUDA-core projection families, selected per process by environment
     import os
     import subprocess
     import sys
@@ -200,12 +201,12 @@ def test_gemv_path_matches_oracle_in_subprocess(native):
         "from gpu_helpers import FfnCase, assert_close, bf16_to_f64;"
         "from nvfp4_quantized_dense_w4a16_b200 import native as N, synth;"
         "c = FfnCase(N, synth.make_inputs('smallm', m=5, hidden=512, inter=1536, seed=3));"
-        "assert_close(bf16_to_f64(c.forward('bf16')), c.oracle('bf16'));"
+        f"assert_close(bf16_to_f64(c.forward('{fmt}')), c.oracle('{fmt}'));"
         "print('gemv-ok')")
-    env = dict(os.environ, FFN_NVFP4_W4A16_PATH="gemv")
+    env_vars = dict(os.environ, **{env: "gemv"})
     root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
-    r = subprocess.run([sys.executable, "-c", code], cwd=root, env=env, capture_output=True, text=True,
-                       timeout=600)
+    r = subprocess.run([sys.executable, "-c", code], cwd=root, env=env_vars, capture_output=True,
+                       text=True, timeout=600)
     assert r.returncode == 0 and "gemv-ok" in r.stdout, r.stdout + r.stderr
 
 
