@@ -84,6 +84,11 @@ struct TcArgs {
   const float* gs;     // tensor scale(s)
   void* out;           // bf16 [m, ldo] or fp32 partials [splits][m][n_pad]
   int m, n_out, ldo, kc_total, kc_per_split, n_pad;
+  // Activation rows one TMA box carries: min(m, tile rows).  Boxes never
+  // extend past row m (no zero fill); shared-memory rows beyond them keep
+  // stale data, which only reaches accumulator columns of rows >= m -- MMA
+  // columns are independent and those columns are never stored.
+  int x_box_rows;
 };
 
 __device__ __forceinline__ uint32_t bmul2(uint32_t a, uint32_t b) {
@@ -325,7 +330,7 @@ tc_w4a16_kernel(const __grid_constant__ CUtensorMap xmap, const TcArgs a) {
       for (int i = 0; i < nk; ++i) {
         const int s = i % SX;
         if (i >= SX && !mbar_wait(&xempty[s], ((i / SX) - 1) & 1, abort_flag, err, 1)) break;
-        mbar_arrive_expect_tx(&xfull[s], C::kXStageBytes);
+        mbar_arrive_expect_tx(&xfull[s], a.x_box_rows * 128);
         tma_load_2d(xs + s * C::kXStageBytes, &xmap, (kc0 + i) * kChunkK, xtile * BN, &xfull[s]);
         ++issued;
       }
@@ -515,7 +520,7 @@ tc_w4a4_kernel(const __grid_constant__ CUtensorMap xmap, const W4Args w4) {
         const int nch = min(kW4Chunks, nk - kW4Chunks * i);
         if (i >= kW4Stages && !mbar_wait(&empty[s], ((i / kW4Stages) - 1) & 1, abort_flag, err, 1)) break;
         uint8_t* st = smem + s * C::kStageBytes;
-        mbar_arrive_expect_tx(&full[s], nch * (kChunkBytes + 512) + C::kXBytes);
+        mbar_arrive_expect_tx(&full[s], nch * (kChunkBytes + 512) + a.x_box_rows * 128);
         bulk_load(st, wsrc + (size_t)kW4Chunks * i * kChunkBytes, nch * kChunkBytes, &full[s]);
         tma_load_2d(st + C::kWBytes, &xmap, 32 * (kc0 + kW4Chunks * i), xtile * kW4BN, &full[s]);
         bulk_load(st + C::kWBytes + C::kXBytes, ssrc + (size_t)kW4Chunks * i * 512, nch * 512, &full[s]);
@@ -729,8 +734,10 @@ TcPlan plan_tc(int64_t m, int64_t n, int64_t k, bool gate_up, int num_sms) {
 cudaError_t launch_tc_w4a16(const void* x, int64_t m, const TcWeight& w, bool silu_mul,
                             const TcPlan& p, void* y, void* partials, cudaStream_t s) {
   CUtensorMap map;
-  if (!make_x_map(&map, x, m, w.k, p.bn)) return cudaErrorInvalidValue;
+  const int box_rows = (int)(m < p.bn ? m : p.bn);
+  if (!make_x_map(&map, x, m, w.k, box_rows)) return cudaErrorInvalidValue;
   TcArgs a;
+  a.x_box_rows = box_rows;
   a.wt = w.tiled;
   a.gs = w.gs;
   a.m = (int)m;
@@ -796,7 +803,7 @@ cudaError_t launch_tc_w4a4(const uint8_t* xcodes, const uint8_t* xsf_blocks, int
   {
     cuuint64_t dims[2] = {(cuuint64_t)(w.k / 2), (cuuint64_t)m};
     cuuint64_t strides[1] = {(cuuint64_t)(w.k / 2)};
-    cuuint32_t box[2] = {128, (cuuint32_t)kW4BN};
+    cuuint32_t box[2] = {128, (cuuint32_t)(m < kW4BN ? m : kW4BN)};
     cuuint32_t estr[2] = {1, 1};
     if (enc(&map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t*>(xcodes), dims, strides, box,
             estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
@@ -804,6 +811,7 @@ cudaError_t launch_tc_w4a4(const uint8_t* xcodes, const uint8_t* xsf_blocks, int
       return cudaErrorInvalidValue;
   }
   W4Args a;
+  a.t.x_box_rows = (int)(m < kW4BN ? m : kW4BN);
   a.t.wt = w.tiled;
   a.t.gs = w.gs;
   a.t.m = (int)m;
