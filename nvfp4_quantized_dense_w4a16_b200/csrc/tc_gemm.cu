@@ -49,20 +49,21 @@ constexpr int kChunkBytes = 4608;  // 128 x (16 + 16 + 4) bytes
 
 enum : int { kEpiStore = 0, kEpiSiluMul = 1, kEpiPartial = 2 };
 
-// Pipeline shape: activation ring of SX stages (released when the MMA that
-// read it completes), weight ring of SW stages (released as soon as the
-// dequant warps have read it), SA tensor-memory stages for the dequantised
-// weights, DQG dequant warpgroups (each dequantises 64 / DQG elements of every
-// row of a chunk).
-template <int BN, int SX, int SW, int SA, int DQG>
+// Pipeline shape: activation ring of SX chunk stages (released when the MMA
+// that read it completes), weight ring of SW chunk stages (released as soon as
+// the dequant warps have read it), SA tensor-memory slots of U chunks each for
+// the dequantised weights, DQG dequant warpgroups.  Work is handed out in
+// units of U consecutive chunks; unit u belongs to warpgroup u % DQG, whose
+// four warps (one per TMEM lane quarter) dequantise all 128 rows of its
+// chunks -- so each synchronisation covers U whole chunks of a warpgroup and
+// the two warpgroups never wait for each other.
+template <int BN, int SX, int SW, int SA, int DQG, int U>
 struct TcCfg {
   static constexpr int kThreads = 128 + 128 * DQG;
   static constexpr int kXStageBytes = BN * 128;
-  // Independent accumulators: narrow tiles rotate their K steps over several
-  // accumulators so that consecutive MMAs do not wait on each other's result.
-  static constexpr int kNacc = BN <= 32 ? 4 : BN <= 64 ? 2 : 1;
-  static constexpr int kAColBase = kNacc * BN < 32 ? 32 : kNacc * BN;  // TMEM column of A stage 0
-  static constexpr int kTmemNeed = kAColBase + 32 * SA;
+  static constexpr int kAColBase = BN < 32 ? 32 : BN;  // TMEM column of A slot 0
+  static constexpr int kSlotCols = 32 * U;
+  static constexpr int kTmemNeed = kAColBase + kSlotCols * SA;
   static constexpr int kTmemCols = kTmemNeed <= 64 ? 64 : kTmemNeed <= 128 ? 128 : kTmemNeed <= 256 ? 256 : 512;
   static constexpr int kEpiBytes = 16384;  // per dequant warpgroup
   static constexpr int kSmemW = SX * kXStageBytes;
@@ -77,6 +78,7 @@ struct TcCfg {
   static_assert(kSmemAlloc <= 232448, "shared memory budget");
   static_assert(BN % 16 == 0 && BN >= 16 && BN <= 256, "MMA N");
   static_assert(DQG == 1 || DQG == 2, "dequant warpgroups");
+  static_assert(SW >= 2 * U, "weight ring must hold a unit");
 };
 
 struct TcArgs {
@@ -253,11 +255,11 @@ __device__ __forceinline__ void epilogue_tile(const TcArgs& a, uint32_t tmem, in
   }
 }
 
-template <int BN, int SX, int SW, int SA, int DQG, int EPI>
-__global__ void __launch_bounds__(TcCfg<BN, SX, SW, SA, DQG>::kThreads,
-                                  TcCfg<BN, SX, SW, SA, DQG>::kMinBlocks)
+template <int BN, int SX, int SW, int SA, int DQG, int U, int EPI>
+__global__ void __launch_bounds__(TcCfg<BN, SX, SW, SA, DQG, U>::kThreads,
+                                  TcCfg<BN, SX, SW, SA, DQG, U>::kMinBlocks)
 tc_w4a16_kernel(const __grid_constant__ CUtensorMap xmap, const TcArgs a) {
-  using C = TcCfg<BN, SX, SW, SA, DQG>;
+  using C = TcCfg<BN, SX, SW, SA, DQG, U>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
@@ -274,7 +276,6 @@ tc_w4a16_kernel(const __grid_constant__ CUtensorMap xmap, const TcArgs a) {
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(accum + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   int* err = &g_ffn_device_error;
-  constexpr int kDqWarps = 4 * DQG;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int xtile = blockIdx.x, wtile = blockIdx.y;
@@ -288,10 +289,10 @@ tc_w4a16_kernel(const __grid_constant__ CUtensorMap xmap, const TcArgs a) {
     }
     for (int s = 0; s < SW; ++s) {
       mbar_init(&wfull[s], 1);
-      mbar_init(&wempty[s], kDqWarps);
+      mbar_init(&wempty[s], 4);  // the four warps of the owning warpgroup
     }
     for (int s = 0; s < SA; ++s) {
-      mbar_init(&afull[s], kDqWarps);
+      mbar_init(&afull[s], 4);
       mbar_init(&aempty[s], 1);
     }
     mbar_init(accum, 1);
@@ -340,19 +341,25 @@ tc_w4a16_kernel(const __grid_constant__ CUtensorMap xmap, const TcArgs a) {
     // ------------------------------------------------------- MMA issuer
     if (lane == 0) {
       const uint32_t idesc = idesc_bf16_f32(kTileRows, BN);
-      for (int i = 0; i < nk; ++i) {
-        const int sa = i % SA, sx = i % SX;
-        if (!mbar_wait(&afull[sa], (i / SA) & 1, abort_flag, err, 2)) break;
-        if (!mbar_wait(&xfull[sx], (i / SX) & 1, abort_flag, err, 2)) break;
+      const int nunits = (nk + U - 1) / U;
+      bool ok = true;
+      for (int u = 0; u < nunits && ok; ++u) {
+        const int sa = u % SA;
+        if (!mbar_wait(&afull[sa], (u / SA) & 1, abort_flag, err, 2)) break;
         tc_fence_after();
-        const uint32_t a_base = tmem + C::kAColBase + 32 * sa;
-        const uint64_t b_base = smem_desc_sw128(smem_u32(xs + sx * C::kXStageBytes));
+        const int nc = min(U, nk - u * U);
+        for (int c = 0; c < nc; ++c) {
+          const int i = u * U + c, sx = i % SX;
+          if (!mbar_wait(&xfull[sx], (i / SX) & 1, abort_flag, err, 2)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t a_base = tmem + C::kAColBase + C::kSlotCols * sa + 32 * c;
+          const uint64_t b_base = smem_desc_sw128(smem_u32(xs + sx * C::kXStageBytes));
 #pragma unroll
-        for (int kk = 0; kk < 4; ++kk)
-          mma_bf16_ts(tmem + (kk % C::kNacc) * BN, a_base + 8 * kk, b_base + 2 * kk, idesc,
-                      (i > 0 || kk >= C::kNacc) ? 1u : 0u);
+          for (int kk = 0; kk < 4; ++kk)
+            mma_bf16_ts(tmem, a_base + 8 * kk, b_base + 2 * kk, idesc, (i | kk) != 0 ? 1u : 0u);
+          mma_commit(&xempty[sx]);
+        }
         mma_commit(&aempty[sa]);
-        mma_commit(&xempty[sx]);
       }
       mma_commit(accum);  // fires once every MMA issued above has completed
     }
@@ -363,59 +370,40 @@ tc_w4a16_kernel(const __grid_constant__ CUtensorMap xmap, const TcArgs a) {
     const int row = 32 * q + lane;                // tile row == TMEM lane
     const uint32_t lane_addr = (uint32_t)(32 * q) << 16;
     const int sf_off = 16 * lane + 4 * q;         // this row's 4 scale bytes (block layout)
-    // The store of chunk i is completed (wait::st, then the MMA is told) only
-    // after chunk i+1 has been dequantised, so the TMEM store latency overlaps
-    // the next chunk's arithmetic.
-    bool pending = false;
-    int pending_sa = 0;
-    for (int i = 0; i < nk; ++i) {
-      const int s = i % SW, sa = i % SA;
-      bool ok = mbar_wait(&wfull[s], (i / SW) & 1, abort_flag, err, 4);
-      if (!__all_sync(0xffffffffu, ok)) break;  // keep the warp converged for tcgen05.st
-      const uint8_t* w = wsm + s * kChunkBytes;
-      uint32_t v[64 / DQG / 2];
-      if constexpr (DQG == 1) {
-        const uint4 lo = *reinterpret_cast<const uint4*>(w + 16 * row);
-        const uint4 hi = *reinterpret_cast<const uint4*>(w + 2048 + 16 * row);
-        const uint32_t sc = *reinterpret_cast<const uint32_t*>(w + 4096 + sf_off);
-        dequant64(lo, hi, sc, *reinterpret_cast<uint32_t(*)[32]>(v));
-      } else {
-        const uint4 c = *reinterpret_cast<const uint4*>(w + 2048 * g + 16 * row);
-        const uint32_t sc = *reinterpret_cast<const uint16_t*>(w + 4096 + sf_off + 2 * g);
-        dequant32(c, sc, *reinterpret_cast<uint32_t(*)[16]>(v));
-      }
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&wempty[s]);   // the shared-memory slot may be refilled
-      if (pending) {
-        tmem_st_wait();
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&afull[pending_sa]);
-        pending = false;
-      }
-      if (i >= SA) {
-        ok = mbar_wait(&aempty[sa], ((i / SA) - 1) & 1, abort_flag, err, 4);
+    const int nunits = (nk + U - 1) / U;
+    for (int u = g; u < nunits; u += DQG) {
+      const int sa = u % SA;
+      if (u >= SA) {  // the MMA that read this TMEM slot U*SA chunks ago is done
+        const bool ok = mbar_wait(&aempty[sa], ((u / SA) - 1) & 1, abort_flag, err, 4);
         if (!__all_sync(0xffffffffu, ok)) break;
         tc_fence_after();
       }
-      const uint32_t taddr = tmem + lane_addr + C::kAColBase + 32 * sa + (64 / DQG / 2) * g;
-      if constexpr (DQG == 1)
-        tmem_st32(taddr, *reinterpret_cast<uint32_t(*)[32]>(v));
-      else
-        tmem_st16(taddr, *reinterpret_cast<uint32_t(*)[16]>(v));
-      pending = true;
-      pending_sa = sa;
-    }
-    if (pending) {
+      const int nc = min(U, nk - u * U);
+      bool ok = true;
+      for (int c = 0; c < nc; ++c) {
+        const int i = u * U + c, s = i % SW;
+        ok = mbar_wait(&wfull[s], (i / SW) & 1, abort_flag, err, 4);
+        if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }  // stay converged for tcgen05.st
+        const uint8_t* w = wsm + s * kChunkBytes;
+        const uint4 lo = *reinterpret_cast<const uint4*>(w + 16 * row);
+        const uint4 hi = *reinterpret_cast<const uint4*>(w + 2048 + 16 * row);
+        const uint32_t sc = *reinterpret_cast<const uint32_t*>(w + 4096 + sf_off);
+        uint32_t v[32];
+        dequant64(lo, hi, sc, v);
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&wempty[s]);   // the shared-memory slot may be refilled
+        tmem_st32(tmem + lane_addr + C::kAColBase + C::kSlotCols * sa + 32 * c, v);
+      }
+      if (!ok) break;
       tmem_st_wait();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&afull[pending_sa]);
+      if (lane == 0) mbar_arrive(&afull[sa]);
     }
     const bool done = __all_sync(0xffffffffu, wait_drain(accum, 0));
     tc_fence_after();
     if (done && !*abort_flag)
-      epilogue_tile<BN, EPI, DQG, C::kNacc>(a, tmem, q, lane, g, epi + g * C::kEpiBytes, xtile, wtile);
+      epilogue_tile<BN, EPI, DQG>(a, tmem, q, lane, g, epi + g * C::kEpiBytes, xtile, wtile);
   }
   tc_fence_before();
   __syncthreads();
@@ -662,10 +650,10 @@ bool make_x_map(CUtensorMap* map, const void* x, int64_t m, int64_t k, int box_r
              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int BN, int SX, int SW, int SA, int DQG, int EPI>
+template <int BN, int SX, int SW, int SA, int DQG, int U, int EPI>
 cudaError_t launch_cfg(const CUtensorMap& map, const TcArgs& a, dim3 grid, cudaStream_t s) {
-  using C = TcCfg<BN, SX, SW, SA, DQG>;
-  auto kern = tc_w4a16_kernel<BN, SX, SW, SA, DQG, EPI>;
+  using C = TcCfg<BN, SX, SW, SA, DQG, U>;
+  auto kern = tc_w4a16_kernel<BN, SX, SW, SA, DQG, U, EPI>;
   static bool attr_set = false;  // per instantiation; idempotent if raced
   if (!attr_set) {
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemAlloc);
@@ -679,12 +667,12 @@ cudaError_t launch_cfg(const CUtensorMap& map, const TcArgs& a, dim3 grid, cudaS
 template <int EPI>
 cudaError_t launch_bn(int bn, const CUtensorMap& map, const TcArgs& a, dim3 grid, cudaStream_t s) {
   switch (bn) {
-    // BN, activation stages, weight stages, TMEM stages, dequant warpgroups
-    case 16: return launch_cfg<16, 6, 12, 4, 2, EPI>(map, a, grid, s);
-    case 32: return launch_cfg<32, 6, 12, 4, 2, EPI>(map, a, grid, s);
-    case 64: return launch_cfg<64, 4, 10, 4, 2, EPI>(map, a, grid, s);
-    case 128: return launch_cfg<128, 6, 10, 4, 2, EPI>(map, a, grid, s);
-    default: return launch_cfg<256, 4, 8, 4, 2, EPI>(map, a, grid, s);
+    // BN, activation stages, weight stages, TMEM slots, dequant warpgroups, chunks per unit
+    case 16: return launch_cfg<16, 8, 12, 3, 2, 2, EPI>(map, a, grid, s);
+    case 32: return launch_cfg<32, 6, 12, 3, 2, 2, EPI>(map, a, grid, s);
+    case 64: return launch_cfg<64, 4, 10, 3, 2, 2, EPI>(map, a, grid, s);
+    case 128: return launch_cfg<128, 6, 10, 4, 2, 1, EPI>(map, a, grid, s);
+    default: return launch_cfg<256, 4, 8, 4, 2, 1, EPI>(map, a, grid, s);
   }
 }
 
