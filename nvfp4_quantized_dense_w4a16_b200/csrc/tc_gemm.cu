@@ -57,11 +57,15 @@ enum : int { kEpiStore = 0, kEpiSiluMul = 1, kEpiPartial = 2 };
 // four warps (one per TMEM lane quarter) dequantise all 128 rows of its
 // chunks -- so each synchronisation covers U whole chunks of a warpgroup and
 // the two warpgroups never wait for each other.
-template <int BN, int SX, int SW, int SA, int DQG, int U>
+template <int BN, int SX, int SW, int SA, int DQG, int U, int NACC>
 struct TcCfg {
   static constexpr int kThreads = 128 + 128 * DQG;
   static constexpr int kXStageBytes = BN * 128;
-  static constexpr int kAColBase = BN < 32 ? 32 : BN;  // TMEM column of A slot 0
+  // NACC independent accumulators: the K steps of a chunk rotate over them, so
+  // that narrow MMAs (whose duration is below the tensor core's accumulate
+  // latency) do not form one serial dependency chain; the epilogue adds them.
+  static constexpr int kNacc = NACC;
+  static constexpr int kAColBase = NACC * BN < 32 ? 32 : NACC * BN;  // TMEM column of A slot 0
   static constexpr int kSlotCols = 32 * U;
   static constexpr int kTmemNeed = kAColBase + kSlotCols * SA;
   static constexpr int kTmemCols = kTmemNeed <= 64 ? 64 : kTmemNeed <= 128 ? 128 : kTmemNeed <= 256 ? 256 : 512;
@@ -255,11 +259,11 @@ __device__ __forceinline__ void epilogue_tile(const TcArgs& a, uint32_t tmem, in
   }
 }
 
-template <int BN, int SX, int SW, int SA, int DQG, int U, int EPI>
-__global__ void __launch_bounds__(TcCfg<BN, SX, SW, SA, DQG, U>::kThreads,
-                                  TcCfg<BN, SX, SW, SA, DQG, U>::kMinBlocks)
+template <int BN, int SX, int SW, int SA, int DQG, int U, int NACC, int EPI>
+__global__ void __launch_bounds__(TcCfg<BN, SX, SW, SA, DQG, U, NACC>::kThreads,
+                                  TcCfg<BN, SX, SW, SA, DQG, U, NACC>::kMinBlocks)
 tc_w4a16_kernel(const __grid_constant__ CUtensorMap xmap, const TcArgs a) {
-  using C = TcCfg<BN, SX, SW, SA, DQG, U>;
+  using C = TcCfg<BN, SX, SW, SA, DQG, U, NACC>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
@@ -356,7 +360,8 @@ tc_w4a16_kernel(const __grid_constant__ CUtensorMap xmap, const TcArgs a) {
           const uint64_t b_base = smem_desc_sw128(smem_u32(xs + sx * C::kXStageBytes));
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk)
-            mma_bf16_ts(tmem, a_base + 8 * kk, b_base + 2 * kk, idesc, (i | kk) != 0 ? 1u : 0u);
+            mma_bf16_ts(tmem + (kk % NACC) * BN, a_base + 8 * kk, b_base + 2 * kk, idesc,
+                        (i > 0 || kk >= NACC) ? 1u : 0u);
           mma_commit(&xempty[sx]);
         }
         mma_commit(&aempty[sa]);
@@ -403,7 +408,7 @@ tc_w4a16_kernel(const __grid_constant__ CUtensorMap xmap, const TcArgs a) {
     const bool done = __all_sync(0xffffffffu, wait_drain(accum, 0));
     tc_fence_after();
     if (done && !*abort_flag)
-      epilogue_tile<BN, EPI, DQG>(a, tmem, q, lane, g, epi + g * C::kEpiBytes, xtile, wtile);
+      epilogue_tile<BN, EPI, DQG, NACC>(a, tmem, q, lane, g, epi + g * C::kEpiBytes, xtile, wtile);
   }
   tc_fence_before();
   __syncthreads();
@@ -650,10 +655,10 @@ bool make_x_map(CUtensorMap* map, const void* x, int64_t m, int64_t k, int box_r
              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int BN, int SX, int SW, int SA, int DQG, int U, int EPI>
+template <int BN, int SX, int SW, int SA, int DQG, int U, int NACC, int EPI>
 cudaError_t launch_cfg(const CUtensorMap& map, const TcArgs& a, dim3 grid, cudaStream_t s) {
-  using C = TcCfg<BN, SX, SW, SA, DQG, U>;
-  auto kern = tc_w4a16_kernel<BN, SX, SW, SA, DQG, U, EPI>;
+  using C = TcCfg<BN, SX, SW, SA, DQG, U, NACC>;
+  auto kern = tc_w4a16_kernel<BN, SX, SW, SA, DQG, U, NACC, EPI>;
   static bool attr_set = false;  // per instantiation; idempotent if raced
   if (!attr_set) {
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemAlloc);
@@ -667,12 +672,13 @@ cudaError_t launch_cfg(const CUtensorMap& map, const TcArgs& a, dim3 grid, cudaS
 template <int EPI>
 cudaError_t launch_bn(int bn, const CUtensorMap& map, const TcArgs& a, dim3 grid, cudaStream_t s) {
   switch (bn) {
-    // BN, activation stages, weight stages, TMEM slots, dequant warpgroups, chunks per unit
-    case 16: return launch_cfg<16, 8, 12, 3, 2, 2, EPI>(map, a, grid, s);
-    case 32: return launch_cfg<32, 6, 12, 3, 2, 2, EPI>(map, a, grid, s);
-    case 64: return launch_cfg<64, 4, 10, 3, 2, 2, EPI>(map, a, grid, s);
-    case 128: return launch_cfg<128, 6, 10, 4, 2, 1, EPI>(map, a, grid, s);
-    default: return launch_cfg<256, 4, 8, 4, 2, 1, EPI>(map, a, grid, s);
+    // BN, activation stages, weight stages, TMEM slots, dequant warpgroups, chunks per
+    // unit, accumulators (TMEM: NACC*BN + 32*U*SA columns, 256 for two CTAs per SM)
+    case 16: return launch_cfg<16, 8, 12, 3, 2, 2, 4, EPI>(map, a, grid, s);
+    case 32: return launch_cfg<32, 6, 12, 3, 2, 2, 2, EPI>(map, a, grid, s);
+    case 64: return launch_cfg<64, 4, 10, 2, 2, 2, 2, EPI>(map, a, grid, s);
+    case 128: return launch_cfg<128, 6, 10, 4, 2, 1, 1, EPI>(map, a, grid, s);
+    default: return launch_cfg<256, 4, 8, 4, 2, 1, 1, EPI>(map, a, grid, s);
   }
 }
 
