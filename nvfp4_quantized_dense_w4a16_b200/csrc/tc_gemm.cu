@@ -49,31 +49,34 @@ constexpr int kChunkBytes = 4608;  // 128 x (16 + 16 + 4) bytes
 
 enum : int { kEpiStore = 0, kEpiSiluMul = 1, kEpiPartial = 2 };
 
-// Pipeline shape: activation ring of SX chunk stages (released when the MMA
-// that read it completes), weight ring of SW chunk stages (released as soon as
-// the dequant warps have read it), SA tensor-memory slots of U chunks each for
-// the dequantised weights, DQG dequant warpgroups.  Work is handed out in
-// units of U consecutive chunks; unit u belongs to warpgroup u % DQG, whose
-// four warps (one per TMEM lane quarter) dequantise all 128 rows of its
-// chunks -- so each synchronisation covers U whole chunks of a warpgroup and
-// the two warpgroups never wait for each other.
-template <int BN, int SX, int SW, int SA, int DQG, int U, int NACC>
+// Pipeline shape.  Work is handed out in units of U consecutive 64-element
+// chunks; every ring holds whole units: SXU activation stages (released when
+// the MMAs that read them complete), SWU weight stages (released as soon as
+// the dequant warps have read them) and SA tensor-memory slots for the
+// dequantised weights.  Unit u belongs to dequant warpgroup u % DQG, whose
+// four warps (one per TMEM lane quarter) dequantise all 128 rows of its chunks
+// and also observe the unit's activation barrier, so the MMA thread waits on
+// one barrier per unit.  NI threads issue MMAs (unit u -> issuer u % NI), each
+// into its own accumulator; the epilogue adds the accumulators.  Every
+// mbarrier wait and tcgen05 fence costs ~0.1 us even when nothing is pending,
+// which is why waits are per unit and narrow tiles use two issuers.
+template <int BN, int SXU, int SWU, int SA, int DQG, int U, int NI>
 struct TcCfg {
   static constexpr int kThreads = 128 + 128 * DQG;
-  static constexpr int kXStageBytes = BN * 128;
-  // NACC independent accumulators: the K steps of a chunk rotate over them, so
-  // that narrow MMAs (whose duration is below the tensor core's accumulate
-  // latency) do not form one serial dependency chain; the epilogue adds them.
-  static constexpr int kNacc = NACC;
-  static constexpr int kAColBase = NACC * BN < 32 ? 32 : NACC * BN;  // TMEM column of A slot 0
+  static constexpr int kXStageBytes = U * BN * 128;    // U chunk tiles of BN rows x 128 B
+  static constexpr int kWStageBytes = U * kChunkBytes;
+  static constexpr int kAColBase = NI * BN < 32 ? 32 : NI * BN;  // TMEM column of A slot 0
   static constexpr int kSlotCols = 32 * U;
   static constexpr int kTmemNeed = kAColBase + kSlotCols * SA;
   static constexpr int kTmemCols = kTmemNeed <= 64 ? 64 : kTmemNeed <= 128 ? 128 : kTmemNeed <= 256 ? 256 : 512;
-  static constexpr int kEpiBytes = 16384;  // per dequant warpgroup
-  static constexpr int kSmemW = SX * kXStageBytes;
-  static constexpr int kSmemEpi = kSmemW + SW * kChunkBytes;
-  static constexpr int kSmemBar = kSmemEpi + DQG * kEpiBytes;
-  static constexpr int kNumBars = 2 * SX + 2 * SW + 2 * SA + 1;
+  // The epilogue staging buffers (16 KB per dequant warpgroup) reuse the start
+  // of the rings: the epilogue runs after every MMA has completed, and those
+  // MMAs consumed every copy the producers issued.
+  static constexpr int kEpiBytes = 16384;
+  static constexpr int kSmemW = SXU * kXStageBytes;
+  static constexpr int kSmemRings = kSmemW + SWU * kWStageBytes;
+  static constexpr int kSmemBar = kSmemRings;
+  static constexpr int kNumBars = 2 * SXU + 2 * SWU + 2 * SA + NI;
   static constexpr int kSmemBytes = kSmemBar + kNumBars * 8 + 16;
   static constexpr int kSmemAlloc = kSmemBytes + 1024;  // slack for 1024-byte alignment
   // two CTAs per SM when both fit (228 KB of shared memory, 512 TMEM columns)
@@ -82,7 +85,18 @@ struct TcCfg {
   static_assert(kSmemAlloc <= 232448, "shared memory budget");
   static_assert(BN % 16 == 0 && BN >= 16 && BN <= 256, "MMA N");
   static_assert(DQG == 1 || DQG == 2, "dequant warpgroups");
-  static_assert(SW >= 2 * U, "weight ring must hold a unit");
+  static_assert(NI == 1 || (NI == 2 && DQG == 2), "MMA issuers pair with warpgroups");
+  static_assert(kSmemRings >= DQG * kEpiBytes, "epilogue buffers alias the rings");
+  // A parity wait can only tell the awaited phase from the one before it, so
+  // the previous phase must be known complete when a thread starts waiting.
+  // With one issuer the MMAs complete in unit order, which covers every ring
+  // whose depth is >= SA.  With two, each TMEM slot must stay with one
+  // warpgroup/issuer pair (SA == DQG); a weight (activation) stage either does
+  // too (even depth) or is deep enough that the sequential activation
+  // producer's progress implies it (depth >= DQG + SXU).
+  static_assert(NI == 1 ? (SWU >= SA && SXU >= SA)
+                        : (SA == DQG && (SWU % 2 == 0 || SWU >= DQG + SXU) && SXU % 2 == 0),
+                "ring depths");
 };
 
 struct TcArgs {
@@ -181,7 +195,8 @@ __device__ __forceinline__ bool wait_drain(uint64_t* bar, uint32_t parity) {
 // 16 KB per warpgroup) so that global writes are 16-byte and row-contiguous.
 template <int BN, int EPI, int NG, int NACC = 1>
 __device__ __forceinline__ void epilogue_tile(const TcArgs& a, uint32_t tmem, int q, int lane,
-                                              int g, uint8_t* ebuf, int xtile, int wtile) {
+                                              int g, uint8_t* ebuf, int xtile, int wtile,
+                                              int nacc_used = 1) {
   const int row = 32 * q + lane;
   const uint32_t lane_addr = (uint32_t)(32 * q) << 16;
   const int rbase = xtile * BN;
@@ -197,6 +212,7 @@ __device__ __forceinline__ void epilogue_tile(const TcArgs& a, uint32_t tmem, in
     // accumulators 1..NACC-1 hold the other K steps: add them in a fixed order
 #pragma unroll
     for (int acc = 1; acc < NACC; ++acc) {
+      if (acc >= nacc_used) break;  // an issuer that had no unit left its accumulator unwritten
 #pragma unroll
       for (int h = 0; h < 2; ++h) {
         uint32_t u[16];
@@ -259,25 +275,25 @@ __device__ __forceinline__ void epilogue_tile(const TcArgs& a, uint32_t tmem, in
   }
 }
 
-template <int BN, int SX, int SW, int SA, int DQG, int U, int NACC, int EPI>
-__global__ void __launch_bounds__(TcCfg<BN, SX, SW, SA, DQG, U, NACC>::kThreads,
-                                  TcCfg<BN, SX, SW, SA, DQG, U, NACC>::kMinBlocks)
+template <int BN, int SXU, int SWU, int SA, int DQG, int U, int NI, int EPI>
+__global__ void __launch_bounds__(TcCfg<BN, SXU, SWU, SA, DQG, U, NI>::kThreads,
+                                  TcCfg<BN, SXU, SWU, SA, DQG, U, NI>::kMinBlocks)
 tc_w4a16_kernel(const __grid_constant__ CUtensorMap xmap, const TcArgs a) {
-  using C = TcCfg<BN, SX, SW, SA, DQG, U, NACC>;
+  using C = TcCfg<BN, SXU, SWU, SA, DQG, U, NI>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
   uint8_t* xs = smem;
   uint8_t* wsm = smem + C::kSmemW;
-  uint8_t* epi = smem + C::kSmemEpi;
+  uint8_t* epi = smem;  // aliases the rings; used only after the last MMA
   uint64_t* xfull = reinterpret_cast<uint64_t*>(smem + C::kSmemBar);
-  uint64_t* xempty = xfull + SX;
-  uint64_t* wfull = xempty + SX;
-  uint64_t* wempty = wfull + SW;
-  uint64_t* afull = wempty + SW;
+  uint64_t* xempty = xfull + SXU;
+  uint64_t* wfull = xempty + SXU;
+  uint64_t* wempty = wfull + SWU;
+  uint64_t* afull = wempty + SWU;
   uint64_t* aempty = afull + SA;
   uint64_t* accum = aempty + SA;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(accum + 1);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(accum + NI);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   int* err = &g_ffn_device_error;
 
@@ -285,13 +301,14 @@ tc_w4a16_kernel(const __grid_constant__ CUtensorMap xmap, const TcArgs a) {
   const int xtile = blockIdx.x, wtile = blockIdx.y;
   const int kc0 = blockIdx.z * a.kc_per_split;
   const int nk = min(a.kc_total, kc0 + a.kc_per_split) - kc0;
+  const int nunits = (nk + U - 1) / U;
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < SX; ++s) {
+    for (int s = 0; s < SXU; ++s) {
       mbar_init(&xfull[s], 1);
       mbar_init(&xempty[s], 1);
     }
-    for (int s = 0; s < SW; ++s) {
+    for (int s = 0; s < SWU; ++s) {
       mbar_init(&wfull[s], 1);
       mbar_init(&wempty[s], 4);  // the four warps of the owning warpgroup
     }
@@ -299,7 +316,7 @@ tc_w4a16_kernel(const __grid_constant__ CUtensorMap xmap, const TcArgs a) {
       mbar_init(&afull[s], 4);
       mbar_init(&aempty[s], 1);
     }
-    mbar_init(accum, 1);
+    for (int j = 0; j < NI; ++j) mbar_init(&accum[j], 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -318,55 +335,58 @@ tc_w4a16_kernel(const __grid_constant__ CUtensorMap xmap, const TcArgs a) {
     if (lane == 0) {
       const uint8_t* wsrc = a.wt + ((size_t)wtile * a.kc_total + kc0) * kChunkBytes;
       int issued = 0;
-      for (int i = 0; i < nk; ++i) {
-        const int s = i % SW;
-        if (i >= SW && !mbar_wait(&wempty[s], ((i / SW) - 1) & 1, abort_flag, err, 1)) break;
-        mbar_arrive_expect_tx(&wfull[s], kChunkBytes);
-        bulk_load(wsm + s * kChunkBytes, wsrc + (size_t)i * kChunkBytes, kChunkBytes, &wfull[s]);
+      for (int u = 0; u < nunits; ++u) {
+        const int s = u % SWU;
+        const int nc = min(U, nk - u * U);
+        if (u >= SWU && !mbar_wait(&wempty[s], ((u / SWU) - 1) & 1, abort_flag, err, 1)) break;
+        mbar_arrive_expect_tx(&wfull[s], nc * kChunkBytes);
+        bulk_load(wsm + s * C::kWStageBytes, wsrc + (size_t)u * U * kChunkBytes, nc * kChunkBytes, &wfull[s]);
         ++issued;
       }
       // no copy into this CTA's shared memory may outlive it
-      for (int i = max(0, issued - SW); i < issued; ++i) wait_drain(&wfull[i % SW], (i / SW) & 1);
+      for (int u = max(0, issued - SWU); u < issued; ++u) wait_drain(&wfull[u % SWU], (u / SWU) & 1);
     }
   } else if (warp == 3) {
     // --------------------------------------------- activation producer
     if (lane == 0) {
       int issued = 0;
-      for (int i = 0; i < nk; ++i) {
-        const int s = i % SX;
-        if (i >= SX && !mbar_wait(&xempty[s], ((i / SX) - 1) & 1, abort_flag, err, 1)) break;
-        mbar_arrive_expect_tx(&xfull[s], a.x_box_rows * 128);
-        tma_load_2d(xs + s * C::kXStageBytes, &xmap, (kc0 + i) * kChunkK, xtile * BN, &xfull[s]);
+      for (int u = 0; u < nunits; ++u) {
+        const int s = u % SXU;
+        const int nc = min(U, nk - u * U);
+        if (u >= SXU && !mbar_wait(&xempty[s], ((u / SXU) - 1) & 1, abort_flag, err, 1)) break;
+        mbar_arrive_expect_tx(&xfull[s], nc * a.x_box_rows * 128);
+        for (int c = 0; c < nc; ++c)
+          tma_load_2d(xs + s * C::kXStageBytes + c * BN * 128, &xmap, (kc0 + u * U + c) * kChunkK,
+                      xtile * BN, &xfull[s]);
         ++issued;
       }
-      for (int i = max(0, issued - SX); i < issued; ++i) wait_drain(&xfull[i % SX], (i / SX) & 1);
+      for (int u = max(0, issued - SXU); u < issued; ++u) wait_drain(&xfull[u % SXU], (u / SXU) & 1);
     }
-  } else if (warp == 1) {
-    // ------------------------------------------------------- MMA issuer
+  } else if (warp == 1 || (NI == 2 && warp == 2)) {
+    // -------------------------------------------------- MMA issuer(s)
     if (lane == 0) {
+      const int j = warp - 1;  // issuer index: units u = j, j + NI, ...
       const uint32_t idesc = idesc_bf16_f32(kTileRows, BN);
-      const int nunits = (nk + U - 1) / U;
-      bool ok = true;
-      for (int u = 0; u < nunits && ok; ++u) {
-        const int sa = u % SA;
-        if (!mbar_wait(&afull[sa], (u / SA) & 1, abort_flag, err, 2)) break;
+      const uint32_t d = tmem + j * BN;  // this issuer's accumulator
+      bool first = true;
+      for (int u = j; u < nunits; u += NI) {
+        const int sa = u % SA, sx = u % SXU;
+        if (!mbar_wait(&afull[sa], (u / SA) & 1, abort_flag, err, 2)) break;  // A and x both ready
         tc_fence_after();
         const int nc = min(U, nk - u * U);
+        const uint64_t b_stage = smem_desc_sw128(smem_u32(xs + sx * C::kXStageBytes));
         for (int c = 0; c < nc; ++c) {
-          const int i = u * U + c, sx = i % SX;
-          if (!mbar_wait(&xfull[sx], (i / SX) & 1, abort_flag, err, 2)) { ok = false; break; }
-          tc_fence_after();
           const uint32_t a_base = tmem + C::kAColBase + C::kSlotCols * sa + 32 * c;
-          const uint64_t b_base = smem_desc_sw128(smem_u32(xs + sx * C::kXStageBytes));
+          const uint64_t b_base = b_stage + (uint64_t)((c * BN * 128) >> 4);
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk)
-            mma_bf16_ts(tmem + (kk % NACC) * BN, a_base + 8 * kk, b_base + 2 * kk, idesc,
-                        (i > 0 || kk >= NACC) ? 1u : 0u);
-          mma_commit(&xempty[sx]);
+            mma_bf16_ts(d, a_base + 8 * kk, b_base + 2 * kk, idesc, (first && kk == 0) ? 0u : 1u);
+          first = false;
         }
         mma_commit(&aempty[sa]);
+        mma_commit(&xempty[sx]);
       }
-      mma_commit(accum);  // fires once every MMA issued above has completed
+      mma_commit(&accum[j]);  // fires once every MMA this thread issued has completed
     }
   } else if (warp >= 4) {
     // ------------------------------------------- dequant, then epilogue
@@ -375,40 +395,42 @@ tc_w4a16_kernel(const __grid_constant__ CUtensorMap xmap, const TcArgs a) {
     const int row = 32 * q + lane;                // tile row == TMEM lane
     const uint32_t lane_addr = (uint32_t)(32 * q) << 16;
     const int sf_off = 16 * lane + 4 * q;         // this row's 4 scale bytes (block layout)
-    const int nunits = (nk + U - 1) / U;
     for (int u = g; u < nunits; u += DQG) {
-      const int sa = u % SA;
-      if (u >= SA) {  // the MMA that read this TMEM slot U*SA chunks ago is done
+      const int sa = u % SA, sw = u % SWU, sx = u % SXU;
+      if (u >= SA) {  // the MMAs that read this TMEM slot SA units ago are done
         const bool ok = mbar_wait(&aempty[sa], ((u / SA) - 1) & 1, abort_flag, err, 4);
         if (!__all_sync(0xffffffffu, ok)) break;
         tc_fence_after();
       }
+      bool ok = mbar_wait(&wfull[sw], (u / SWU) & 1, abort_flag, err, 4);
+      if (!__all_sync(0xffffffffu, ok)) break;  // stay converged for tcgen05.st
       const int nc = min(U, nk - u * U);
-      bool ok = true;
+      const uint8_t* wst = wsm + sw * C::kWStageBytes;
       for (int c = 0; c < nc; ++c) {
-        const int i = u * U + c, s = i % SW;
-        ok = mbar_wait(&wfull[s], (i / SW) & 1, abort_flag, err, 4);
-        if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }  // stay converged for tcgen05.st
-        const uint8_t* w = wsm + s * kChunkBytes;
+        const uint8_t* w = wst + c * kChunkBytes;
         const uint4 lo = *reinterpret_cast<const uint4*>(w + 16 * row);
         const uint4 hi = *reinterpret_cast<const uint4*>(w + 2048 + 16 * row);
         const uint32_t sc = *reinterpret_cast<const uint32_t*>(w + 4096 + sf_off);
         uint32_t v[32];
         dequant64(lo, hi, sc, v);
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&wempty[s]);   // the shared-memory slot may be refilled
         tmem_st32(tmem + lane_addr + C::kAColBase + C::kSlotCols * sa + 32 * c, v);
       }
-      if (!ok) break;
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&wempty[sw]);   // the shared-memory stage may be refilled
+      ok = mbar_wait(&xfull[sx], (u / SXU) & 1, abort_flag, err, 4);  // the unit's activations
+      if (!__all_sync(0xffffffffu, ok)) break;
       tmem_st_wait();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&afull[sa]);
     }
-    const bool done = __all_sync(0xffffffffu, wait_drain(accum, 0));
+    bool done = true;
+    for (int j = 0; j < NI; ++j) done = wait_drain(&accum[j], 0) && done;
+    done = __all_sync(0xffffffffu, done);
     tc_fence_after();
     if (done && !*abort_flag)
-      epilogue_tile<BN, EPI, DQG, NACC>(a, tmem, q, lane, g, epi + g * C::kEpiBytes, xtile, wtile);
+      epilogue_tile<BN, EPI, DQG, NI>(a, tmem, q, lane, g, epi + g * C::kEpiBytes, xtile, wtile,
+                                      min(NI, nunits));
   }
   tc_fence_before();
   __syncthreads();
@@ -470,7 +492,7 @@ tc_w4a4_kernel(const __grid_constant__ CUtensorMap xmap, const W4Args w4) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
-  uint8_t* epi = smem + C::kSmemEpi;
+  uint8_t* epi = smem;  // aliases the rings; used only after the last MMA
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::kSmemBar);
   uint64_t* empty = full + kW4Stages;
   uint64_t* accum = empty + kW4Stages;
@@ -655,10 +677,10 @@ bool make_x_map(CUtensorMap* map, const void* x, int64_t m, int64_t k, int box_r
              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int BN, int SX, int SW, int SA, int DQG, int U, int NACC, int EPI>
+template <int BN, int SXU, int SWU, int SA, int DQG, int U, int NI, int EPI>
 cudaError_t launch_cfg(const CUtensorMap& map, const TcArgs& a, dim3 grid, cudaStream_t s) {
-  using C = TcCfg<BN, SX, SW, SA, DQG, U, NACC>;
-  auto kern = tc_w4a16_kernel<BN, SX, SW, SA, DQG, U, NACC, EPI>;
+  using C = TcCfg<BN, SXU, SWU, SA, DQG, U, NI>;
+  auto kern = tc_w4a16_kernel<BN, SXU, SWU, SA, DQG, U, NI, EPI>;
   static bool attr_set = false;  // per instantiation; idempotent if raced
   if (!attr_set) {
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemAlloc);
@@ -672,13 +694,14 @@ cudaError_t launch_cfg(const CUtensorMap& map, const TcArgs& a, dim3 grid, cudaS
 template <int EPI>
 cudaError_t launch_bn(int bn, const CUtensorMap& map, const TcArgs& a, dim3 grid, cudaStream_t s) {
   switch (bn) {
-    // BN, activation stages, weight stages, TMEM slots, dequant warpgroups, chunks per
-    // unit, accumulators (TMEM: NACC*BN + 32*U*SA columns, 256 for two CTAs per SM)
-    case 16: return launch_cfg<16, 8, 12, 3, 2, 2, 4, EPI>(map, a, grid, s);
-    case 32: return launch_cfg<32, 6, 12, 3, 2, 2, 2, EPI>(map, a, grid, s);
-    case 64: return launch_cfg<64, 4, 10, 2, 2, 2, 2, EPI>(map, a, grid, s);
-    case 128: return launch_cfg<128, 6, 10, 4, 2, 1, 1, EPI>(map, a, grid, s);
-    default: return launch_cfg<256, 4, 8, 4, 2, 1, 1, EPI>(map, a, grid, s);
+    // BN, activation stages, weight stages, TMEM slots (all in units), dequant
+    // warpgroups, chunks per unit, MMA issuers.  TMEM: NI*BN + 32*U*SA columns
+    // (<= 256 for two CTAs per SM).
+    case 16: return launch_cfg<16, 4, 8, 2, 2, 2, 2, EPI>(map, a, grid, s);
+    case 32: return launch_cfg<32, 4, 8, 2, 2, 2, 2, EPI>(map, a, grid, s);
+    case 64: return launch_cfg<64, 2, 8, 2, 2, 2, 2, EPI>(map, a, grid, s);
+    case 128: return launch_cfg<128, 3, 5, 2, 2, 2, 1, EPI>(map, a, grid, s);
+    default: return launch_cfg<256, 2, 6, 2, 2, 2, 1, EPI>(map, a, grid, s);
   }
 }
 
