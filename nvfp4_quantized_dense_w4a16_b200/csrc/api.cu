@@ -18,9 +18,10 @@ struct ffn_nvfp4_weight {
   uint8_t* codes = nullptr;   // [n, k/2] canonical
   uint8_t* scales = nullptr;  // [n, k/16] canonical
   float* gs = nullptr;        // 1 float, or 2 (gate, up) for a fused handle
-  uint8_t* tiled = nullptr;   // tensor-core layout (see tc_gemm.cu)
+  uint8_t* tiled = nullptr;   // tensor-core layout (see tc_gemm.cu), natural codes
+  uint8_t* tiled16 = nullptr; // the same tiles with the W4A16 code-bit arrangement
   WeightView view() const { return WeightView{codes, scales, gs, n, k}; }
-  ffn::TcWeight tc() const { return ffn::TcWeight{tiled, gs, n, k}; }
+  ffn::TcWeight tc() const { return ffn::TcWeight{tiled, tiled16, gs, n, k}; }
 };
 
 namespace {
@@ -174,6 +175,7 @@ void free_weight(ffn_nvfp4_weight* w) {
   cudaFree(w->scales);
   cudaFree(w->gs);
   cudaFree(w->tiled);
+  cudaFree(w->tiled16);
   delete w;
 }
 
@@ -254,11 +256,14 @@ ffn_status ffn_nvfp4_weight_create(const void* codes, const void* block_scales,
   if (e == cudaSuccess)
     e = cudaMemcpyAsync(w->gs, global_scale, sizeof(float), cudaMemcpyDeviceToDevice, s);
   if (e == cudaSuccess) {
-    if ((st = alloc(&w->tiled, (size_t)ffn::tc_tiled_bytes(n, k, false)))) {
+    const size_t tb = (size_t)ffn::tc_tiled_bytes(n, k, false);
+    if ((st = alloc(&w->tiled, tb)) || (st = alloc(&w->tiled16, tb))) {
       free_weight(w);
       return st;
     }
-    e = ffn::launch_tile_weight(w->codes, w->scales, n, k, false, w->tiled, s);
+    e = ffn::launch_tile_weight(w->codes, w->scales, n, k, false, false, w->tiled, s);
+    if (e == cudaSuccess)
+      e = ffn::launch_tile_weight(w->codes, w->scales, n, k, false, true, w->tiled16, s);
   }
   if (e != cudaSuccess) {
     cudaGetLastError();
@@ -300,11 +305,14 @@ ffn_status ffn_nvfp4_weight_create_gate_up(const ffn_nvfp4_weight* gate,
   if (e == cudaSuccess) e = cudaMemcpyAsync(w->gs, gate->gs, sizeof(float), cudaMemcpyDeviceToDevice, s);
   if (e == cudaSuccess) e = cudaMemcpyAsync(w->gs + 1, up->gs, sizeof(float), cudaMemcpyDeviceToDevice, s);
   if (e == cudaSuccess) {
-    if ((st = alloc(&w->tiled, (size_t)ffn::tc_tiled_bytes(2 * I, H, true)))) {
+    const size_t tb = (size_t)ffn::tc_tiled_bytes(2 * I, H, true);
+    if ((st = alloc(&w->tiled, tb)) || (st = alloc(&w->tiled16, tb))) {
       free_weight(w);
       return st;
     }
-    e = ffn::launch_tile_weight(w->codes, w->scales, 2 * I, H, true, w->tiled, s);
+    e = ffn::launch_tile_weight(w->codes, w->scales, 2 * I, H, true, false, w->tiled, s);
+    if (e == cudaSuccess)
+      e = ffn::launch_tile_weight(w->codes, w->scales, 2 * I, H, true, true, w->tiled16, s);
   }
   if (e != cudaSuccess) {
     cudaGetLastError();

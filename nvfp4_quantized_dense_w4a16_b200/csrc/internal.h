@@ -25,7 +25,8 @@ enum class Epilogue : int {
 
 // Tensor-core (tcgen05) projection over the pre-tiled weight layout.
 struct TcWeight {
-  const uint8_t* tiled;  // [tiles][ceil(k/64)][4608]
+  const uint8_t* tiled;    // [tiles][ceil(k/64)][4608], natural codes (W4A4)
+  const uint8_t* tiled16;  // same layout, code bits rearranged for the W4A16 decode
   const float* gs;       // 1 or 2 device floats
   int64_t n, k;          // logical dims (n = 2*inter for a fused gate+up weight)
 };
@@ -39,7 +40,7 @@ struct TcPlan {
 TcPlan plan_tc(int64_t m, int64_t n, int64_t k, bool gate_up, int num_sms);
 int64_t tc_tiled_bytes(int64_t n, int64_t k, bool gate_up);
 cudaError_t launch_tile_weight(const uint8_t* codes, const uint8_t* scales, int64_t n, int64_t k,
-                               bool gate_up, uint8_t* out, cudaStream_t s);
+                               bool gate_up, bool for_w4a16, uint8_t* out, cudaStream_t s);
 cudaError_t launch_tc_w4a16(const void* x, int64_t m, const TcWeight& w, bool silu_mul,
                             const TcPlan& p, void* y, void* partials, cudaStream_t s);
 // Fixed-format (W4A4) projection on the block-scaled FP4 tensor core.  The

@@ -91,11 +91,11 @@ struct TcCfg {
   // the previous phase must be known complete when a thread starts waiting.
   // With one issuer the MMAs complete in unit order, which covers every ring
   // whose depth is >= SA.  With two, each TMEM slot must stay with one
-  // warpgroup/issuer pair (SA == DQG); a weight (activation) stage either does
-  // too (even depth) or is deep enough that the sequential activation
-  // producer's progress implies it (depth >= DQG + SXU).
+  // warpgroup/issuer pair (SA a multiple of DQG); a weight (activation) stage
+  // either does too (even depth) or is deep enough that the sequential
+  // activation producer's progress implies it (depth >= DQG + SXU).
   static_assert(NI == 1 ? (SWU >= SA && SXU >= SA)
-                        : (SA == DQG && (SWU % 2 == 0 || SWU >= DQG + SXU) && SXU % 2 == 0),
+                        : (SA % DQG == 0 && (SWU % 2 == 0 || SWU >= DQG + SXU) && SXU % 2 == 0),
                 "ring depths");
 };
 
@@ -117,55 +117,87 @@ __device__ __forceinline__ uint32_t bmul2(uint32_t a, uint32_t b) {
   return *reinterpret_cast<uint32_t*>(&r);
 }
 
-// E4M3 byte -> (s, s) as bf16x2 (exact: 4 significant bits, exponent 2^-9..2^8).
-__device__ __forceinline__ uint32_t scale_pair(uint32_t s8) {
-  const uint32_t b = __float_as_uint(e4m3_decode(s8)) >> 16;
-  return b | (b << 16);
+// ------------------------------------------------ W4A16 operand decoding
+//
+// The bf16-activation path streams a second copy of the weight tiles whose
+// code bits are rearranged inside every 32-bit word (eight E2M1 codes) so
+// that each bf16x2 pair of the A operand comes out of one or two rotations
+// and a mask.  The decoded half-word of a code (s, e1, e0, m) is
+//   bit 15 = s, bits 8..6 = e1 e0 m, all other bits 0,
+// which as a bf16 number is exactly the E2M1 value times 2^-126: the two
+// exponent bits land in the exponent field and m in the top mantissa bit, and
+// the e = 0 codes (0 and 0.5) become the bf16 subnormals 0 and 2^-127.  The
+// block scale is applied as the bf16 number s * 2^118 (at most 448 * 2^118 <
+// bf16 max), so every A element equals (E2M1 * s) * 2^-8 exactly, and the
+// epilogue multiplies the fp32 accumulator by gs * 2^8.
+//
+// Within a word, output pair k (elements 2k, 2k+1) is read from
+//   k = 0: c & M,  k = 1: rotr(c, 4) & M,  k = 2: rotr(c, 10) & M,
+//   k = 3: (rotr(c, 6) & MA) | (rotr(c, 14) & MB)
+// with M the eight destination bits {6,7,8,15,22,23,24,31}; these source
+// positions are disjoint and cover the word (permute_codes_w4a16 writes it).
+constexpr uint32_t kPairMask = 0x81C081C0u;
+constexpr uint32_t kPairMaskA = 0x81808180u;  // bits 7, 8, 15 of each half
+constexpr uint32_t kPairMaskB = 0x00400040u;  // bit 6 of each half
+constexpr float kW4A16Unscale = 256.0f;        // 2^8
+
+__device__ __forceinline__ uint32_t rotr32(uint32_t x, int r) { return __funnelshift_r(x, x, r); }
+
+// Source bit of destination bit p of output pair k.
+__host__ __device__ constexpr int w4a16_src_bit(int k, int p) {
+  return (p + (k == 0 ? 0 : k == 1 ? 4 : k == 2 ? 10 : ((p & 15) == 6 ? 14 : 6))) & 31;
 }
 
-// Eight E2M1 codes (nibble i = element i) times the block scale pair ->
-// four bf16x2 words (element 2j in the low half of word j).  The bf16 bytes of
-// the magnitudes {0, .5, 1, 1.5, 2, 3, 4, 6} are looked up with byte permutes:
-// high bytes {00,3F,3F,3F,40,40,40,40}, low bytes {00,00,80,C0,00,40,80,C0};
-// the sign (nibble bit 3) is moved to bit 7 of the high byte.
-__device__ __forceinline__ void dequant8(uint32_t c, uint32_t s2, uint32_t* o) {
-  const uint32_t mags = c & 0x77777777u;
-  const uint32_t m47 = mags >> 16;
-  const uint32_t c4 = c << 4;
-  uint32_t hi03 = __byte_perm(0x3F3F3F00u, 0x40404040u, mags);
-  uint32_t lo03 = __byte_perm(0xC0800000u, 0xC0804000u, mags);
-  uint32_t hi47 = __byte_perm(0x3F3F3F00u, 0x40404040u, m47);
-  uint32_t lo47 = __byte_perm(0xC0800000u, 0xC0804000u, m47);
-  hi03 |= __byte_perm(c4, c, 0x5140) & 0x80808080u;
-  hi47 |= __byte_perm(c4, c, 0x7362) & 0x80808080u;
-  o[0] = bmul2(__byte_perm(lo03, hi03, 0x5140), s2);
-  o[1] = bmul2(__byte_perm(lo03, hi03, 0x7362), s2);
-  o[2] = bmul2(__byte_perm(lo47, hi47, 0x5140), s2);
-  o[3] = bmul2(__byte_perm(lo47, hi47, 0x7362), s2);
+// Natural word (element e in bits 4e..4e+3) -> the rearranged word.
+__device__ __forceinline__ uint32_t permute_codes_w4a16(uint32_t nat) {
+  uint32_t out = 0;
+#pragma unroll
+  for (int e = 0; e < 8; ++e) {
+#pragma unroll
+    for (int b = 0; b < 4; ++b) {
+      const int p = (b == 3 ? 15 : 6 + b) + 16 * (e & 1);
+      out |= ((nat >> (4 * e + b)) & 1u) << w4a16_src_bit(e >> 1, p);
+    }
+  }
+  return out;
 }
 
-// One thread's 64-element chunk of its weight row -> 32 bf16x2 TMEM columns.
-__device__ __forceinline__ void dequant64(const uint4 lo, const uint4 hi, uint32_t sc,
-                                          uint32_t (&v)[32]) {
-  const uint32_t s0 = scale_pair(sc & 0xffu), s1 = scale_pair((sc >> 8) & 0xffu);
-  const uint32_t s2 = scale_pair((sc >> 16) & 0xffu), s3 = scale_pair(sc >> 24);
-  dequant8(lo.x, s0, v + 0);
-  dequant8(lo.y, s0, v + 4);
-  dequant8(lo.z, s1, v + 8);
-  dequant8(lo.w, s1, v + 12);
-  dequant8(hi.x, s2, v + 16);
-  dequant8(hi.y, s2, v + 20);
-  dequant8(hi.z, s3, v + 24);
-  dequant8(hi.w, s3, v + 28);
+__device__ __forceinline__ uint32_t cvt_e4m3x2_f16x2(uint32_t two) {
+  uint32_t r;
+  asm("{\n\t.reg .b16 t;\n\tcvt.u16.u32 t, %1;\n\tcvt.rn.f16x2.e4m3x2 %0, t;\n\t}" : "=r"(r) : "r"(two));
+  return r;
 }
 
-// Half a chunk (32 elements: 16 bytes of codes, two block scales) -> 16 columns.
-__device__ __forceinline__ void dequant32(const uint4 c, uint32_t sc2, uint32_t (&v)[16]) {
-  const uint32_t s0 = scale_pair(sc2 & 0xffu), s1 = scale_pair((sc2 >> 8) & 0xffu);
-  dequant8(c.x, s0, v + 0);
-  dequant8(c.y, s0, v + 4);
-  dequant8(c.z, s1, v + 8);
-  dequant8(c.w, s1, v + 12);
+// Two E4M3 scales (low byte -> low half) -> bf16 bits of s * 2^118 in each
+// half: the f16 value is exact, and shifting its bits right by 3 leaves the
+// bf16 layout with the exponent re-biased by -112; adding 230 << 7 sets the
+// bias to +118.  (A zero scale yields 2^103; its codes are zero.)
+__device__ __forceinline__ uint32_t scale2_w4a16(uint32_t two_e4m3) {
+  const uint32_t h = cvt_e4m3x2_f16x2(two_e4m3);
+  return ((h >> 3) & 0x1FFF1FFFu) + 0x73007300u;
+}
+
+__device__ __forceinline__ void dequant8_w4a16(uint32_t c, uint32_t s2, uint32_t* o) {
+  o[0] = bmul2(c & kPairMask, s2);
+  o[1] = bmul2(rotr32(c, 4) & kPairMask, s2);
+  o[2] = bmul2(rotr32(c, 10) & kPairMask, s2);
+  o[3] = bmul2((rotr32(c, 6) & kPairMaskA) | (rotr32(c, 14) & kPairMaskB), s2);
+}
+
+// One thread's 64-element chunk (rearranged codes, four scales) -> 32 columns.
+__device__ __forceinline__ void dequant64_w4a16(const uint4 lo, const uint4 hi, uint32_t sc,
+                                                uint32_t (&v)[32]) {
+  const uint32_t t01 = scale2_w4a16(sc & 0xffffu), t23 = scale2_w4a16(sc >> 16);
+  const uint32_t s0 = __byte_perm(t01, 0, 0x1010), s1 = __byte_perm(t01, 0, 0x3232);
+  const uint32_t s2 = __byte_perm(t23, 0, 0x1010), s3 = __byte_perm(t23, 0, 0x3232);
+  dequant8_w4a16(lo.x, s0, v + 0);
+  dequant8_w4a16(lo.y, s0, v + 4);
+  dequant8_w4a16(lo.z, s1, v + 8);
+  dequant8_w4a16(lo.w, s1, v + 12);
+  dequant8_w4a16(hi.x, s2, v + 16);
+  dequant8_w4a16(hi.y, s2, v + 20);
+  dequant8_w4a16(hi.z, s3, v + 24);
+  dequant8_w4a16(hi.w, s3, v + 28);
 }
 
 // SiLU with the fast exponential and division (a few ulp in fp32; the result
@@ -191,12 +223,13 @@ __device__ __forceinline__ bool wait_drain(uint64_t* bar, uint32_t parity) {
 // chunk; thread (q, lane) owns tile row 32q + lane.  kEpiStore writes
 // y = bf16(gs * acc); kEpiSiluMul (rows 0-63 gate, 64-127 the matching up rows)
 // writes h = bf16(silu(bf16(gs_g * g)) * bf16(gs_u * u)); kEpiPartial writes
-// fp32 split-K partials.  Stores are staged through shared memory (ebuf,
+// fp32 split-K partials (gs_mul: a power of two folded into the operands,
+// applied with gs).  Stores are staged through shared memory (ebuf,
 // 16 KB per warpgroup) so that global writes are 16-byte and row-contiguous.
 template <int BN, int EPI, int NG, int NACC = 1>
 __device__ __forceinline__ void epilogue_tile(const TcArgs& a, uint32_t tmem, int q, int lane,
                                               int g, uint8_t* ebuf, int xtile, int wtile,
-                                              int nacc_used = 1) {
+                                              int nacc_used = 1, float gs_mul = 1.0f) {
   const int row = 32 * q + lane;
   const uint32_t lane_addr = (uint32_t)(32 * q) << 16;
   const int rbase = xtile * BN;
@@ -231,7 +264,7 @@ __device__ __forceinline__ void epilogue_tile(const TcArgs& a, uint32_t tmem, in
         if (j < jmax && r0 + j < a.m) P[(size_t)(r0 + j) * a.n_pad + col] = __uint_as_float(v[j]);
     } else if (EPI == kEpiStore) {
       uint16_t* T = reinterpret_cast<uint16_t*>(ebuf);  // [32][128] bf16
-      const float gs = a.gs[0];
+      const float gs = a.gs[0] * gs_mul;
 #pragma unroll
       for (int j = 0; j < 32; ++j) T[j * 128 + row] = f32_to_bf16_bits(gs * __uint_as_float(v[j]));
       named_bar_sync(1 + g, 128);
@@ -248,13 +281,13 @@ __device__ __forceinline__ void epilogue_tile(const TcArgs& a, uint32_t tmem, in
       float* U = reinterpret_cast<float*>(ebuf);                  // [32][64] fp32
       uint16_t* Hs = reinterpret_cast<uint16_t*>(ebuf + 8192);    // [32][64] bf16
       if (q >= 2) {
-        const float gsu = a.gs[1];
+        const float gsu = a.gs[1] * gs_mul;
 #pragma unroll
         for (int j = 0; j < 32; ++j) U[j * 64 + (row - 64)] = bf16_round(gsu * __uint_as_float(v[j]));
       }
       named_bar_sync(1 + g, 128);
       if (q < 2) {
-        const float gsg = a.gs[0];
+        const float gsg = a.gs[0] * gs_mul;
 #pragma unroll
         for (int j = 0; j < 32; ++j) {
           const float gv = bf16_round(gsg * __uint_as_float(v[j]));
@@ -412,7 +445,7 @@ tc_w4a16_kernel(const __grid_constant__ CUtensorMap xmap, const TcArgs a) {
         const uint4 hi = *reinterpret_cast<const uint4*>(w + 2048 + 16 * row);
         const uint32_t sc = *reinterpret_cast<const uint32_t*>(w + 4096 + sf_off);
         uint32_t v[32];
-        dequant64(lo, hi, sc, v);
+        dequant64_w4a16(lo, hi, sc, v);
         tmem_st32(tmem + lane_addr + C::kAColBase + C::kSlotCols * sa + 32 * c, v);
       }
       __syncwarp();
@@ -430,7 +463,7 @@ tc_w4a16_kernel(const __grid_constant__ CUtensorMap xmap, const TcArgs a) {
     tc_fence_after();
     if (done && !*abort_flag)
       epilogue_tile<BN, EPI, DQG, NI>(a, tmem, q, lane, g, epi + g * C::kEpiBytes, xtile, wtile,
-                                      min(NI, nunits));
+                                      min(NI, nunits), kW4A16Unscale);
   }
   tc_fence_before();
   __syncthreads();
@@ -584,7 +617,7 @@ tc_w4a4_kernel(const __grid_constant__ CUtensorMap xmap, const W4Args w4) {
 // Split-K reduction in a fixed order (z = 0, 1, ...), then the epilogue.
 template <bool kGateUp>
 __global__ void splitk_reduce_kernel(const float* __restrict__ P, int splits, int m, int n_pad,
-                                     int n_out, const float* __restrict__ gs,
+                                     int n_out, const float* __restrict__ gs, float gs_mul,
                                      uint16_t* __restrict__ out, int ldo) {
   const int64_t idx = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;
   if (idx >= (int64_t)m * n_out) return;
@@ -597,12 +630,12 @@ __global__ void splitk_reduce_kernel(const float* __restrict__ P, int splits, in
       g += P[z * plane + (size_t)r * n_pad + gcol];
       u += P[z * plane + (size_t)r * n_pad + ucol];
     }
-    const float gb = bf16_round(gs[0] * g), ub = bf16_round(gs[1] * u);
+    const float gb = bf16_round(gs[0] * gs_mul * g), ub = bf16_round(gs[1] * gs_mul * u);
     out[(size_t)r * ldo + n] = f32_to_bf16_bits(silu_fast(gb) * ub);
   } else {
     float acc = 0.0f;
     for (int z = 0; z < splits; ++z) acc += P[z * plane + (size_t)r * n_pad + n];
-    out[(size_t)r * ldo + n] = f32_to_bf16_bits(gs[0] * acc);
+    out[(size_t)r * ldo + n] = f32_to_bf16_bits(gs[0] * gs_mul * acc);
   }
 }
 
@@ -612,7 +645,8 @@ __global__ void splitk_reduce_kernel(const float* __restrict__ P, int splits, in
 // by the up rows with the same indices.  Padding rows / K tails are zero.
 __global__ void tile_weight_kernel(const uint8_t* __restrict__ codes,
                                    const uint8_t* __restrict__ scales, int64_t nrows, int64_t k,
-                                   int64_t half, int ntiles, int kc, uint8_t* __restrict__ out) {
+                                   int64_t half, int ntiles, int kc, bool for_w4a16,
+                                   uint8_t* __restrict__ out) {
   const int64_t idx = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;
   if (idx >= (int64_t)ntiles * kc * kTileRows) return;
   const int r = (int)(idx % kTileRows);
@@ -640,6 +674,20 @@ __global__ void tile_weight_kernel(const uint8_t* __restrict__ codes,
     if (off + 32 <= cb) hi = *reinterpret_cast<const uint4*>(crow + off + 16);
     for (int b = 0; b < 4; ++b)
       if (4 * (int64_t)j + b < sb) sc |= (uint32_t)srow[4 * j + b] << (8 * b);
+  }
+  if (for_w4a16) {
+    // The bf16-activation copy: scales lose the sign bit (scales are
+    // magnitudes), a block whose scale is zero gets zero codes (the decoded
+    // scale of such a block is not zero), and the code bits are rearranged.
+    uint32_t w[8] = {lo.x, lo.y, lo.z, lo.w, hi.x, hi.y, hi.z, hi.w};
+    sc &= 0x7F7F7F7Fu;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      if (((sc >> (8 * (i >> 1))) & 0xFFu) == 0) w[i] = 0;
+      w[i] = permute_codes_w4a16(w[i]);
+    }
+    lo = make_uint4(w[0], w[1], w[2], w[3]);
+    hi = make_uint4(w[4], w[5], w[6], w[7]);
   }
   uint8_t* base = out + ((int64_t)t * kc + j) * kChunkBytes;
   *reinterpret_cast<uint4*>(base + 16 * r) = lo;
@@ -716,13 +764,13 @@ int64_t tc_tiled_bytes(int64_t n, int64_t k, bool gate_up) {
 }
 
 cudaError_t launch_tile_weight(const uint8_t* codes, const uint8_t* scales, int64_t n, int64_t k,
-                               bool gate_up, uint8_t* out, cudaStream_t s) {
+                               bool gate_up, bool for_w4a16, uint8_t* out, cudaStream_t s) {
   const int64_t half = gate_up ? n / 2 : 0;
   const int ntiles = (int)(gate_up ? (half + 63) / 64 : (n + kTileRows - 1) / kTileRows);
   const int kc = (int)((k + kChunkK - 1) / kChunkK);
   const int64_t total = (int64_t)ntiles * kc * kTileRows;
   tile_weight_kernel<<<(unsigned)((total + 255) / 256), 256, 0, s>>>(codes, scales, n, k, half, ntiles,
-                                                                   kc, out);
+                                                                   kc, for_w4a16, out);
   return cudaGetLastError();
 }
 
@@ -755,7 +803,7 @@ cudaError_t launch_tc_w4a16(const void* x, int64_t m, const TcWeight& w, bool si
   if (!make_x_map(&map, x, m, w.k, box_rows)) return cudaErrorInvalidValue;
   TcArgs a;
   a.x_box_rows = box_rows;
-  a.wt = w.tiled;
+  a.wt = w.tiled16;
   a.gs = w.gs;
   a.m = (int)m;
   a.n_out = (int)(silu_mul ? w.n / 2 : w.n);
@@ -776,10 +824,12 @@ cudaError_t launch_tc_w4a16(const void* x, int64_t m, const TcWeight& w, bool si
     ProfScope prof(s, silu_mul ? "splitk_reduce_silu_mul" : "splitk_reduce");
     if (silu_mul)
       splitk_reduce_kernel<true><<<(unsigned)((total + 255) / 256), 256, 0, s>>>(
-          (const float*)partials, p.splits, (int)m, p.n_pad, a.n_out, w.gs, (uint16_t*)y, a.ldo);
+          (const float*)partials, p.splits, (int)m, p.n_pad, a.n_out, w.gs, kW4A16Unscale,
+          (uint16_t*)y, a.ldo);
     else
       splitk_reduce_kernel<false><<<(unsigned)((total + 255) / 256), 256, 0, s>>>(
-          (const float*)partials, p.splits, (int)m, p.n_pad, a.n_out, w.gs, (uint16_t*)y, a.ldo);
+          (const float*)partials, p.splits, (int)m, p.n_pad, a.n_out, w.gs, kW4A16Unscale,
+          (uint16_t*)y, a.ldo);
     return cudaGetLastError();
   }
   a.out = y;
@@ -861,10 +911,12 @@ cudaError_t launch_tc_w4a4(const uint8_t* xcodes, const uint8_t* xsf_blocks, int
     ProfScope prof(s, silu_mul ? "splitk_reduce_silu_mul" : "splitk_reduce");
     if (silu_mul)
       splitk_reduce_kernel<true><<<(unsigned)((total + 255) / 256), 256, 0, s>>>(
-          (const float*)partials, p.splits, (int)m, p.n_pad, a.t.n_out, w.gs, (uint16_t*)y, a.t.ldo);
+          (const float*)partials, p.splits, (int)m, p.n_pad, a.t.n_out, w.gs, 1.0f, (uint16_t*)y,
+          a.t.ldo);
     else
       splitk_reduce_kernel<false><<<(unsigned)((total + 255) / 256), 256, 0, s>>>(
-          (const float*)partials, p.splits, (int)m, p.n_pad, a.t.n_out, w.gs, (uint16_t*)y, a.t.ldo);
+          (const float*)partials, p.splits, (int)m, p.n_pad, a.t.n_out, w.gs, 1.0f, (uint16_t*)y,
+          a.t.ldo);
     return cudaGetLastError();
   }
   a.t.out = y;
