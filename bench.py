@@ -19,6 +19,7 @@ from __future__ import annotations
 
 import argparse
 import json
+import math
 import os
 import statistics
 import subprocess
@@ -137,15 +138,27 @@ class Workload:
         self.name, self.m, self.H, self.I, self.fmt = name, (m or m0), H, I, fmt
         inp = synth.make_inputs(recipe, m=self.m)
         dev = lambda b: torch.from_numpy(np.ascontiguousarray(b).view(np.int16)).view(torch.bfloat16).cuda()
-        hs = []
+        q = []
         for bits in (inp.w_gate, inp.w_up, inp.w_down):
             w = dev(bits)
-            c, s, g = native.ffn_nvfp4_quantize_weights(w)
-            hs.append(native.ffn_nvfp4_weight_create(c, s, g))
-            del w, c, s, g
-        self.gate_up = native.ffn_nvfp4_weight_create_gate_up(hs[0], hs[1])
-        self.down = hs[2]
-        del hs[:2]
+            q.append(native.ffn_nvfp4_quantize_weights(w))
+            del w
+        self.weight_bytes = nvfp4_bytes(2 * I, H) + nvfp4_bytes(H, I)
+        # A step that reads less than twice the L2 would find part of its
+        # weights still cached from earlier steps: such layers rotate through R
+        # copies of their weights (R x weight bytes >= 4 x L2), so every step
+        # streams weights that 3+ other steps' worth of traffic has evicted.
+        act_bytes = self.m * (H + I) * 2 * 2
+        self.sets = 1
+        if self.weight_bytes + act_bytes < 2 * L2_BYTES:
+            self.sets = int(math.ceil(4 * L2_BYTES / self.weight_bytes))
+        self.handles = []
+        for _ in range(self.sets):
+            g, u, d = (native.ffn_nvfp4_weight_create(*t) for t in q)
+            self.handles.append((native.ffn_nvfp4_weight_create_gate_up(g, u), d))
+            del g, u
+        del q
+        self.gate_up, self.down = self.handles[0]
         self.x = dev(inp.x)
         self.x_bits = inp.x
         self.out = torch.empty((self.m, H), dtype=torch.bfloat16, device="cuda")
@@ -153,13 +166,14 @@ class Workload:
                               dtype=torch.uint8, device="cuda")
         self.native = native
         torch.cuda.synchronize()
-        # reads per step exceed L2 for prefill-size batches; otherwise flush
-        self.weight_bytes = nvfp4_bytes(2 * I, H) + nvfp4_bytes(H, I)
-        self.flush_l2 = self.weight_bytes + self.m * (H + I) * 4 < 2 * L2_BYTES
+        self.flush_l2 = False
+        self.l2_note = (f"weights rotated through {self.sets} copies ({self.sets} x "
+                        f"{self.weight_bytes / 1e6:.1f} MB >= 4 x L2)" if self.sets > 1
+                        else "reads per step exceed 2 x L2")
 
-    def step(self):
-        self.native.ffn_nvfp4_forward(self.x, self.gate_up, self.down, self.fmt, out=self.out,
-                                      workspace=self.ws)
+    def step(self, i=0):
+        gate_up, down = self.handles[i % self.sets]
+        self.native.ffn_nvfp4_forward(self.x, gate_up, down, self.fmt, out=self.out, workspace=self.ws)
 
     def kernel_units(self, kname):
         """(bound, algorithmic flops or bytes per launch) of a kernel of this layer."""
@@ -193,22 +207,18 @@ def run_ours(args, rank, world, dist):
 
     clocks = Clocks(dev_index)
     clocks.start()
-    for _ in range(args.warmup):
-        wl.step()
+    for i in range(args.warmup):
+        wl.step(i)
     barrier()
-    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
-    stops = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
-    N.ffn_nvfp4_profile_begin()
-    for i in range(args.steps):
-        if flush is not None:
-            flush.zero_()
-        starts[i].record()
-        wl.step()
-        stops[i].record()
+    graph, starts, stops = capture_steps(N, wl, args.steps, flush)
+    graph.replay()  # untimed: loads the graph onto the device
+    barrier()
+    graph.replay()  # the timed region: K steps
     barrier()
     prof = N.ffn_nvfp4_profile_end()
     clk = clocks.stop()
     ms = max_over_ranks(sum(a.elapsed_time(b) for a, b in zip(starts, stops)), dist, "cuda")
+    del graph
     ms_step = ms / args.steps
     flops = ffn_flops(wl.m, wl.H, wl.I)
     value = aggregate_throughput(flops, args.steps, ms, world) / 1e12
@@ -246,9 +256,10 @@ def run_ours(args, rank, world, dist):
     barrier()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record()
-    for _ in range(e2e_steps):
+    for i in range(e2e_steps):
         x_dev.copy_(x_host, non_blocking=True)
-        N.ffn_nvfp4_forward(x_dev, wl.gate_up, wl.down, wl.fmt, out=wl.out, workspace=wl.ws)
+        gate_up, down = wl.handles[i % wl.sets]
+        N.ffn_nvfp4_forward(x_dev, gate_up, down, wl.fmt, out=wl.out, workspace=wl.ws)
         out_host.copy_(wl.out, non_blocking=True)
     e1.record()
     barrier()
@@ -257,6 +268,7 @@ def run_ours(args, rank, world, dist):
            "h2d_bytes_per_step": wl.m * wl.H * 2, "d2h_bytes_per_step": wl.m * wl.H * 2,
            "ms_per_step": round(e2e_ms / e2e_steps, 4)}
 
+    l2_note = wl.l2_note
     extra = {}
     if not args.no_extra and args.workload == "prefill":
         del wl, x_dev
@@ -268,28 +280,47 @@ def run_ours(args, rank, world, dist):
         "value": round(value, 3), "ms_per_step": round(ms_step, 4), "roofline": roof,
         "kernels": kernels, "gpu_launches": gpu_launches, "clocks": clk, "e2e": e2e,
         "workload": args.workload, "m": args.m or WORKLOADS[args.workload][1], "extra": extra,
-        "l2": "flushed between timed steps" if flush is not None else "inputs larger than L2",
+        "l2": l2_note,
     }
+
+
+def capture_steps(N, wl, steps, flush):
+    """Capture `steps` forward steps (each after an optional L2 flush, between
+    a pair of timing events) into one CUDA graph, with the library's per-kernel
+    profiling on, so every timestamp is taken on the device during replay and
+    none includes host launch latency.  Returns (graph, starts, stops); the
+    profiling recording stays open until ffn_nvfp4_profile_end."""
+    import torch
+    starts = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(steps)]
+    stops = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(steps)]
+    graph = torch.cuda.CUDAGraph()
+    N.ffn_nvfp4_profile_begin()
+    with torch.cuda.graph(graph, stream=torch.cuda.Stream()):
+        for i in range(steps):
+            if flush is not None:
+                flush.zero_()
+            starts[i].record()
+            wl.step(i)
+            stops[i].record()
+    return graph, starts, stops
 
 
 def secondary(N, name, m, peaks, steps):
     """Time another layer shape: per-step µs, weight GB/s and TFLOP/s."""
     import torch
     wl = Workload(N, name, m)
-    flush = torch.empty(2 * L2_BYTES // 4, dtype=torch.float32, device="cuda")
-    for _ in range(3):
-        wl.step()
+    flush = None  # cold weights come from rotating weight copies (Workload)
+    for i in range(3):
+        wl.step(i)
     torch.cuda.synchronize()
-    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
-    N.ffn_nvfp4_profile_begin()
-    for a, b in ev:
-        flush.zero_()
-        a.record()
-        wl.step()
-        b.record()
+    graph, starts, stops = capture_steps(N, wl, steps, flush)
+    graph.replay()
+    torch.cuda.synchronize()
+    graph.replay()
     torch.cuda.synchronize()
     prof = N.ffn_nvfp4_profile_end()
-    ms = sum(a.elapsed_time(b) for a, b in ev) / steps
+    ms = sum(a.elapsed_time(b) for a, b in zip(starts, stops)) / steps
+    del graph
     res = {"m": m, "hidden": wl.H, "inter": wl.I, "format": wl.fmt, "us_per_layer": round(ms * 1e3, 2),
            "weight_gbs": round(wl.weight_bytes / (ms * 1e-3) / 1e9, 1),
            "tflops": round(ffn_flops(m, wl.H, wl.I) / (ms * 1e-3) / 1e12, 3),
@@ -400,7 +431,8 @@ def main():
         "dtype": "bf16 x nvfp4 (fp32 accumulate)" if fmt == "bf16" else "nvfp4 x nvfp4 (fp32 accumulate)",
         "data": "synthetic (seeded numpy draws; random-init weights)",
         "config": {"workload": args.workload, "m": res["m"], "hidden": H, "inter": I, "act_format": fmt,
-                   "parallelism": f"replicas x{world}", "l2": res["l2"]},
+                   "parallelism": f"replicas x{world}", "l2": res["l2"],
+                   "launch": "the K timed steps captured in one CUDA graph, replayed once"},
         "roofline": res["roofline"], "cpu_baseline": cpu, "e2e": res["e2e"],
         "gpu_launches": res["gpu_launches"], "kernels": res["kernels"], "clocks": res["clocks"],
     }

@@ -206,7 +206,12 @@ ffn_status ffn_nvfp4_device_error(int* flags, int clear);
  * kernel into out[0..*count) (name: static string; capacity entries at most,
  * FFN_ERR_INVALID_ARG if more distinct kernels ran).  Recording adds event
  * records to the streams but no device work; it creates CUDA events (host
- * resources) on first use and reuses them afterwards. */
+ * resources) on first use and reuses them afterwards.  Launches made while
+ * their stream is being captured into a CUDA graph get event-record nodes in
+ * the graph instead: the durations are then those of the graph's latest
+ * replay (replay it before ffn_nvfp4_profile_end).  Host-recorded events can
+ * include time the device spends waiting for the host to submit the launch;
+ * graph-recorded ones cannot. */
 typedef struct ffn_kernel_time {
   const char* name;
   int launches;

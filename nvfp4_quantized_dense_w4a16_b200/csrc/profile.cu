@@ -35,16 +35,26 @@ thread_local Recorder rec;
 
 bool profiling() { return rec.active; }
 
+// While the stream is being captured into a CUDA graph the events become
+// event-record nodes of the graph, so they time each replay on the device.
+static void prof_record(cudaEvent_t e, cudaStream_t s) {
+  cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+  if (cudaStreamIsCapturing(s, &cs) == cudaSuccess && cs == cudaStreamCaptureStatusActive)
+    cudaEventRecordWithFlags(e, s, cudaEventRecordExternal);
+  else
+    cudaEventRecord(e, s);
+}
+
 void prof_mark_start(cudaStream_t s, const char* name) {
   Mark m{name, rec.take(), rec.take()};
   if (m.start && m.stop) {
-    cudaEventRecord(m.start, s);
+    prof_record(m.start, s);
     rec.marks.push_back(m);
   }
 }
 
 void prof_mark_stop(cudaStream_t s) {
-  if (!rec.marks.empty()) cudaEventRecord(rec.marks.back().stop, s);
+  if (!rec.marks.empty()) prof_record(rec.marks.back().stop, s);
 }
 
 }  // namespace ffn

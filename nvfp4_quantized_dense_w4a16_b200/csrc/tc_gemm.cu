@@ -49,34 +49,43 @@ constexpr int kChunkBytes = 4608;  // 128 x (16 + 16 + 4) bytes
 
 enum : int { kEpiStore = 0, kEpiSiluMul = 1, kEpiPartial = 2 };
 
-// Pipeline shape.  Work is handed out in units of U consecutive 64-element
-// chunks; every ring holds whole units: SXU activation stages (released when
-// the MMAs that read them complete), SWU weight stages (released as soon as
-// the dequant warps have read them) and SA tensor-memory slots for the
-// dequantised weights.  Unit u belongs to dequant warpgroup u % DQG, whose
-// four warps (one per TMEM lane quarter) dequantise all 128 rows of its chunks
-// and also observe the unit's activation barrier, so the MMA thread waits on
-// one barrier per unit.  NI threads issue MMAs (unit u -> issuer u % NI), each
-// into its own accumulator; the epilogue adds the accumulators.  Every
-// mbarrier wait and tcgen05 fence costs ~0.1 us even when nothing is pending,
-// which is why waits are per unit and narrow tiles use two issuers.
-template <int BN, int SXU, int SWU, int SA, int DQG, int U, int NI>
+// Pipeline shape.  The K range of a CTA is a sequence of 64-element chunks,
+// grouped into units of UA consecutive chunks; unit u is dequantised by
+// warpgroup u % DQG (its four warps cover the 128 TMEM lanes) into TMEM slot
+// u % SA and multiplied by MMA-issuing thread u % NI into that thread's own
+// accumulator (the epilogue adds them).  Three rings, each with its own
+// granularity:
+//  * weights: SWS stages of one round (DQG consecutive units, one per
+//    warpgroup), released once every warpgroup has read its unit;
+//  * activations: SXS stages of XC chunks, released when the MMAs that read
+//    them complete and waited for either by the MMA threads (once per stage)
+//    or, with DQX (one stage per unit), by the unit's dequant warps before
+//    they hand the slot over -- which keeps that wait off the MMA thread, the
+//    critical role of wide tiles;
+//  * TMEM: SA A slots of one unit, released when their MMAs complete, so a
+//    warpgroup can dequantise its next units while earlier ones are still in
+//    the tensor pipe.
+// Every mbarrier wait and tcgen05 fence costs ~0.1 us even when nothing is
+// pending, so the dequant warps wait on two barriers per unit (slot free,
+// weights landed) and the MMA threads on one (plus one per activation stage).
+template <int BN, int SXS, int XC, int SWS, int SA, int DQG, int UA, int NI, bool DQX>
 struct TcCfg {
   static constexpr int kThreads = 128 + 128 * DQG;
-  static constexpr int kXStageBytes = U * BN * 128;    // U chunk tiles of BN rows x 128 B
-  static constexpr int kWStageBytes = U * kChunkBytes;
+  static constexpr int kXStageBytes = XC * BN * 128;   // XC chunk tiles of BN rows x 128 B
+  static constexpr int kUnitBytes = UA * kChunkBytes;
+  static constexpr int kWStageBytes = DQG * kUnitBytes;
   static constexpr int kAColBase = NI * BN < 32 ? 32 : NI * BN;  // TMEM column of A slot 0
-  static constexpr int kSlotCols = 32 * U;
+  static constexpr int kSlotCols = 32 * UA;
   static constexpr int kTmemNeed = kAColBase + kSlotCols * SA;
   static constexpr int kTmemCols = kTmemNeed <= 64 ? 64 : kTmemNeed <= 128 ? 128 : kTmemNeed <= 256 ? 256 : 512;
   // The epilogue staging buffers (16 KB per dequant warpgroup) reuse the start
   // of the rings: the epilogue runs after every MMA has completed, and those
   // MMAs consumed every copy the producers issued.
   static constexpr int kEpiBytes = 16384;
-  static constexpr int kSmemW = SXU * kXStageBytes;
-  static constexpr int kSmemRings = kSmemW + SWU * kWStageBytes;
+  static constexpr int kSmemW = SXS * kXStageBytes;
+  static constexpr int kSmemRings = kSmemW + SWS * kWStageBytes;
   static constexpr int kSmemBar = kSmemRings;
-  static constexpr int kNumBars = 2 * SXU + 2 * SWU + 2 * SA + NI;
+  static constexpr int kNumBars = 2 * SXS + 2 * SWS + 2 * SA + NI;
   static constexpr int kSmemBytes = kSmemBar + kNumBars * 8 + 16;
   static constexpr int kSmemAlloc = kSmemBytes + 1024;  // slack for 1024-byte alignment
   // two CTAs per SM when both fit (228 KB of shared memory, 512 TMEM columns)
@@ -84,18 +93,18 @@ struct TcCfg {
   static_assert(kTmemNeed <= 512, "TMEM budget");
   static_assert(kSmemAlloc <= 232448, "shared memory budget");
   static_assert(BN % 16 == 0 && BN >= 16 && BN <= 256, "MMA N");
-  static_assert(DQG == 1 || DQG == 2, "dequant warpgroups");
-  static_assert(NI == 1 || (NI == 2 && DQG == 2), "MMA issuers pair with warpgroups");
+  static_assert(DQG >= 1 && DQG <= 3 && (NI == 1 || NI == 2) && UA >= 1, "roles");
   static_assert(kSmemRings >= DQG * kEpiBytes, "epilogue buffers alias the rings");
   // A parity wait can only tell the awaited phase from the one before it, so
   // the previous phase must be known complete when a thread starts waiting.
-  // With one issuer the MMAs complete in unit order, which covers every ring
-  // whose depth is >= SA.  With two, each TMEM slot must stay with one
-  // warpgroup/issuer pair (SA a multiple of DQG); a weight (activation) stage
-  // either does too (even depth) or is deep enough that the sequential
-  // activation producer's progress implies it (depth >= DQG + SXU).
-  static_assert(NI == 1 ? (SWU >= SA && SXU >= SA)
-                        : (SA % DQG == 0 && (SWU % 2 == 0 || SWU >= DQG + SXU) && SXU % 2 == 0),
+  // Slot u % SA is reused by unit u + SA: with SA a multiple of DQG and of NI
+  // that unit has the same warpgroup and the same MMA thread, each of which
+  // waited for the slot's previous phase itself.  Every warpgroup waits for
+  // every weight round and (XC a multiple of UA * NI) every MMA thread for
+  // every activation stage, in order, which covers those rings.
+  // With DQX, stage u % SXS is reused by unit u + SXS of the same warpgroup.
+  static_assert(SA % DQG == 0 && SA % NI == 0 &&
+                    (DQX ? (XC == UA && SXS % DQG == 0) : XC % (UA * NI) == 0),
                 "ring depths");
 };
 
@@ -308,11 +317,11 @@ __device__ __forceinline__ void epilogue_tile(const TcArgs& a, uint32_t tmem, in
   }
 }
 
-template <int BN, int SXU, int SWU, int SA, int DQG, int U, int NI, int EPI>
-__global__ void __launch_bounds__(TcCfg<BN, SXU, SWU, SA, DQG, U, NI>::kThreads,
-                                  TcCfg<BN, SXU, SWU, SA, DQG, U, NI>::kMinBlocks)
+template <int BN, int SXS, int XC, int SWS, int SA, int DQG, int UA, int NI, bool DQX, int EPI>
+__global__ void __launch_bounds__(TcCfg<BN, SXS, XC, SWS, SA, DQG, UA, NI, DQX>::kThreads,
+                                  TcCfg<BN, SXS, XC, SWS, SA, DQG, UA, NI, DQX>::kMinBlocks)
 tc_w4a16_kernel(const __grid_constant__ CUtensorMap xmap, const TcArgs a) {
-  using C = TcCfg<BN, SXU, SWU, SA, DQG, U, NI>;
+  using C = TcCfg<BN, SXS, XC, SWS, SA, DQG, UA, NI, DQX>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
@@ -320,10 +329,10 @@ tc_w4a16_kernel(const __grid_constant__ CUtensorMap xmap, const TcArgs a) {
   uint8_t* wsm = smem + C::kSmemW;
   uint8_t* epi = smem;  // aliases the rings; used only after the last MMA
   uint64_t* xfull = reinterpret_cast<uint64_t*>(smem + C::kSmemBar);
-  uint64_t* xempty = xfull + SXU;
-  uint64_t* wfull = xempty + SXU;
-  uint64_t* wempty = wfull + SWU;
-  uint64_t* afull = wempty + SWU;
+  uint64_t* xempty = xfull + SXS;
+  uint64_t* wfull = xempty + SXS;
+  uint64_t* wempty = wfull + SWS;
+  uint64_t* afull = wempty + SWS;
   uint64_t* aempty = afull + SA;
   uint64_t* accum = aempty + SA;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(accum + NI);
@@ -333,17 +342,17 @@ tc_w4a16_kernel(const __grid_constant__ CUtensorMap xmap, const TcArgs a) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int xtile = blockIdx.x, wtile = blockIdx.y;
   const int kc0 = blockIdx.z * a.kc_per_split;
-  const int nk = min(a.kc_total, kc0 + a.kc_per_split) - kc0;
-  const int nunits = (nk + U - 1) / U;
+  const int nk = min(a.kc_total, kc0 + a.kc_per_split) - kc0;  // >= 1 by the plan
+  const int nunits = (nk + UA - 1) / UA;
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < SXU; ++s) {
+    for (int s = 0; s < SXS; ++s) {
       mbar_init(&xfull[s], 1);
-      mbar_init(&xempty[s], 1);
+      mbar_init(&xempty[s], DQX ? 1 : NI);  // one commit per MMA thread using the stage
     }
-    for (int s = 0; s < SWU; ++s) {
+    for (int s = 0; s < SWS; ++s) {
       mbar_init(&wfull[s], 1);
-      mbar_init(&wempty[s], 4);  // the four warps of the owning warpgroup
+      mbar_init(&wempty[s], 4 * DQG);  // every dequant warp
     }
     for (int s = 0; s < SA; ++s) {
       mbar_init(&afull[s], 4);
@@ -367,57 +376,63 @@ tc_w4a16_kernel(const __grid_constant__ CUtensorMap xmap, const TcArgs a) {
     // ------------------------------------------------- weight producer
     if (lane == 0) {
       const uint8_t* wsrc = a.wt + ((size_t)wtile * a.kc_total + kc0) * kChunkBytes;
+      const int rounds = (nunits + DQG - 1) / DQG;
       int issued = 0;
-      for (int u = 0; u < nunits; ++u) {
-        const int s = u % SWU;
-        const int nc = min(U, nk - u * U);
-        if (u >= SWU && !mbar_wait(&wempty[s], ((u / SWU) - 1) & 1, abort_flag, err, 1)) break;
+      for (int r = 0; r < rounds; ++r) {
+        const int s = r % SWS;
+        const int nc = min(DQG * UA, nk - r * DQG * UA);
+        if (r >= SWS && !mbar_wait(&wempty[s], ((r / SWS) - 1) & 1, abort_flag, err, 1)) break;
         mbar_arrive_expect_tx(&wfull[s], nc * kChunkBytes);
-        bulk_load(wsm + s * C::kWStageBytes, wsrc + (size_t)u * U * kChunkBytes, nc * kChunkBytes, &wfull[s]);
+        bulk_load(wsm + s * C::kWStageBytes, wsrc + (size_t)r * C::kWStageBytes, nc * kChunkBytes,
+                  &wfull[s]);
         ++issued;
       }
       // no copy into this CTA's shared memory may outlive it
-      for (int u = max(0, issued - SWU); u < issued; ++u) wait_drain(&wfull[u % SWU], (u / SWU) & 1);
+      for (int r = max(0, issued - SWS); r < issued; ++r) wait_drain(&wfull[r % SWS], (r / SWS) & 1);
     }
   } else if (warp == 3) {
     // --------------------------------------------- activation producer
     if (lane == 0) {
+      const int stages = (nk + XC - 1) / XC;
       int issued = 0;
-      for (int u = 0; u < nunits; ++u) {
-        const int s = u % SXU;
-        const int nc = min(U, nk - u * U);
-        if (u >= SXU && !mbar_wait(&xempty[s], ((u / SXU) - 1) & 1, abort_flag, err, 1)) break;
+      for (int t = 0; t < stages; ++t) {
+        const int s = t % SXS;
+        const int nc = min(XC, nk - t * XC);
+        if (t >= SXS && !mbar_wait(&xempty[s], ((t / SXS) - 1) & 1, abort_flag, err, 1)) break;
         mbar_arrive_expect_tx(&xfull[s], nc * a.x_box_rows * 128);
         for (int c = 0; c < nc; ++c)
-          tma_load_2d(xs + s * C::kXStageBytes + c * BN * 128, &xmap, (kc0 + u * U + c) * kChunkK,
+          tma_load_2d(xs + s * C::kXStageBytes + c * BN * 128, &xmap, (kc0 + t * XC + c) * kChunkK,
                       xtile * BN, &xfull[s]);
         ++issued;
       }
-      for (int u = max(0, issued - SXU); u < issued; ++u) wait_drain(&xfull[u % SXU], (u / SXU) & 1);
+      for (int t = max(0, issued - SXS); t < issued; ++t) wait_drain(&xfull[t % SXS], (t / SXS) & 1);
     }
   } else if (warp == 1 || (NI == 2 && warp == 2)) {
     // -------------------------------------------------- MMA issuer(s)
     if (lane == 0) {
-      const int j = warp - 1;  // issuer index: units u = j, j + NI, ...
+      const int j = warp - 1;  // units u = j, j + NI, ...
       const uint32_t idesc = idesc_bf16_f32(kTileRows, BN);
-      const uint32_t d = tmem + j * BN;  // this issuer's accumulator
-      bool first = true;
+      const uint32_t d = tmem + j * BN;  // this thread's accumulator
+      constexpr int kUnitsPerX = XC / UA;
       for (int u = j; u < nunits; u += NI) {
-        const int sa = u % SA, sx = u % SXU;
-        if (!mbar_wait(&afull[sa], (u / SA) & 1, abort_flag, err, 2)) break;  // A and x both ready
+        const int t = u / kUnitsPerX, sx = t % SXS, sa = u % SA;
+        if (!DQX && u % kUnitsPerX == j && !mbar_wait(&xfull[sx], (t / SXS) & 1, abort_flag, err, 2))
+          break;
+        if (!mbar_wait(&afull[sa], (u / SA) & 1, abort_flag, err, 2)) break;
         tc_fence_after();
-        const int nc = min(U, nk - u * U);
-        const uint64_t b_stage = smem_desc_sw128(smem_u32(xs + sx * C::kXStageBytes));
+        const int nc = min(UA, nk - u * UA);
         for (int c = 0; c < nc; ++c) {
           const uint32_t a_base = tmem + C::kAColBase + C::kSlotCols * sa + 32 * c;
-          const uint64_t b_base = b_stage + (uint64_t)((c * BN * 128) >> 4);
+          const uint64_t b_base = smem_desc_sw128(
+              smem_u32(xs + sx * C::kXStageBytes + ((u % kUnitsPerX) * UA + c) * BN * 128));
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk)
-            mma_bf16_ts(d, a_base + 8 * kk, b_base + 2 * kk, idesc, (first && kk == 0) ? 0u : 1u);
-          first = false;
+            mma_bf16_ts(d, a_base + 8 * kk, b_base + 2 * kk, idesc,
+                        (u == j && c == 0 && kk == 0) ? 0u : 1u);
         }
         mma_commit(&aempty[sa]);
-        mma_commit(&xempty[sx]);
+        if (DQX || u + NI >= (t + 1) * kUnitsPerX || u + NI >= nunits)
+          mma_commit(&xempty[sx]);  // this thread's last unit of the stage
       }
       mma_commit(&accum[j]);  // fires once every MMA this thread issued has completed
     }
@@ -429,18 +444,18 @@ tc_w4a16_kernel(const __grid_constant__ CUtensorMap xmap, const TcArgs a) {
     const uint32_t lane_addr = (uint32_t)(32 * q) << 16;
     const int sf_off = 16 * lane + 4 * q;         // this row's 4 scale bytes (block layout)
     for (int u = g; u < nunits; u += DQG) {
-      const int sa = u % SA, sw = u % SWU, sx = u % SXU;
+      const int r = u / DQG, sw = r % SWS, sa = u % SA;
       if (u >= SA) {  // the MMAs that read this TMEM slot SA units ago are done
         const bool ok = mbar_wait(&aempty[sa], ((u / SA) - 1) & 1, abort_flag, err, 4);
         if (!__all_sync(0xffffffffu, ok)) break;
         tc_fence_after();
       }
-      bool ok = mbar_wait(&wfull[sw], (u / SWU) & 1, abort_flag, err, 4);
+      const bool ok = mbar_wait(&wfull[sw], (r / SWS) & 1, abort_flag, err, 4);
       if (!__all_sync(0xffffffffu, ok)) break;  // stay converged for tcgen05.st
-      const int nc = min(U, nk - u * U);
-      const uint8_t* wst = wsm + sw * C::kWStageBytes;
+      const uint8_t* wu = wsm + sw * C::kWStageBytes + g * C::kUnitBytes;
+      const int nc = min(UA, nk - u * UA);
       for (int c = 0; c < nc; ++c) {
-        const uint8_t* w = wst + c * kChunkBytes;
+        const uint8_t* w = wu + c * kChunkBytes;
         const uint4 lo = *reinterpret_cast<const uint4*>(w + 16 * row);
         const uint4 hi = *reinterpret_cast<const uint4*>(w + 2048 + 16 * row);
         const uint32_t sc = *reinterpret_cast<const uint32_t*>(w + 4096 + sf_off);
@@ -450,8 +465,10 @@ tc_w4a16_kernel(const __grid_constant__ CUtensorMap xmap, const TcArgs a) {
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(&wempty[sw]);   // the shared-memory stage may be refilled
-      ok = mbar_wait(&xfull[sx], (u / SXU) & 1, abort_flag, err, 4);  // the unit's activations
-      if (!__all_sync(0xffffffffu, ok)) break;
+      if (DQX) {  // the unit's activations, on the MMA thread's behalf
+        const bool okx = mbar_wait(&xfull[u % SXS], (u / SXS) & 1, abort_flag, err, 4);
+        if (!__all_sync(0xffffffffu, okx)) break;
+      }
       tmem_st_wait();
       tc_fence_before();
       __syncwarp();
@@ -725,10 +742,10 @@ bool make_x_map(CUtensorMap* map, const void* x, int64_t m, int64_t k, int box_r
              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int BN, int SXU, int SWU, int SA, int DQG, int U, int NI, int EPI>
+template <int BN, int SXS, int XC, int SWS, int SA, int DQG, int UA, int NI, bool DQX, int EPI>
 cudaError_t launch_cfg(const CUtensorMap& map, const TcArgs& a, dim3 grid, cudaStream_t s) {
-  using C = TcCfg<BN, SXU, SWU, SA, DQG, U, NI>;
-  auto kern = tc_w4a16_kernel<BN, SXU, SWU, SA, DQG, U, NI, EPI>;
+  using C = TcCfg<BN, SXS, XC, SWS, SA, DQG, UA, NI, DQX>;
+  auto kern = tc_w4a16_kernel<BN, SXS, XC, SWS, SA, DQG, UA, NI, DQX, EPI>;
   static bool attr_set = false;  // per instantiation; idempotent if raced
   if (!attr_set) {
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemAlloc);
@@ -742,14 +759,15 @@ cudaError_t launch_cfg(const CUtensorMap& map, const TcArgs& a, dim3 grid, cudaS
 template <int EPI>
 cudaError_t launch_bn(int bn, const CUtensorMap& map, const TcArgs& a, dim3 grid, cudaStream_t s) {
   switch (bn) {
-    // BN, activation stages, weight stages, TMEM slots (all in units), dequant
-    // warpgroups, chunks per unit, MMA issuers.  TMEM: NI*BN + 32*U*SA columns
-    // (<= 256 for two CTAs per SM).
-    case 16: return launch_cfg<16, 4, 8, 2, 2, 2, 2, EPI>(map, a, grid, s);
-    case 32: return launch_cfg<32, 4, 8, 2, 2, 2, 2, EPI>(map, a, grid, s);
-    case 64: return launch_cfg<64, 2, 8, 2, 2, 2, 2, EPI>(map, a, grid, s);
-    case 128: return launch_cfg<128, 3, 5, 2, 2, 2, 1, EPI>(map, a, grid, s);
-    default: return launch_cfg<256, 2, 6, 2, 2, 2, 1, EPI>(map, a, grid, s);
+    // BN, activation stages, chunks per activation stage, weight stages
+    // (rounds), TMEM A slots (units), dequant warpgroups, chunks per unit, MMA
+    // threads, activation wait by the dequant warps.  TMEM: max(32, NI*BN) +
+    // 32*UA*SA columns (<= 256 for two CTAs per SM).
+    case 16: return launch_cfg<16, 2, 8, 8, 6, 2, 1, 2, false, EPI>(map, a, grid, s);
+    case 32: return launch_cfg<32, 2, 4, 8, 6, 2, 1, 2, false, EPI>(map, a, grid, s);
+    case 64: return launch_cfg<64, 2, 2, 8, 4, 2, 1, 2, false, EPI>(map, a, grid, s);
+    case 128: return launch_cfg<128, 4, 2, 3, 4, 2, 2, 1, true, EPI>(map, a, grid, s);
+    default: return launch_cfg<256, 2, 2, 4, 4, 2, 2, 1, true, EPI>(map, a, grid, s);
   }
 }
 
