@@ -215,10 +215,19 @@ def run_ours(args, rank, world, dist):
     barrier()
     graph.replay()  # the timed region: K steps
     barrier()
-    prof = N.ffn_nvfp4_profile_end()
-    clk = clocks.stop()
     ms = max_over_ranks(sum(a.elapsed_time(b) for a, b in zip(starts, stops)), dist, "cuda")
     del graph
+    # per-kernel durations: the same K steps with an event pair around every
+    # kernel (events between kernels also stop them from overlapping, which is
+    # why the timed replay above has none)
+    pgraph, _, _ = capture_steps(N, wl, args.steps, flush, profile=True)
+    pgraph.replay()
+    barrier()
+    pgraph.replay()
+    barrier()
+    prof = N.ffn_nvfp4_profile_end()
+    clk = clocks.stop()
+    del pgraph
     ms_step = ms / args.steps
     flops = ffn_flops(wl.m, wl.H, wl.I)
     value = aggregate_throughput(flops, args.steps, ms, world) / 1e12
@@ -284,17 +293,18 @@ def run_ours(args, rank, world, dist):
     }
 
 
-def capture_steps(N, wl, steps, flush):
+def capture_steps(N, wl, steps, flush, profile=False):
     """Capture `steps` forward steps (each after an optional L2 flush, between
-    a pair of timing events) into one CUDA graph, with the library's per-kernel
-    profiling on, so every timestamp is taken on the device during replay and
-    none includes host launch latency.  Returns (graph, starts, stops); the
-    profiling recording stays open until ffn_nvfp4_profile_end."""
+    a pair of timing events) into one CUDA graph, so every timestamp is taken
+    on the device during replay and none includes host launch latency.  With
+    `profile`, the library's per-kernel events are captured too (the recording
+    stays open until ffn_nvfp4_profile_end).  Returns (graph, starts, stops)."""
     import torch
     starts = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(steps)]
     stops = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(steps)]
     graph = torch.cuda.CUDAGraph()
-    N.ffn_nvfp4_profile_begin()
+    if profile:
+        N.ffn_nvfp4_profile_begin()
     with torch.cuda.graph(graph, stream=torch.cuda.Stream()):
         for i in range(steps):
             if flush is not None:
@@ -318,9 +328,15 @@ def secondary(N, name, m, peaks, steps):
     torch.cuda.synchronize()
     graph.replay()
     torch.cuda.synchronize()
-    prof = N.ffn_nvfp4_profile_end()
     ms = sum(a.elapsed_time(b) for a, b in zip(starts, stops)) / steps
     del graph
+    pgraph, _, _ = capture_steps(N, wl, steps, flush, profile=True)
+    pgraph.replay()
+    torch.cuda.synchronize()
+    pgraph.replay()
+    torch.cuda.synchronize()
+    prof = N.ffn_nvfp4_profile_end()
+    del pgraph
     res = {"m": m, "hidden": wl.H, "inter": wl.I, "format": wl.fmt, "us_per_layer": round(ms * 1e3, 2),
            "weight_gbs": round(wl.weight_bytes / (ms * 1e-3) / 1e9, 1),
            "tflops": round(ffn_flops(m, wl.H, wl.I) / (ms * 1e-3) / 1e12, 3),
@@ -432,7 +448,8 @@ def main():
         "data": "synthetic (seeded numpy draws; random-init weights)",
         "config": {"workload": args.workload, "m": res["m"], "hidden": H, "inter": I, "act_format": fmt,
                    "parallelism": f"replicas x{world}", "l2": res["l2"],
-                   "launch": "the K timed steps captured in one CUDA graph, replayed once"},
+                   "launch": "the K timed steps captured in one CUDA graph, replayed once; "
+                             "kernel durations from a second replay with an event pair per kernel"},
         "roofline": res["roofline"], "cpu_baseline": cpu, "e2e": res["e2e"],
         "gpu_launches": res["gpu_launches"], "kernels": res["kernels"], "clocks": res["clocks"],
     }

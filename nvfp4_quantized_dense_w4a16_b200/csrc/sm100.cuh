@@ -69,6 +69,18 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
   }
 }
 
+// ------------------------------------------- programmatic dependent launch
+// A kernel launched with programmatic stream serialisation may start while
+// the previous kernel in the stream is still running.  griddep_wait blocks
+// until that kernel has completed and its writes are visible (a no-op for a
+// kernel launched normally); every thread that reads the previous kernel's
+// output or writes memory it may still read calls it first.
+// griddep_launch_dependents lets the next such kernel start now.
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void griddep_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // ------------------------------------------------------------- async copies
 
 // 2-D tiled TMA load of a box at (c0 = innermost, c1) into shared memory,

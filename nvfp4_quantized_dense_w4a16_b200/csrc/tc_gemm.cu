@@ -29,6 +29,7 @@
 #include <cudaTypedefs.h>
 
 #include <mutex>
+#include <utility>
 
 #include "common.cuh"
 #include "internal.h"
@@ -371,6 +372,9 @@ tc_w4a16_kernel(const __grid_constant__ CUtensorMap xmap, const TcArgs a) {
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  // The next kernel may be scheduled now; the weights streamed here do not
+  // depend on the previous kernel, the activations and the output do.
+  griddep_launch_dependents();
 
   if (warp == 0) {
     // ------------------------------------------------- weight producer
@@ -393,6 +397,7 @@ tc_w4a16_kernel(const __grid_constant__ CUtensorMap xmap, const TcArgs a) {
   } else if (warp == 3) {
     // --------------------------------------------- activation producer
     if (lane == 0) {
+      griddep_wait();  // the activations may come from the previous kernel
       const int stages = (nk + XC - 1) / XC;
       int issued = 0;
       for (int t = 0; t < stages; ++t) {
@@ -478,6 +483,7 @@ tc_w4a16_kernel(const __grid_constant__ CUtensorMap xmap, const TcArgs a) {
     for (int j = 0; j < NI; ++j) done = wait_drain(&accum[j], 0) && done;
     done = __all_sync(0xffffffffu, done);
     tc_fence_after();
+    griddep_wait();  // the previous kernel may still read the output buffer
     if (done && !*abort_flag)
       epilogue_tile<BN, EPI, DQG, NI>(a, tmem, q, lane, g, epi + g * C::kEpiBytes, xtile, wtile,
                                       min(NI, nunits), kW4A16Unscale);
@@ -636,6 +642,8 @@ template <bool kGateUp>
 __global__ void splitk_reduce_kernel(const float* __restrict__ P, int splits, int m, int n_pad,
                                      int n_out, const float* __restrict__ gs, float gs_mul,
                                      uint16_t* __restrict__ out, int ldo) {
+  griddep_wait();  // the partial sums come from the previous kernel
+  griddep_launch_dependents();
   const int64_t idx = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;
   if (idx >= (int64_t)m * n_out) return;
   const int r = (int)(idx / n_out), n = (int)(idx % n_out);
@@ -742,6 +750,25 @@ bool make_x_map(CUtensorMap* map, const void* x, int64_t m, int64_t k, int box_r
              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// Launch with programmatic stream serialisation: the kernel may begin while
+// the previous kernel in the stream finishes (the kernels wait for its
+// results with griddep_wait).
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
+                       Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
+}
+
 template <int BN, int SXS, int XC, int SWS, int SA, int DQG, int UA, int NI, bool DQX, int EPI>
 cudaError_t launch_cfg(const CUtensorMap& map, const TcArgs& a, dim3 grid, cudaStream_t s) {
   using C = TcCfg<BN, SXS, XC, SWS, SA, DQG, UA, NI, DQX>;
@@ -752,8 +779,7 @@ cudaError_t launch_cfg(const CUtensorMap& map, const TcArgs& a, dim3 grid, cudaS
     if (e != cudaSuccess) return e;
     attr_set = true;
   }
-  kern<<<grid, C::kThreads, C::kSmemAlloc, s>>>(map, a);
-  return cudaGetLastError();
+  return launch_pdl(kern, grid, dim3(C::kThreads), C::kSmemAlloc, s, map, a);
 }
 
 template <int EPI>
@@ -840,15 +866,14 @@ cudaError_t launch_tc_w4a16(const void* x, int64_t m, const TcWeight& w, bool si
     if (e != cudaSuccess) return e;
     const int64_t total = m * a.n_out;
     ProfScope prof(s, silu_mul ? "splitk_reduce_silu_mul" : "splitk_reduce");
-    if (silu_mul)
-      splitk_reduce_kernel<true><<<(unsigned)((total + 255) / 256), 256, 0, s>>>(
-          (const float*)partials, p.splits, (int)m, p.n_pad, a.n_out, w.gs, kW4A16Unscale,
-          (uint16_t*)y, a.ldo);
-    else
-      splitk_reduce_kernel<false><<<(unsigned)((total + 255) / 256), 256, 0, s>>>(
-          (const float*)partials, p.splits, (int)m, p.n_pad, a.n_out, w.gs, kW4A16Unscale,
-          (uint16_t*)y, a.ldo);
-    return cudaGetLastError();
+    const dim3 rgrid((unsigned)((total + 255) / 256));
+    const float* P = static_cast<const float*>(partials);
+    return silu_mul ? launch_pdl(splitk_reduce_kernel<true>, rgrid, dim3(256), 0, s, P, p.splits,
+                                 (int)m, p.n_pad, a.n_out, w.gs, kW4A16Unscale,
+                                 static_cast<uint16_t*>(y), a.ldo)
+                    : launch_pdl(splitk_reduce_kernel<false>, rgrid, dim3(256), 0, s, P, p.splits,
+                                 (int)m, p.n_pad, a.n_out, w.gs, kW4A16Unscale,
+                                 static_cast<uint16_t*>(y), a.ldo);
   }
   a.out = y;
   ProfScope prof(s, silu_mul ? "tc_w4a16_gate_up_silu" : "tc_w4a16");
