@@ -80,6 +80,34 @@ def nvfp4_bytes(n, k):
 
 # --------------------------------------------------------------- clocks
 
+# DRAM traffic per launch (dram__bytes_read.sum + dram__bytes_write.sum) from
+# one ncu capture, keyed by (kernel, workload), with a fingerprint of the kernel
+# sources it was taken on: reported only while the sources are unchanged.
+KERNEL_SOURCES = ("csrc/tc_gemm.cu", "csrc/sm100.cuh", "csrc/common.cuh", "csrc/internal.h")
+TRAFFIC = {
+    ("tc_w4a16_gate_up_silu", "prefill"): {
+        "bytes": 148931840 + 131985920, "sources_sha1": "f706c30fd1af98f501d43537f939adf4bed8c391",
+        "profile": "profiles/tc_w4a16_gate_up_prefill_m4096.md"},
+}
+
+
+def kernel_sources_sha1():
+    import hashlib
+    h = hashlib.sha1()
+    pkg = os.path.join(os.path.dirname(os.path.abspath(__file__)), "nvfp4_quantized_dense_w4a16_b200")
+    for f in KERNEL_SOURCES:
+        with open(os.path.join(pkg, f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()
+
+
+def measured_traffic(kname, workload):
+    t = TRAFFIC.get((kname, workload))
+    if t is None or t["sources_sha1"] != kernel_sources_sha1():
+        return None
+    return t["bytes"]
+
+
 class Clocks:
     """nvidia-smi sampling of SM clocks and throttle reasons while running."""
     Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
@@ -91,13 +119,24 @@ class Clocks:
         self.proc = None
         self.tmp = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
 
+    @staticmethod
+    def _die_with_parent():
+        # the sampler must not outlive this process, even if it crashes
+        # (a profiler waits for every process of the tree to exit)
+        import ctypes
+        import signal
+        ctypes.CDLL("libc.so.6", use_errno=True).prctl(1, signal.SIGTERM)  # PR_SET_PDEATHSIG
+
     def start(self):
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.Q}", "--format=csv,noheader,nounits",
-                 "-lms", "50"], stdout=self.tmp, stderr=subprocess.DEVNULL)
+                 "-lms", "50"], stdout=self.tmp, stderr=subprocess.DEVNULL, preexec_fn=self._die_with_parent)
         except OSError:
             self.proc = None
+        if self.proc is not None:
+            import atexit
+            atexit.register(self.proc.kill)
 
     def stop(self):
         if self.proc is None:
@@ -210,24 +249,9 @@ def run_ours(args, rank, world, dist):
     for i in range(args.warmup):
         wl.step(i)
     barrier()
-    graph, starts, stops = capture_steps(N, wl, args.steps, flush)
-    graph.replay()  # untimed: loads the graph onto the device
-    barrier()
-    graph.replay()  # the timed region: K steps
-    barrier()
-    ms = max_over_ranks(sum(a.elapsed_time(b) for a, b in zip(starts, stops)), dist, "cuda")
-    del graph
-    # per-kernel durations: the same K steps with an event pair around every
-    # kernel (events between kernels also stop them from overlapping, which is
-    # why the timed replay above has none)
-    pgraph, _, _ = capture_steps(N, wl, args.steps, flush, profile=True)
-    pgraph.replay()
-    barrier()
-    pgraph.replay()
-    barrier()
-    prof = N.ffn_nvfp4_profile_end()
+    ms_local, prof = time_steps(N, wl, args.steps, flush, args.eager, barrier)
+    ms = max_over_ranks(ms_local, dist, "cuda")
     clk = clocks.stop()
-    del pgraph
     ms_step = ms / args.steps
     flops = ffn_flops(wl.m, wl.H, wl.I)
     value = aggregate_throughput(flops, args.steps, ms, world) / 1e12
@@ -248,7 +272,8 @@ def run_ours(args, rank, world, dist):
             unit = "GB/s"
         roof = {"kernel": kname, "bound": bound, "achieved": round(achieved, 2), "peak": peak,
                 "peak_source": peak_src, "unit": unit, "frac": round(achieved / peak, 4),
-                "traffic": None, "avg_launch_us": round(avg_s * 1e6, 2), "launches": launches}
+                "traffic": measured_traffic(kname, args.workload),
+                "avg_launch_us": round(avg_s * 1e6, 2), "launches": launches}
     kernels = {k: {"launches": l, "total_ms": round(t, 4), "share": round(t / max(1e-9, sum(v[1] for v in prof.values())), 4)}
                for k, (l, t) in prof.items()}
     gpu_launches = sum(v[0] for v in prof.values())
@@ -282,8 +307,8 @@ def run_ours(args, rank, world, dist):
     if not args.no_extra and args.workload == "prefill":
         del wl, x_dev
         torch.cuda.empty_cache()
-        extra["decode_m1"] = secondary(N, "decode", 1, peaks, steps=max(args.steps, 20))
-        extra["w4a4_m512"] = secondary(N, "w4a4", 512, peaks, steps=max(args.steps // 2, 5))
+        extra["decode_m1"] = secondary(N, "decode", 1, peaks, max(args.steps, 20), args.eager)
+        extra["w4a4_m512"] = secondary(N, "w4a4", 512, peaks, max(args.steps // 2, 5), args.eager)
         torch.cuda.empty_cache()
     return {
         "value": round(value, 3), "ms_per_step": round(ms_step, 4), "roofline": roof,
@@ -291,6 +316,47 @@ def run_ours(args, rank, world, dist):
         "workload": args.workload, "m": args.m or WORKLOADS[args.workload][1], "extra": extra,
         "l2": l2_note,
     }
+
+
+def time_steps(N, wl, steps, flush, eager, barrier):
+    """Time `steps` forward steps; returns (total ms, per-kernel profile).
+
+    Default: the steps are captured in one CUDA graph with a timing-event pair
+    around each step, replayed once untimed and once timed; per-kernel
+    durations come from a second graph of the same steps with an event pair
+    around every kernel (events between kernels also keep them from
+    overlapping, which is why the timed graph has none).  With `eager` (for
+    runs under a profiler) the steps are launched directly and timed with the
+    same events, which then include host launch latency."""
+    import torch
+    if eager:
+        starts = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+        stops = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+        N.ffn_nvfp4_profile_begin()
+        for i in range(steps):
+            if flush is not None:
+                flush.zero_()
+            starts[i].record()
+            wl.step(i)
+            stops[i].record()
+        barrier()
+        prof = N.ffn_nvfp4_profile_end()
+        return sum(a.elapsed_time(b) for a, b in zip(starts, stops)), prof
+    graph, starts, stops = capture_steps(N, wl, steps, flush)
+    graph.replay()  # untimed: loads the graph onto the device
+    barrier()
+    graph.replay()  # the timed region
+    barrier()
+    ms = sum(a.elapsed_time(b) for a, b in zip(starts, stops))
+    del graph
+    pgraph, _, _ = capture_steps(N, wl, steps, flush, profile=True)
+    pgraph.replay()
+    barrier()
+    pgraph.replay()
+    barrier()
+    prof = N.ffn_nvfp4_profile_end()
+    del pgraph
+    return ms, prof
 
 
 def capture_steps(N, wl, steps, flush, profile=False):
@@ -315,7 +381,7 @@ def capture_steps(N, wl, steps, flush, profile=False):
     return graph, starts, stops
 
 
-def secondary(N, name, m, peaks, steps):
+def secondary(N, name, m, peaks, steps, eager=False):
     """Time another layer shape: per-step µs, weight GB/s and TFLOP/s."""
     import torch
     wl = Workload(N, name, m)
@@ -323,20 +389,8 @@ def secondary(N, name, m, peaks, steps):
     for i in range(3):
         wl.step(i)
     torch.cuda.synchronize()
-    graph, starts, stops = capture_steps(N, wl, steps, flush)
-    graph.replay()
-    torch.cuda.synchronize()
-    graph.replay()
-    torch.cuda.synchronize()
-    ms = sum(a.elapsed_time(b) for a, b in zip(starts, stops)) / steps
-    del graph
-    pgraph, _, _ = capture_steps(N, wl, steps, flush, profile=True)
-    pgraph.replay()
-    torch.cuda.synchronize()
-    pgraph.replay()
-    torch.cuda.synchronize()
-    prof = N.ffn_nvfp4_profile_end()
-    del pgraph
+    ms, prof = time_steps(N, wl, steps, flush, eager, torch.cuda.synchronize)
+    ms /= steps
     res = {"m": m, "hidden": wl.H, "inter": wl.I, "format": wl.fmt, "us_per_layer": round(ms * 1e3, 2),
            "weight_gbs": round(wl.weight_bytes / (ms * 1e-3) / 1e9, 1),
            "tflops": round(ffn_flops(m, wl.H, wl.I) / (ms * 1e-3) / 1e12, 3),
@@ -411,6 +465,9 @@ def main():
     ap.add_argument("--m", type=int, default=None)
     ap.add_argument("--no-extra", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
+    ap.add_argument("--eager", action="store_true",
+                    help="launch the timed steps directly instead of through a CUDA graph "
+                         "(for runs under a profiler; times then include launch latency)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -448,8 +505,9 @@ def main():
         "data": "synthetic (seeded numpy draws; random-init weights)",
         "config": {"workload": args.workload, "m": res["m"], "hidden": H, "inter": I, "act_format": fmt,
                    "parallelism": f"replicas x{world}", "l2": res["l2"],
-                   "launch": "the K timed steps captured in one CUDA graph, replayed once; "
-                             "kernel durations from a second replay with an event pair per kernel"},
+                   "launch": ("eager launches" if args.eager else
+                              "the K timed steps captured in one CUDA graph, replayed once; "
+                              "kernel durations from a second replay with an event pair per kernel")},
         "roofline": res["roofline"], "cpu_baseline": cpu, "e2e": res["e2e"],
         "gpu_launches": res["gpu_launches"], "kernels": res["kernels"], "clocks": res["clocks"],
     }
