@@ -11,13 +11,18 @@ import numpy as np
 
 from oracle import nvfp4_ffn as O
 
-M, MA, MB = 0x81C081C0, 0x81808180, 0x00400040
+M, MA, MB = 0x81C081C0, 0x80C080C0, 0x01000100
 POS = [6, 7, 8, 15]          # destination bits of code bits m, e0, e1, s
 
 
 def src_bit(k, p):
-    r = 0 if k == 0 else 4 if k == 1 else 10 if k == 2 else (14 if (p & 15) == 6 else 6)
-    return (p + r) & 31
+    if k == 0:
+        return p
+    if k == 1:
+        return p - 4
+    if k == 2:
+        return (p + 6) & 31
+    return (p + 2) & 31 if (p & 15) == 8 else p - 6
 
 
 def permute(nat):
@@ -34,7 +39,8 @@ def rotr(x, r):
 
 
 def decode(c):
-    return [c & M, rotr(c, 4) & M, rotr(c, 10) & M, (rotr(c, 6) & MA) | (rotr(c, 14) & MB)]
+    shl = lambda x, k: (x << k) & 0xFFFFFFFF
+    return [c & M, shl(c, 4) & M, rotr(c, 6) & M, (shl(c, 6) & MA) | (rotr(c, 2) & MB)]
 
 
 def bf16_value(bits16):
