@@ -86,7 +86,7 @@ def nvfp4_bytes(n, k):
 KERNEL_SOURCES = ("csrc/tc_gemm.cu", "csrc/sm100.cuh", "csrc/common.cuh", "csrc/internal.h")
 TRAFFIC = {
     ("tc_w4a16_gate_up_silu", "prefill"): {
-        "bytes": 148931840 + 131985920, "sources_sha1": "f706c30fd1af98f501d43537f939adf4bed8c391",
+        "bytes": 146800896 + 128328960, "sources_sha1": "d8d96a35fd126d08397e3ecf5c0868cc138ca51d",
         "profile": "profiles/tc_w4a16_gate_up_prefill_m4096.md"},
 }
 

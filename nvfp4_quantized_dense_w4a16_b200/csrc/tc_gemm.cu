@@ -758,7 +758,8 @@ bool make_x_map(CUtensorMap* map, const void* x, int64_t m, int64_t k, int box_r
 
 // Launch with programmatic stream serialisation: the kernel may begin while
 // the previous kernel in the stream finishes (the kernels wait for its
-// results with griddep_wait).
+// results with griddep_wait).  Not while per-kernel timing is recorded: an
+// event between two kernels must not let the second start early.
 template <typename... KArgs, typename... Args>
 cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
                        Args&&... args) {
@@ -771,7 +772,7 @@ cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t sme
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = profiling() ? 0 : 1;
   return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
 }
 
