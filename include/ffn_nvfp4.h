@@ -156,7 +156,14 @@ ffn_status ffn_nvfp4_workspace_size(int64_t m, int64_t hidden, int64_t inter,
  * x and h are quantised per row (as ffn_nvfp4_quantize_activations) before
  * their projections, and the kernels and reduction order do not depend on m,
  * so each output row is bit-identical whatever m is.
- * m == 0 is a no-op.  Allocates nothing and does not synchronise. */
+ * m == 0 is a no-op.  Allocates nothing and does not synchronise.
+ * Launch order: the bf16-format kernels are launched with programmatic stream
+ * serialisation, so each may start while the previous kernel in the stream is
+ * finishing; it streams and dequantises weights meanwhile and waits for that
+ * kernel's completion before reading x (or h) and before writing out, h or
+ * the workspace.  Stream order is therefore kept for every buffer the call
+ * reads or writes except the weight handles, which must not be modified by
+ * an earlier kernel still in flight (handles are immutable after creation). */
 ffn_status ffn_nvfp4_forward(const void* x, int64_t m, int64_t hidden, int64_t inter,
                              const ffn_nvfp4_weight* gate_up, const ffn_nvfp4_weight* down,
                              ffn_act_format format, void* out, void* workspace,
