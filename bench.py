@@ -82,22 +82,35 @@ def nvfp4_bytes(n, k):
 
 # DRAM traffic per launch (dram__bytes_read.sum + dram__bytes_write.sum) from
 # one ncu capture, keyed by (kernel, workload), with a fingerprint of the kernel
-# sources it was taken on: reported only while the sources are unchanged.
+# sources it was taken on (comments and whitespace ignored): reported only
+# while the sources are unchanged.
 KERNEL_SOURCES = ("csrc/tc_gemm.cu", "csrc/sm100.cuh", "csrc/common.cuh", "csrc/internal.h")
 TRAFFIC = {
     ("tc_w4a16_gate_up_silu", "prefill"): {
-        "bytes": 146800896 + 128328960, "sources_sha1": "d8d96a35fd126d08397e3ecf5c0868cc138ca51d",
+        "bytes": 146800896 + 128328960, "sources_sha1": "5976b4c07ea6be5b9cb88fe0ad51fe53f300e557",
         "profile": "profiles/tc_w4a16_gate_up_prefill_m4096.md"},
 }
 
 
-def kernel_sources_sha1():
+def normalised_source(text):
+    """Source text without comments and whitespace (edits to either do not
+    change the compiled kernel)."""
+    import re
+    text = re.sub(r"/\*.*?\*/", " ", text, flags=re.S)
+    text = re.sub(r"//[^\n]*", " ", text)
+    return re.sub(r"\s+", "", text)
+
+
+def kernel_sources_sha1(read=None):
     import hashlib
-    h = hashlib.sha1()
     pkg = os.path.join(os.path.dirname(os.path.abspath(__file__)), "nvfp4_quantized_dense_w4a16_b200")
+    if read is None:
+        def read(rel):
+            with open(os.path.join(pkg, rel), encoding="utf-8") as fh:
+                return fh.read()
+    h = hashlib.sha1()
     for f in KERNEL_SOURCES:
-        with open(os.path.join(pkg, f), "rb") as fh:
-            h.update(fh.read())
+        h.update(normalised_source(read(f)).encode())
     return h.hexdigest()
 
 

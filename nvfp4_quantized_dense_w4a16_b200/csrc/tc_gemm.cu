@@ -6,24 +6,28 @@
 // Design (one CTA per 128-weight-row tile x BN activation rows x K range):
 //  * weights are streamed in a pre-tiled layout (per 128-row tile and
 //    64-element K chunk: 128 x 16 B low codes, 128 x 16 B high codes,
-//    128 x 4 B E4M3 scales = 4608 B) by one bulk async copy per stage; the
-//    codes are the canonical no-swizzle K-major operand layout of the
-//    block-scaled FP4 MMA and the scale bytes its 512-byte scale-factor block
-//    (row r at byte 16*(r%32) + 4*(r/32)), so the W4A4 kernel streams the
-//    same bytes;
+//    128 x 4 B E4M3 scales = 4608 B) by bulk async copies.  The natural-code
+//    copy is the canonical no-swizzle K-major operand of the block-scaled FP4
+//    MMA with its 512-byte scale-factor block (row r at byte
+//    16*(r%32) + 4*(r/32)), streamed by the W4A4 kernel; the bf16-activation
+//    kernel streams a second copy whose code bits are rearranged for a cheap
+//    decode (see "W4A16 operand decoding");
 //  * activations X [m, K] bf16 arrive by 2-D TMA with the 128-byte swizzle
 //    (box 64 x BN), the layout the MMA reads directly;
-//  * four dequant warps turn each thread's row of codes into exact bf16
-//    values (E2M1 value * E4M3 block scale: at most 6 significant bits) with
-//    byte-permute table lookups and write them straight into tensor memory,
-//    where they are the MMA's A operand (M = 128 weight rows) -- so the
-//    dequantised weights never occupy shared-memory bandwidth;
-//  * one thread issues tcgen05.mma kind::f16 (A from TMEM, B = X tile from
-//    shared memory, fp32 accumulator in TMEM, N = BN);
-//  * the four dequant warps then read the accumulator back (tcgen05.ld) and
-//    run the epilogue: y = bf16(gs * acc); or for the fused gate+up weight
-//    (64 gate rows then the matching 64 up rows per tile) the SiLU*mul
-//    h = bf16(silu(bf16(gs_g*g)) * bf16(gs_u*u)); or fp32 split-K partials.
+//  * dequant warpgroups (four warps, one per TMEM lane quarter) turn each
+//    thread's row of codes into exact bf16 values (E2M1 * E4M3 scale * 2^-8:
+//    at most 6 significant bits) with rotations, masks and one bf16x2
+//    multiply, and write them straight into tensor memory, where they are the
+//    MMA's A operand (M = 128 weight rows) -- so the dequantised weights never
+//    occupy shared-memory bandwidth;
+//  * one to three threads issue tcgen05.mma kind::f16 (A from TMEM, B = X
+//    tile from shared memory, an fp32 accumulator each in TMEM, N = BN);
+//  * the dequant warps then read the accumulators back (tcgen05.ld), add them
+//    in a fixed order and run the epilogue: y = bf16(gs * acc); or for the
+//    fused gate+up weight (64 gate rows then the matching 64 up rows per tile)
+//    h = bf16(silu(bf16(gs_g*g)) * bf16(gs_u*u)); or fp32 split-K partials;
+//  * the kernels are launched with programmatic dependent launch and wait for
+//    the previous kernel only before reading activations and writing results.
 // Pipelines are mbarrier-driven; every wait is bounded and, on timeout, sets
 // a device error bit and lets the CTA free its TMEM and exit.
 #include <cudaTypedefs.h>
