@@ -1,0 +1,73 @@
+"""CPU tests of bench.py's host-side logic: which layers rotate through weight
+copies (and how many), that every timed step uses the copy it should, and the
+kernel-source fingerprint that gates the reported DRAM traffic."""
+import types
+
+import numpy as np
+import pytest
+import torch
+
+import bench
+
+
+@pytest.fixture
+def cpu_torch(monkeypatch):
+    # run Workload on the CPU: no device transfers, no synchronisation
+    monkeypatch.setattr(torch.Tensor, "cuda", lambda self, *a, **k: self)
+    monkeypatch.setattr(torch.cuda, "synchronize", lambda *a, **k: None)
+    real_empty = torch.empty
+
+    def empty(*a, **k):
+        k.pop("device", None)
+        return real_empty(*a, **k)
+    monkeypatch.setattr(torch, "empty", empty)
+
+
+def fake_native(calls):
+    counter = iter(range(10**6))
+    return types.SimpleNamespace(
+        ffn_nvfp4_quantize_weights=lambda w: (w, w, w),
+        ffn_nvfp4_weight_create=lambda c, s, g: ("w", next(counter)),
+        ffn_nvfp4_weight_create_gate_up=lambda g, u: ("gu", g, u),
+        ffn_nvfp4_workspace_size=lambda m, H, I, f: 1024,
+        ffn_nvfp4_forward=lambda x, gu, d, f, out=None, workspace=None: calls.append((gu, d)))
+
+
+@pytest.mark.parametrize("name,m", [("decode", 1), ("w4a4", 512)])
+def test_small_layers_rotate_weight_copies(cpu_torch, name, m):
+    calls = []
+    wl = bench.Workload(fake_native(calls), name, m)
+    assert wl.sets >= 2
+    assert wl.sets * wl.weight_bytes >= 4 * bench.L2_BYTES
+    assert (wl.sets - 1) * wl.weight_bytes < 4 * bench.L2_BYTES  # no more copies than needed
+    assert "rotated" in wl.l2_note
+    for i in range(2 * wl.sets):
+        wl.step(i)
+    # step i uses copy i mod R, and the R copies are distinct handles
+    used = [c[0] for c in calls]
+    assert used[:wl.sets] == used[wl.sets:]
+    assert len({id(h) for h in used[:wl.sets]}) == wl.sets
+
+
+def test_weight_bytes_are_the_nvfp4_footprint(cpu_torch):
+    wl = bench.Workload(fake_native([]), "decode", 1)
+    H, I = 5120, 17408
+    assert wl.weight_bytes == 3 * H * I * (0.5 + 1 / 16)
+
+
+def test_fingerprint_ignores_comments_and_whitespace():
+    a = "int f(int x) {\n  // note\n  return x + 1; /* block\n comment */\n}\n"
+    b = "int f(int x){return x+1;}"
+    c = "int f(int x){return x+2;}"
+    assert bench.normalised_source(a) == bench.normalised_source(b)
+    assert bench.normalised_source(a) != bench.normalised_source(c)
+
+
+def test_traffic_reported_only_for_the_captured_sources():
+    files = {f: "kernel body" for f in bench.KERNEL_SOURCES}
+    sha = bench.kernel_sources_sha1(lambda rel: files[rel])
+    files[bench.KERNEL_SOURCES[0]] = "kernel body // with a comment"
+    assert bench.kernel_sources_sha1(lambda rel: files[rel]) == sha
+    files[bench.KERNEL_SOURCES[0]] = "changed kernel body"
+    assert bench.kernel_sources_sha1(lambda rel: files[rel]) != sha
+    assert bench.measured_traffic("no_such_kernel", "prefill") is None
