@@ -79,7 +79,7 @@ struct TcCfg {
   static constexpr int kXStageBytes = XC * BN * 128;   // XC chunk tiles of BN rows x 128 B
   static constexpr int kUnitBytes = UA * kChunkBytes;
   static constexpr int kWStageBytes = DQG * kUnitBytes;
-  static constexpr int kAColBase = (NI * BN + 31) / 32 * 32;  // TMEM column of A slot 0
+  static constexpr int kAColBase = NI * BN < 32 ? 32 : NI * BN;  // TMEM column of A slot 0
   static constexpr int kSlotCols = 32 * UA;
   static constexpr int kTmemNeed = kAColBase + kSlotCols * SA;
   static constexpr int kTmemCols = kTmemNeed <= 64 ? 64 : kTmemNeed <= 128 ? 128 : kTmemNeed <= 256 ? 256 : 512;
@@ -98,7 +98,7 @@ struct TcCfg {
   static_assert(kTmemNeed <= 512, "TMEM budget");
   static_assert(kSmemAlloc <= 232448, "shared memory budget");
   static_assert(BN % 16 == 0 && BN >= 16 && BN <= 256, "MMA N");
-  static_assert(DQG >= 1 && DQG <= 3 && NI >= 1 && NI <= 3 && UA >= 1, "roles");
+  static_assert(DQG >= 1 && DQG <= 3 && (NI == 1 || NI == 2) && UA >= 1, "roles");
   static_assert(kSmemRings >= DQG * kEpiBytes, "epilogue buffers alias the rings");
   // A parity wait can only tell the awaited phase from the one before it, so
   // the previous phase must be known complete when a thread starts waiting.
@@ -377,10 +377,7 @@ tc_w4a16_kernel(const __grid_constant__ CUtensorMap xmap, const TcArgs a) {
     tmem_alloc(tmem_slot, C::kTmemCols);
     tmem_relinquish();
   }
-  // The activation producer is warp 3's first thread, or, when warp 3 issues
-  // MMAs (three MMA threads), a second thread of the weight producer's warp.
-  constexpr int kXWarp = NI == 3 ? 0 : 3, kXLane = NI == 3 ? 16 : 0;
-  if (warp == kXWarp && lane == kXLane) tma_prefetch_desc(&xmap);
+  if (warp == 3 && lane == 0) tma_prefetch_desc(&xmap);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -407,24 +404,25 @@ tc_w4a16_kernel(const __grid_constant__ CUtensorMap xmap, const TcArgs a) {
       // no copy into this CTA's shared memory may outlive it
       for (int r = max(0, issued - SWS); r < issued; ++r) wait_drain(&wfull[r % SWS], (r / SWS) & 1);
     }
-  }
-  if (warp == kXWarp && lane == kXLane) {
+  } else if (warp == 3) {
     // --------------------------------------------- activation producer
-    griddep_wait();  // the activations may come from the previous kernel
-    const int stages = (nk + XC - 1) / XC;
-    int issued = 0;
-    for (int t = 0; t < stages; ++t) {
-      const int s = t % SXS;
-      const int nc = min(XC, nk - t * XC);
-      if (t >= SXS && !mbar_wait(&xempty[s], ((t / SXS) - 1) & 1, abort_flag, err, 1)) break;
-      mbar_arrive_expect_tx(&xfull[s], nc * a.x_box_rows * 128);
-      for (int c = 0; c < nc; ++c)
-        tma_load_2d(xs + s * C::kXStageBytes + c * BN * 128, &xmap, (kc0 + t * XC + c) * kChunkK,
-                    xtile * BN, &xfull[s]);
-      ++issued;
+    if (lane == 0) {
+      griddep_wait();  // the activations may come from the previous kernel
+      const int stages = (nk + XC - 1) / XC;
+      int issued = 0;
+      for (int t = 0; t < stages; ++t) {
+        const int s = t % SXS;
+        const int nc = min(XC, nk - t * XC);
+        if (t >= SXS && !mbar_wait(&xempty[s], ((t / SXS) - 1) & 1, abort_flag, err, 1)) break;
+        mbar_arrive_expect_tx(&xfull[s], nc * a.x_box_rows * 128);
+        for (int c = 0; c < nc; ++c)
+          tma_load_2d(xs + s * C::kXStageBytes + c * BN * 128, &xmap, (kc0 + t * XC + c) * kChunkK,
+                      xtile * BN, &xfull[s]);
+        ++issued;
+      }
+      for (int t = max(0, issued - SXS); t < issued; ++t) wait_drain(&xfull[t % SXS], (t / SXS) & 1);
     }
-    for (int t = max(0, issued - SXS); t < issued; ++t) wait_drain(&xfull[t % SXS], (t / SXS) & 1);
-  } else if (warp >= 1 && warp <= NI) {
+  } else if (warp == 1 || (NI == 2 && warp == 2)) {
     // -------------------------------------------------- MMA issuer(s)
     if (lane == 0) {
       const int j = warp - 1;  // units u = j, j + NI, ...
@@ -802,7 +800,7 @@ cudaError_t launch_bn(int bn, const CUtensorMap& map, const TcArgs& a, dim3 grid
     // (rounds), TMEM A slots (units), dequant warpgroups, chunks per unit, MMA
     // threads, activation wait by the dequant warps.  TMEM: max(32, NI*BN) +
     // 32*UA*SA columns (<= 256 for two CTAs per SM).
-    case 16: return launch_cfg<16, 2, 6, 8, 6, 2, 1, 3, false, EPI>(map, a, grid, s);
+    case 16: return launch_cfg<16, 2, 8, 8, 6, 2, 1, 2, false, EPI>(map, a, grid, s);
     case 32: return launch_cfg<32, 2, 4, 8, 6, 2, 1, 2, false, EPI>(map, a, grid, s);
     case 64: return launch_cfg<64, 2, 2, 8, 4, 2, 1, 2, false, EPI>(map, a, grid, s);
     case 128: return launch_cfg<128, 4, 2, 3, 4, 2, 2, 1, true, EPI>(map, a, grid, s);
