@@ -71,3 +71,19 @@ def test_traffic_reported_only_for_the_captured_sources():
     files[bench.KERNEL_SOURCES[0]] = "changed kernel body"
     assert bench.kernel_sources_sha1(lambda rel: files[rel]) != sha
     assert bench.measured_traffic("no_such_kernel", "prefill") is None
+
+
+def test_roofline_bound_uses_each_formats_own_peak(cpu_torch):
+    peaks = {"hbm_gbs": 6557.8, "bf16_tflops": 1671.7, "bf16_tflops_sustained": 1402.4}
+    assert bench.tensor_peak(peaks, "bf16")[0] == 1671.7
+    assert bench.tensor_peak(peaks, "nvfp4_fixed")[0] == 1671.7 * 4
+    dec = bench.Workload(fake_native([]), "decode", 1)
+    bound, units = dec.kernel_units("tc_w4a16_gate_up_silu", peaks)
+    assert bound == "hbm" and units == bench.nvfp4_bytes(2 * 17408, 5120) + 5120 * 2 + 17408 * 2
+    w4 = bench.Workload(fake_native([]), "w4a4", 512)
+    bound, units = w4.kernel_units("tc_w4a4_gate_up_silu", peaks)
+    assert bound == "tensor" and units == 2.0 * 512 * 2 * 12288 * 4096
+    # the same intensity against the bf16 ridge (~255 flop/B) would also be
+    # tensor-bound; against the FP4 ridge (~1020 flop/B) a quarter of it is not
+    ridge = bench.tensor_peak(peaks, "nvfp4_fixed")[0] * 1e12 / (peaks["hbm_gbs"] * 1e9)
+    assert 1000 < ridge < 1040
