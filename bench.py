@@ -255,6 +255,29 @@ class Workload:
         return ("tensor", flops) if flops / byts > ridge else ("hbm", byts)
 
 
+def roofline(wl, prof, peaks, peak_src, workload):
+    """The `roofline` object for the dominant kernel of a profile
+    {kernel name: (launches, total ms)}: algorithmic units per launch over the
+    average launch duration, against the peak of the bound it is under."""
+    if not prof:
+        return None
+    kname, (launches, kms) = max(prof.items(), key=lambda kv: kv[1][1])
+    bound, units = wl.kernel_units(kname, peaks)
+    avg_s = kms / launches * 1e-3
+    if bound == "tensor":
+        peak, what = tensor_peak(peaks, wl.fmt)
+        achieved = units / avg_s / 1e12
+        unit = "TFLOP/s"
+    else:
+        peak, what = peaks["hbm_gbs"], "HBM copy"
+        achieved = units / avg_s / 1e9
+        unit = "GB/s"
+    return {"kernel": kname, "bound": bound, "achieved": round(achieved, 2), "peak": peak,
+            "peak_source": f"{peak_src} ({what})", "unit": unit, "frac": round(achieved / peak, 4),
+            "traffic": measured_traffic(kname, workload),
+            "avg_launch_us": round(avg_s * 1e6, 2), "launches": launches}
+
+
 def run_ours(args, rank, world, dist):
     import torch
     from nvfp4_quantized_dense_w4a16_b200 import build as B
@@ -284,24 +307,7 @@ def run_ours(args, rank, world, dist):
     flops = ffn_flops(wl.m, wl.H, wl.I)
     value = aggregate_throughput(flops, args.steps, ms, world) / 1e12
 
-    # dominant kernel and its roofline
-    roof = None
-    if prof:
-        kname, (launches, kms) = max(prof.items(), key=lambda kv: kv[1][1])
-        bound, units = wl.kernel_units(kname, peaks)
-        avg_s = kms / launches * 1e-3
-        if bound == "tensor":
-            peak, what = tensor_peak(peaks, wl.fmt)
-            achieved = units / avg_s / 1e12
-            unit = "TFLOP/s"
-        else:
-            peak, what = peaks["hbm_gbs"], "HBM copy"
-            achieved = units / avg_s / 1e9
-            unit = "GB/s"
-        roof = {"kernel": kname, "bound": bound, "achieved": round(achieved, 2), "peak": peak,
-                "peak_source": f"{peak_src} ({what})", "unit": unit, "frac": round(achieved / peak, 4),
-                "traffic": measured_traffic(kname, args.workload),
-                "avg_launch_us": round(avg_s * 1e6, 2), "launches": launches}
+    roof = roofline(wl, prof, peaks, peak_src, args.workload)
     kernels = {k: {"launches": l, "total_ms": round(t, 4), "share": round(t / max(1e-9, sum(v[1] for v in prof.values())), 4)}
                for k, (l, t) in prof.items()}
     gpu_launches = sum(v[0] for v in prof.values())

@@ -87,3 +87,20 @@ def test_roofline_bound_uses_each_formats_own_peak(cpu_torch):
     # tensor-bound; against the FP4 ridge (~1020 flop/B) a quarter of it is not
     ridge = bench.tensor_peak(peaks, "nvfp4_fixed")[0] * 1e12 / (peaks["hbm_gbs"] * 1e9)
     assert 1000 < ridge < 1040
+
+
+def test_roofline_object_of_the_dominant_kernel(cpu_torch):
+    peaks = {"hbm_gbs": 6557.8, "bf16_tflops": 1671.7, "bf16_tflops_sustained": 1402.4}
+    dec = bench.Workload(fake_native([]), "decode", 1)
+    prof = {"tc_w4a16_gate_up_silu": (20, 20 * 0.0430), "tc_w4a16_partial": (20, 20 * 0.0244),
+            "splitk_reduce": (20, 20 * 0.0075)}
+    r = bench.roofline(dec, prof, peaks, "measured", "decode")
+    assert r["kernel"] == "tc_w4a16_gate_up_silu" and r["bound"] == "hbm" and r["unit"] == "GB/s"
+    assert r["avg_launch_us"] == 43.0 and r["launches"] == 20
+    want = dec.kernel_units("tc_w4a16_gate_up_silu", peaks)[1] / 43.0e-6 / 1e9
+    assert abs(r["achieved"] - want) < 0.01 and abs(r["frac"] - want / 6557.8) < 1e-4
+    assert r["traffic"] is None  # no capture for this (kernel, workload)
+    assert bench.roofline(dec, {}, peaks, "measured", "decode") is None
+    w4 = bench.Workload(fake_native([]), "w4a4", 512)
+    r = bench.roofline(w4, {"tc_w4a4_gate_up_silu": (10, 10 * 0.147)}, peaks, "measured", "w4a4")
+    assert r["bound"] == "tensor" and r["peak"] == 1671.7 * 4 and "fp4" in r["peak_source"]
