@@ -10,17 +10,30 @@ import torch
 import bench
 
 
-@pytest.fixture
-def cpu_torch(monkeypatch):
+@pytest.fixture(scope="module")
+def cpu_torch():
     # run Workload on the CPU: no device transfers, no synchronisation
-    monkeypatch.setattr(torch.Tensor, "cuda", lambda self, *a, **k: self)
-    monkeypatch.setattr(torch.cuda, "synchronize", lambda *a, **k: None)
+    mp = pytest.MonkeyPatch()
+    mp.setattr(torch.Tensor, "cuda", lambda self, *a, **k: self)
+    mp.setattr(torch.cuda, "synchronize", lambda *a, **k: None)
     real_empty = torch.empty
 
     def empty(*a, **k):
         k.pop("device", None)
         return real_empty(*a, **k)
-    monkeypatch.setattr(torch, "empty", empty)
+    mp.setattr(torch, "empty", empty)
+    yield
+    mp.undo()
+
+
+@pytest.fixture(scope="module")
+def layers(cpu_torch):
+    """(Workload, list of forward calls it made) per layer, built once."""
+    out = {}
+    for name, m in (("decode", 1), ("w4a4", 512)):
+        calls = []
+        out[name] = (bench.Workload(fake_native(calls), name, m), calls)
+    return out
 
 
 def fake_native(calls):
@@ -33,10 +46,10 @@ def fake_native(calls):
         ffn_nvfp4_forward=lambda x, gu, d, f, out=None, workspace=None: calls.append((gu, d)))
 
 
-@pytest.mark.parametrize("name,m", [("decode", 1), ("w4a4", 512)])
-def test_small_layers_rotate_weight_copies(cpu_torch, name, m):
-    calls = []
-    wl = bench.Workload(fake_native(calls), name, m)
+@pytest.mark.parametrize("name", ["decode", "w4a4"])
+def test_small_layers_rotate_weight_copies(layers, name):
+    wl, calls = layers[name]
+    calls.clear()
     assert wl.sets >= 2
     assert wl.sets * wl.weight_bytes >= 4 * bench.L2_BYTES
     assert (wl.sets - 1) * wl.weight_bytes < 4 * bench.L2_BYTES  # no more copies than needed
@@ -49,8 +62,8 @@ def test_small_layers_rotate_weight_copies(cpu_torch, name, m):
     assert len({id(h) for h in used[:wl.sets]}) == wl.sets
 
 
-def test_weight_bytes_are_the_nvfp4_footprint(cpu_torch):
-    wl = bench.Workload(fake_native([]), "decode", 1)
+def test_weight_bytes_are_the_nvfp4_footprint(layers):
+    wl = layers["decode"][0]
     H, I = 5120, 17408
     assert wl.weight_bytes == 3 * H * I * (0.5 + 1 / 16)
 
@@ -73,14 +86,14 @@ def test_traffic_reported_only_for_the_captured_sources():
     assert bench.measured_traffic("no_such_kernel", "prefill") is None
 
 
-def test_roofline_bound_uses_each_formats_own_peak(cpu_torch):
+def test_roofline_bound_uses_each_formats_own_peak(layers):
     peaks = {"hbm_gbs": 6557.8, "bf16_tflops": 1671.7, "bf16_tflops_sustained": 1402.4}
     assert bench.tensor_peak(peaks, "bf16")[0] == 1671.7
     assert bench.tensor_peak(peaks, "nvfp4_fixed")[0] == 1671.7 * 4
-    dec = bench.Workload(fake_native([]), "decode", 1)
+    dec = layers["decode"][0]
     bound, units = dec.kernel_units("tc_w4a16_gate_up_silu", peaks)
     assert bound == "hbm" and units == bench.nvfp4_bytes(2 * 17408, 5120) + 5120 * 2 + 17408 * 2
-    w4 = bench.Workload(fake_native([]), "w4a4", 512)
+    w4 = layers["w4a4"][0]
     bound, units = w4.kernel_units("tc_w4a4_gate_up_silu", peaks)
     assert bound == "tensor" and units == 2.0 * 512 * 2 * 12288 * 4096
     # the same intensity against the bf16 ridge (~255 flop/B) would also be
@@ -89,9 +102,9 @@ def test_roofline_bound_uses_each_formats_own_peak(cpu_torch):
     assert 1000 < ridge < 1040
 
 
-def test_roofline_object_of_the_dominant_kernel(cpu_torch):
+def test_roofline_object_of_the_dominant_kernel(layers):
     peaks = {"hbm_gbs": 6557.8, "bf16_tflops": 1671.7, "bf16_tflops_sustained": 1402.4}
-    dec = bench.Workload(fake_native([]), "decode", 1)
+    dec = layers["decode"][0]
     prof = {"tc_w4a16_gate_up_silu": (20, 20 * 0.0430), "tc_w4a16_partial": (20, 20 * 0.0244),
             "splitk_reduce": (20, 20 * 0.0075)}
     r = bench.roofline(dec, prof, peaks, "measured", "decode")
@@ -101,6 +114,6 @@ def test_roofline_object_of_the_dominant_kernel(cpu_torch):
     assert abs(r["achieved"] - want) < 0.01 and abs(r["frac"] - want / 6557.8) < 1e-4
     assert r["traffic"] is None  # no capture for this (kernel, workload)
     assert bench.roofline(dec, {}, peaks, "measured", "decode") is None
-    w4 = bench.Workload(fake_native([]), "w4a4", 512)
+    w4 = layers["w4a4"][0]
     r = bench.roofline(w4, {"tc_w4a4_gate_up_silu": (10, 10 * 0.147)}, peaks, "measured", "w4a4")
     assert r["bound"] == "tensor" and r["peak"] == 1671.7 * 4 and "fp4" in r["peak_source"]
