@@ -100,8 +100,7 @@ def nvfp4_bytes(n, k):
 KERNEL_SOURCES = ("csrc/tc_gemm.cu", "csrc/sm100.cuh", "csrc/common.cuh", "csrc/internal.h")
 TRAFFIC = {
     ("tc_w4a16_gate_up_silu", "prefill"): {
-        "bytes": 146800896 + 128328960, "sources_sha1": "5976b4c07ea6be5b9cb88fe0ad51fe53f300e557",
-        "profile": "profiles/tc_w4a16_gate_up_prefill_m4096.md"},
+        "bytes": 146800896 + 128328960, "sources_sha1": "5976b4c07ea6be5b9cb88fe0ad51fe53f300e557"},
 }
 
 

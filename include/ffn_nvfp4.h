@@ -185,18 +185,51 @@ ffn_status ffn_nvfp4_linear(const void* x, int64_t m, const ffn_nvfp4_weight* w,
  * running (cudaMalloc can synchronise the whole device).  The source pages
  * have no counterpart; this entry point exists only for such callers.
  *   x [m, k] bf16, w a plain (not gate+up) handle of shape [n, k],
- *   y [m, n] bf16 = bf16(gs * x @ w^T), the same kernels as ffn_nvfp4_linear.
+ *   y [m, n] bf16 = bf16(gs * x @ w^T).  It always runs the tensor-core
+ *   projection kernels (whatever kernel ffn_nvfp4_linear would pick for m).
  * The split-K partial sums live in one fixed 16 MiB device array that every
- * GPU loading the library holds until the process exits; a shape whose
- * partials would need more returns FFN_ERR_WORKSPACE (nothing launched).  It
- * calls no cudaMalloc, cudaFree or allocating library routine.  The first
- * call on each device looks up that device's address of the array (with the
- * device current), so make that first call before any stream capture.  All
- * calls share the array: calls that overlap on the GPU (other streams, other
- * threads) race and must be serialised by the caller.  Every partial a call
- * reads is written earlier in the same call, so nothing needs clearing. */
+ * GPU context loading the library holds until the process exits; a shape
+ * whose partials would need more returns FFN_ERR_WORKSPACE (nothing
+ * launched).  It calls no cudaMalloc, cudaFree or allocating library routine.
+ * Set-up: the first call in each CUDA context looks up that context's address
+ * of the array (with the context current).  Under lazy module loading (the
+ * CUDA default) that first lookup also loads the module and so reserves the
+ * 16 MiB: it can fail with FFN_ERR_OOM and may synchronise.  Make the first
+ * call at set-up time, before any stream capture.  A device reset creates a
+ * new context, whose first call repeats the look-up.  All calls share the
+ * array: calls that overlap on the GPU (other streams, other threads) race
+ * and must be serialised by the caller.  Every partial a call reads is written
+ * earlier in the same call, so nothing needs clearing. */
 ffn_status ffn_nvfp4_linear_noalloc(const void* x, int64_t m, const ffn_nvfp4_weight* w,
                                     void* y, void* stream);
+
+/* Kernel configuration a projection of m rows would use (the m-dispatch),
+ * without launching anything; callable without a GPU (the SM count of the
+ * current device is used when there is one, else 148).  Lets callers and
+ * tests see which kernel family, activation tile width and split-K count
+ * ffn_nvfp4_linear (gate_up = 0, shape [n, k]) or the gate+up projection of
+ * ffn_nvfp4_forward (gate_up = 1, n = 2 * inter, k = hidden) selects.
+ * The m-tiered kernel choice follows "metrale_model_layers/layers/
+ * dense_ffn_prefill.rs", DenseFfnLayer::w4a16_prefill_gemm (a projection
+ * kernel chosen by m and the weight's shape); the tiers are this library's. */
+typedef enum ffn_kernel_family {
+  FFN_KERNEL_NONE = 0,       /* m == 0: nothing is launched                     */
+  FFN_KERNEL_TC_W4A16 = 1,   /* tcgen05 kind::f16 MMA over dequantised weights  */
+  FFN_KERNEL_TC_W4A4 = 2,    /* tcgen05 block-scaled FP4 MMA (kind::mxf4nvf4)   */
+  FFN_KERNEL_GEMV_W4A16 = 3, /* CUDA-core projection, bf16 activations          */
+  FFN_KERNEL_GEMV_W4A4 = 4   /* CUDA-core projection, fixed activation format   */
+} ffn_kernel_family;
+
+typedef struct ffn_projection_plan {
+  int family;    /* ffn_kernel_family                                          */
+  int tile_rows; /* activation rows per tile (the MMA's N); 0 for CUDA cores   */
+  int k_splits;  /* K ranges whose fp32 partial sums are added afterwards in a
+                    fixed order (1 = no split)                                 */
+  int grid;      /* CTAs of the projection kernel                              */
+} ffn_projection_plan;
+
+ffn_status ffn_nvfp4_projection_plan(int64_t m, int64_t n, int64_t k, ffn_act_format format,
+                                     int gate_up, ffn_projection_plan* out);
 
 /* Device-side error bits.  Kernels that wait on asynchronous copies or on
  * tensor-core completion give up after about two seconds instead of hanging,

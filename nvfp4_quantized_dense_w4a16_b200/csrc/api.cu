@@ -34,6 +34,17 @@ inline ffn_status cuda_status(cudaError_t e) { return e == cudaSuccess ? FFN_OK 
 
 inline size_t round_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
+// A handle's buffers live on the device it was created on; using it with
+// another device current would hand that device foreign pointers.
+ffn_status check_device(const ffn_nvfp4_weight* w) {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess) {
+    cudaGetLastError();
+    return FFN_ERR_CUDA;
+  }
+  return dev == w->device ? FFN_OK : FFN_ERR_INVALID_ARG;
+}
+
 // Pick up errors of earlier asynchronous work before enqueuing more.
 inline ffn_status precheck() {
   const cudaError_t e = cudaPeekAtLastError();
@@ -186,6 +197,8 @@ void ffn::handle_tc_view(const ffn_nvfp4_weight* w, ffn::TcWeight* out, bool* ga
   *gate_up = w->gate_up != 0;
 }
 
+ffn_status ffn::handle_check_device(const ffn_nvfp4_weight* w) { return check_device(w); }
+
 extern "C" {
 
 const char* ffn_status_string(ffn_status s) {
@@ -282,6 +295,8 @@ ffn_status ffn_nvfp4_weight_create_gate_up(const ffn_nvfp4_weight* gate,
   if (!gate || !up) return FFN_ERR_INVALID_ARG;
   if (gate->gate_up || up->gate_up) return FFN_ERR_INVALID_ARG;
   if (gate->n != up->n || gate->k != up->k) return FFN_ERR_SHAPE;
+  if (gate->device != up->device) return FFN_ERR_INVALID_ARG;
+  if (ffn_status st = check_device(gate)) return st;
   if (ffn_status st = precheck()) return st;
   const int64_t I = gate->n, H = gate->k;
   auto* w = new (std::nothrow) ffn_nvfp4_weight;
@@ -360,6 +375,8 @@ ffn_status ffn_nvfp4_forward(const void* x, int64_t m, int64_t hidden, int64_t i
     return FFN_ERR_SHAPE;
   if (m == 0) return FFN_OK;
   if (!x || !out) return FFN_ERR_INVALID_ARG;
+  if (ffn_status st = check_device(gate_up)) return st;
+  if (ffn_status st = check_device(down)) return st;
   const Carve c = carve_ffn(m, hidden, inter, format);
   if (!workspace || workspace_bytes < c.total) return FFN_ERR_WORKSPACE;
   if (!aligned16(x) || !aligned16(out) || !aligned16(workspace)) return FFN_ERR_ALIGNMENT;
@@ -394,6 +411,28 @@ ffn_status ffn_nvfp4_forward(const void* x, int64_t m, int64_t hidden, int64_t i
   return cuda_status(e);
 }
 
+ffn_status ffn_nvfp4_projection_plan(int64_t m, int64_t n, int64_t k, ffn_act_format format,
+                                     int gate_up, ffn_projection_plan* out) {
+  if (!out || m < 0 || n <= 0) return FFN_ERR_INVALID_ARG;
+  if (format != FFN_ACT_BF16 && format != FFN_ACT_NVFP4_FIXED) return FFN_ERR_INVALID_ARG;
+  if (!valid_k(k) || (gate_up && n % 2)) return FFN_ERR_SHAPE;
+  *out = ffn_projection_plan{FFN_KERNEL_NONE, 0, 1, 0};
+  if (m == 0) return FFN_OK;
+  const int ncols = (int)(gate_up ? n / 2 : n);
+  if (format == FFN_ACT_BF16 && w4a16_path(m) == Path::kTc) {
+    const ffn::TcPlan p = ffn::plan_tc(m, n, k, gate_up != 0, num_sms());
+    *out = ffn_projection_plan{FFN_KERNEL_TC_W4A16, p.bn, p.splits, p.xtiles * p.wtiles * p.splits};
+  } else if (format == FFN_ACT_BF16) {
+    *out = ffn_projection_plan{FFN_KERNEL_GEMV_W4A16, 0, 1, ffn::gemv_grid(ncols)};
+  } else if (w4a4_path() == Path::kTc) {
+    const ffn::TcPlan p = ffn::plan_w4a4(m, n, k, gate_up != 0, num_sms());
+    *out = ffn_projection_plan{FFN_KERNEL_TC_W4A4, p.bn, p.splits, p.xtiles * p.wtiles * p.splits};
+  } else {
+    *out = ffn_projection_plan{FFN_KERNEL_GEMV_W4A4, 0, 1, ffn::gemv_grid(ncols)};
+  }
+  return FFN_OK;
+}
+
 ffn_status ffn_nvfp4_device_error(int* flags, int clear) {
   if (!flags) return FFN_ERR_INVALID_ARG;
   if (cudaDeviceSynchronize() != cudaSuccess) {
@@ -420,6 +459,7 @@ ffn_status ffn_nvfp4_linear(const void* x, int64_t m, const ffn_nvfp4_weight* w,
   if (w->gate_up) return FFN_ERR_UNSUPPORTED;
   if (m == 0) return FFN_OK;
   if (!x || !y) return FFN_ERR_INVALID_ARG;
+  if (ffn_status st = check_device(w)) return st;
   const Carve c = carve_linear(m, w->n, w->k, format);
   if (c.total && (!workspace || workspace_bytes < c.total)) return FFN_ERR_WORKSPACE;
   if (!aligned16(x) || !aligned16(y) || (c.total && !aligned16(workspace)))

@@ -248,6 +248,8 @@ cudaError_t gemv16(const void* x, int64_t m, const WeightView& w, Epilogue ep, v
 
 }  // namespace
 
+int gemv_grid(int64_t ncols) { return (int)((ncols + kWarps - 1) / kWarps); }
+
 cudaError_t launch_gemv_w4a16(const void* x, int64_t m, const WeightView& w, Epilogue ep,
                               void* y, cudaStream_t s) {
   if (m <= 1) return gemv16<1>(x, m, w, ep, y, s);

@@ -57,6 +57,8 @@ cudaError_t launch_quantize_activations_blocked(const void* x, int64_t m, int64_
 
 // Tensor-core view of a handle (and whether it is a fused gate+up handle).
 void handle_tc_view(const ffn_nvfp4_weight* w, TcWeight* out, bool* gate_up);
+// FFN_OK when the handle belongs to the current device.
+ffn_status handle_check_device(const ffn_nvfp4_weight* w);
 
 // Device-wide error bits set by kernels whose bounded waits gave up.
 cudaError_t read_device_error(int* flags, bool clear);
@@ -67,6 +69,7 @@ cudaError_t launch_quantize_activations(const void* x, int64_t m, int64_t k, voi
                                         void* scales, cudaStream_t s);
 
 // CUDA-core projections (any m; used for small m and as the general path).
+int gemv_grid(int64_t ncols);
 cudaError_t launch_gemv_w4a16(const void* x, int64_t m, const WeightView& w, Epilogue ep,
                               void* y, cudaStream_t s);
 cudaError_t launch_gemv_w4a4(const uint8_t* xcodes, const uint8_t* xscales, int64_t m,

@@ -784,12 +784,10 @@ template <int BN, int SXS, int XC, int SWS, int SA, int DQG, int UA, int NI, boo
 cudaError_t launch_cfg(const CUtensorMap& map, const TcArgs& a, dim3 grid, cudaStream_t s) {
   using C = TcCfg<BN, SXS, XC, SWS, SA, DQG, UA, NI, DQX>;
   auto kern = tc_w4a16_kernel<BN, SXS, XC, SWS, SA, DQG, UA, NI, DQX, EPI>;
-  static bool attr_set = false;  // per instantiation; idempotent if raced
-  if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemAlloc);
-    if (e != cudaSuccess) return e;
-    attr_set = true;
-  }
+  // The attribute belongs to the current device's context, so it is set on
+  // every launch (a host-side call): correct on any device and after a reset.
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemAlloc);
+  if (e != cudaSuccess) return e;
   return launch_pdl(kern, grid, dim3(C::kThreads), C::kSmemAlloc, s, map, a);
 }
 
@@ -943,13 +941,10 @@ cudaError_t launch_tc_w4a4(const uint8_t* xcodes, const uint8_t* xsf_blocks, int
   a.t.n_pad = p.n_pad;
   a.sfb = xsf_blocks;
   const dim3 grid(p.xtiles, p.wtiles, p.splits);
-  static bool attr_set[3] = {false, false, false};
-  auto launch = [&](auto kern, int epi) -> cudaError_t {
-    if (!attr_set[epi]) {
-      cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, W4Cfg::kSmemAlloc);
-      if (e != cudaSuccess) return e;
-      attr_set[epi] = true;
-    }
+  auto launch = [&](auto kern, int) -> cudaError_t {
+    // set on every launch: the attribute belongs to the current device's context
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, W4Cfg::kSmemAlloc);
+    if (e != cudaSuccess) return e;
     kern<<<grid, 256, W4Cfg::kSmemAlloc, s>>>(map, a);
     return cudaGetLastError();
   };

@@ -31,6 +31,14 @@ class FfnError(RuntimeError):
         self.status_name = name
 
 
+class ProjectionPlan(ctypes.Structure):
+    _fields_ = [("family", ctypes.c_int), ("tile_rows", ctypes.c_int), ("k_splits", ctypes.c_int),
+                ("grid", ctypes.c_int)]
+
+
+KERNEL_FAMILIES = {0: "none", 1: "tc_w4a16", 2: "tc_w4a4", 3: "gemv_w4a16", 4: "gemv_w4a4"}
+
+
 class KernelTime(ctypes.Structure):
     _fields_ = [("name", ctypes.c_char_p), ("launches", ctypes.c_int), ("total_ms", ctypes.c_double)]
 
@@ -57,6 +65,8 @@ def _load() -> ctypes.CDLL:
         "ffn_nvfp4_linear_workspace_size": (ctypes.c_int, [i64, i64, i64, ctypes.c_int, P(sz)]),
         "ffn_nvfp4_linear": (ctypes.c_int, [vp, i64, vp, ctypes.c_int, vp, vp, sz, vp]),
         "ffn_nvfp4_linear_noalloc": (ctypes.c_int, [vp, i64, vp, vp, vp]),
+        "ffn_nvfp4_projection_plan": (ctypes.c_int, [i64, i64, i64, ctypes.c_int, ctypes.c_int,
+                                                     P(ProjectionPlan)]),
         "ffn_nvfp4_profile_begin": (ctypes.c_int, []),
         "ffn_nvfp4_device_error": (ctypes.c_int, [P(ctypes.c_int), ctypes.c_int]),
         "ffn_nvfp4_profile_end": (ctypes.c_int, [P(KernelTime), ctypes.c_int, P(ctypes.c_int)]),
@@ -282,3 +292,12 @@ def ffn_nvfp4_linear_noalloc(x: torch.Tensor, w: Weight, y=None, stream=None) ->
     _check("ffn_nvfp4_linear_noalloc", lib.ffn_nvfp4_linear_noalloc(
         _ptr(x), m, w.handle, _ptr(y), _stream(stream)))
     return y
+
+
+def ffn_nvfp4_projection_plan(m: int, n: int, k: int, fmt="bf16", gate_up: bool = False) -> dict:
+    """The kernel configuration a projection of m rows selects (nothing launched)."""
+    p = ProjectionPlan()
+    _check("ffn_nvfp4_projection_plan", lib.ffn_nvfp4_projection_plan(m, n, k, _fmt(fmt), int(gate_up),
+                                                                      ctypes.byref(p)))
+    return {"family": KERNEL_FAMILIES.get(p.family, str(p.family)), "tile_rows": p.tile_rows,
+            "k_splits": p.k_splits, "grid": p.grid}

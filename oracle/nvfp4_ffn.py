@@ -27,7 +27,7 @@ What is computed, and where it comes from
   consecutive elements along K (OCP 8-bit Floating Point v1.0, E4M3: bias 7,
   no infinities, max 448), and one FP32 scale per tensor.
 
-Readings taken where the pages are silent (each is listed in the design doc):
+Readings taken where the pages are silent:
   R1 E2M1 encoding rounds to nearest, ties to the even magnitude index,
      saturating at 6; the sign bit is kept (so -0.1 encodes as 0x8).  Packing:
      element 2j in the low nibble of byte j.

@@ -34,3 +34,12 @@ def read_golden(name):
 @pytest.fixture
 def golden():
     return read_golden
+
+
+def pytest_sessionstart(session):
+    # A planted oracle mistake for the mutation check (tests/oracle_mutations.py);
+    # unset in every ordinary run.
+    name = os.environ.get("FFN_ORACLE_MUTATION")
+    if name:
+        import oracle_mutations
+        oracle_mutations.apply(name)

@@ -73,3 +73,25 @@ def test_host_side_argument_errors(native):
     assert L.ffn_nvfp4_linear(fake, 1, None, 0, fake, fake, 0, None) == 1
     assert L.ffn_nvfp4_weight_destroy(None) == 0
     assert L.ffn_nvfp4_weight_dims(None, None, None, None) == 1
+
+
+def test_projection_plan_m_dispatch(native):
+    # W4A16: the tile width follows m in tiers, split-K fills the GPU for
+    # few output tiles; nothing is launched and no GPU is needed.
+    for m, bn in ((1, 16), (16, 16), (17, 32), (32, 32), (33, 64), (64, 64), (65, 128),
+                  (128, 128), (129, 256), (4096, 256)):
+        p = native.ffn_nvfp4_projection_plan(m, 384, 512, "bf16")
+        assert p["family"] == "tc_w4a16" and p["tile_rows"] == bn, (m, p)
+    assert native.ffn_nvfp4_projection_plan(4, 384, 512)["k_splits"] == 1
+    assert native.ffn_nvfp4_projection_plan(4, 128, 4096)["k_splits"] == 8
+    assert native.ffn_nvfp4_projection_plan(0, 128, 4096)["family"] == "none"
+    # fixed format: the K split does not depend on m (row invariance)
+    splits = {native.ffn_nvfp4_projection_plan(m, 4096, 12288, "nvfp4_fixed")["k_splits"]
+              for m in (1, 7, 64, 512)}
+    assert len(splits) == 1
+    L = native.lib
+    p = native.ProjectionPlan()
+    assert L.ffn_nvfp4_projection_plan(4, 128, 48, 0, 0, ctypes.byref(p)) == 2    # k % 32
+    assert L.ffn_nvfp4_projection_plan(4, 129, 64, 0, 1, ctypes.byref(p)) == 2    # odd gate+up n
+    assert L.ffn_nvfp4_projection_plan(-1, 128, 64, 0, 0, ctypes.byref(p)) == 1
+    assert L.ffn_nvfp4_projection_plan(4, 128, 64, 0, 0, None) == 1

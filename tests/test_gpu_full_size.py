@@ -65,11 +65,11 @@ def test_w4a4_full_matches_oracle(native, w4a4, m):
 
 def test_prefill_m4096_full_sampled_rows(native):
     # the bench's primary workload in its launch configuration (m = 4096, 16
-    # activation tiles of 256 rows); rows sampled from the first, middle and
-    # last tiles, including tile edges, are checked against the oracle.
+    # activation tiles of 256 rows): every row of the first 256-row tile, and
+    # rows of the middle and last tiles at tile edges, against the oracle.
     case = FfnCase(native, synth.make_inputs("prefill"))
     out = bf16_to_f64(case.forward("bf16"))
-    rows = [0, 255, 256, 2048, 3839, 4095]
+    rows = list(range(256)) + [256, 2048, 3839, 4095]
     assert_close(out[rows], case.oracle("bf16", rows=rows), "prefill m=4096")
     assert np.all(np.isfinite(out))
     assert native.ffn_nvfp4_device_error(clear=False) == 0
