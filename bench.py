@@ -70,17 +70,33 @@ def load_peaks():
     return dict(FALLBACK_PEAKS), "fallback"
 
 
-# Nominal dense FP4 / bf16 tensor-core throughput ratio (9 vs 2.25 PFLOP/s):
-# the fixed format's block-scaled FP4 MMAs are measured against the measured
-# bf16 peak times this ratio.
+# Nominal dense FP4 / bf16 tensor-core throughput ratio (9 vs 2.25 PFLOP/s),
+# used only when the library's own block-scaled FP4 MMA probe could not run.
 FP4_OVER_BF16 = 4.0
 
 
 def tensor_peak(peaks, fmt):
-    """(TFLOP/s, description) of the tensor-core peak for a projection's dtype."""
+    """(TFLOP/s, description) of the tensor-core peak for a projection's dtype:
+    the measured bf16 matmul peak, and for the fixed format the measured
+    kind::mxf4nvf4 probe ('fp4_tflops', added at run time) when present."""
     if fmt == "nvfp4_fixed":
+        if peaks.get("fp4_tflops"):
+            return peaks["fp4_tflops"], "fp4 (tcgen05 kind::mxf4nvf4 probe, measured in this run)"
         return peaks["bf16_tflops"] * FP4_OVER_BF16, "bf16 x nominal fp4/bf16 ratio 4"
     return peaks["bf16_tflops"], "bf16"
+
+
+def measure_tensor_probes(native):
+    """Dense tensor-core TFLOP/s of this GPU for the MMA kinds the library
+    issues (its own probe kernels; best of one and two issuing threads)."""
+    out = {}
+    for kind in ("bf16", "nvfp4"):
+        try:
+            out[kind] = round(max(native.ffn_nvfp4_tensor_peak(kind, issuers, 20000) for issuers in (1, 2)), 1)
+        except Exception as e:  # reported, never fatal to the bench line
+            out[kind] = None
+            out[kind + "_error"] = str(e)
+    return out
 
 
 def ffn_flops(m, H, I):
@@ -286,6 +302,9 @@ def run_ours(args, rank, world, dist):
     peaks, peak_src = load_peaks()
     dev_index = int(os.environ.get("LOCAL_RANK", "0"))
     torch.cuda.set_device(dev_index)
+    probes = measure_tensor_probes(N)
+    if probes.get("nvfp4"):
+        peaks["fp4_tflops"] = probes["nvfp4"]
     wl = Workload(N, args.workload, args.m)
     flush = torch.empty(2 * L2_BYTES // 4, dtype=torch.float32, device="cuda") if wl.flush_l2 else None
 
@@ -340,9 +359,13 @@ def run_ours(args, rank, world, dist):
     if not args.no_extra and args.workload == "prefill":
         del wl, x_dev
         torch.cuda.empty_cache()
-        extra["decode_m1"] = secondary(N, "decode", 1, peaks, max(args.steps, 20), args.eager)
-        extra["w4a4_m512"] = secondary(N, "w4a4", 512, peaks, max(args.steps // 2, 5), args.eager)
+        extra["decode_m1"] = secondary(N, "decode", [1], peaks, max(args.steps, 20), args.eager)[1]
+        extra["smallm"] = secondary(N, "smallm", [8, 16, 32, 64], peaks, max(args.steps, 20), args.eager)
+        w4 = secondary(N, "w4a4", [1, 7, 64, 512], peaks, max(args.steps // 2, 10), args.eager)
+        extra["w4a4_m512"] = w4.pop(512)
+        extra["w4a4_small"] = w4
         torch.cuda.empty_cache()
+    extra["tensor_probes_tflops"] = probes
     return {
         "value": round(value, 3), "ms_per_step": round(ms_step, 4), "roofline": roof,
         "kernels": kernels, "gpu_launches": gpu_launches, "clocks": clk, "e2e": e2e,
@@ -414,21 +437,32 @@ def capture_steps(N, wl, steps, flush, profile=False):
     return graph, starts, stops
 
 
-def secondary(N, name, m, peaks, steps, eager=False):
-    """Time another layer shape: per-step µs, weight GB/s and TFLOP/s."""
+def secondary(N, name, ms, peaks, steps, eager=False):
+    """Time other layer shapes of one workload (its weights built once) at
+    each row count in `ms`: {m: per-step µs, weight GB/s, TFLOP/s, fraction
+    of the roofline, per-kernel µs}."""
     import torch
-    wl = Workload(N, name, m)
-    flush = None  # cold weights come from rotating weight copies (Workload)
-    for i in range(3):
-        wl.step(i)
-    torch.cuda.synchronize()
-    ms, prof = time_steps(N, wl, steps, flush, eager, torch.cuda.synchronize)
-    ms /= steps
-    res = {"m": m, "hidden": wl.H, "inter": wl.I, "format": wl.fmt, "us_per_layer": round(ms * 1e3, 2),
-           "weight_gbs": round(wl.weight_bytes / (ms * 1e-3) / 1e9, 1),
-           "tflops": round(ffn_flops(m, wl.H, wl.I) / (ms * 1e-3) / 1e12, 3),
-           "hbm_roofline_frac": round(wl.weight_bytes / (ms * 1e-3) / 1e9 / peaks["hbm_gbs"], 4),
-           "kernels": {k: {"launches": l, "avg_us": round(t / l * 1e3, 2)} for k, (l, t) in prof.items()}}
+    wl = Workload(N, name, max(ms))
+    x_all, out_all = wl.x, wl.out
+    res = {}
+    for m in ms:
+        wl.m, wl.x, wl.out = m, x_all[:m].contiguous(), out_all[:m]
+        wl.ws = torch.empty((max(16, N.ffn_nvfp4_workspace_size(m, wl.H, wl.I, wl.fmt)),), dtype=torch.uint8,
+                            device="cuda")
+        for i in range(3):
+            wl.step(i)
+        torch.cuda.synchronize()
+        ms_total, prof = time_steps(N, wl, steps, None, eager, torch.cuda.synchronize)
+        t = ms_total / steps * 1e-3
+        byts = wl.weight_bytes + m * (wl.H + wl.I) * 2 * 2
+        flops = ffn_flops(m, wl.H, wl.I)
+        roof = max(byts / (peaks["hbm_gbs"] * 1e9), flops / (tensor_peak(peaks, wl.fmt)[0] * 1e12))
+        res[m] = {"m": m, "hidden": wl.H, "inter": wl.I, "format": wl.fmt, "us_per_layer": round(t * 1e6, 2),
+                  "weight_gbs": round(wl.weight_bytes / t / 1e9, 1),
+                  "tflops": round(flops / t / 1e12, 3),
+                  "hbm_roofline_frac": round(wl.weight_bytes / t / 1e9 / peaks["hbm_gbs"], 4),
+                  "roofline_frac": round(roof / t, 4),
+                  "kernels": {k: {"launches": l, "avg_us": round(tt / l * 1e3, 2)} for k, (l, tt) in prof.items()}}
     del wl
     return res
 

@@ -207,8 +207,9 @@ ffn_status ffn_nvfp4_linear_noalloc(const void* x, int64_t m, const ffn_nvfp4_we
  * without launching anything; callable without a GPU (the SM count of the
  * current device is used when there is one, else 148).  Lets callers and
  * tests see which kernel family, activation tile width and split-K count
- * ffn_nvfp4_linear (gate_up = 0, shape [n, k]) or the gate+up projection of
- * ffn_nvfp4_forward (gate_up = 1, n = 2 * inter, k = hidden) selects.
+ * ffn_nvfp4_linear (role FFN_ROLE_LINEAR, shape [n, k]) or the projections of
+ * ffn_nvfp4_forward (FFN_ROLE_GATE_UP: n = 2 * inter, k = hidden;
+ * FFN_ROLE_DOWN: n = hidden, k = inter) select.
  * The m-tiered kernel choice follows "metrale_model_layers/layers/
  * dense_ffn_prefill.rs", DenseFfnLayer::w4a16_prefill_gemm (a projection
  * kernel chosen by m and the weight's shape); the tiers are this library's. */
@@ -217,19 +218,41 @@ typedef enum ffn_kernel_family {
   FFN_KERNEL_TC_W4A16 = 1,   /* tcgen05 kind::f16 MMA over dequantised weights  */
   FFN_KERNEL_TC_W4A4 = 2,    /* tcgen05 block-scaled FP4 MMA (kind::mxf4nvf4)   */
   FFN_KERNEL_GEMV_W4A16 = 3, /* CUDA-core projection, bf16 activations          */
-  FFN_KERNEL_GEMV_W4A4 = 4   /* CUDA-core projection, fixed activation format   */
+  FFN_KERNEL_GEMV_W4A4 = 4,  /* CUDA-core projection, fixed activation format   */
+  FFN_KERNEL_TC_W4A16_PERSISTENT = 5 /* few-row FFN layer: persistent tcgen05
+                                kernels, one CTA per SM, gate+up over whole tiles,
+                                down over equal K ranges reduced in-kernel       */
 } ffn_kernel_family;
+
+typedef enum ffn_projection_role {
+  FFN_ROLE_LINEAR = 0,   /* ffn_nvfp4_linear                                  */
+  FFN_ROLE_GATE_UP = 1,  /* the fused gate+up projection of ffn_nvfp4_forward  */
+  FFN_ROLE_DOWN = 2      /* the down projection of ffn_nvfp4_forward           */
+} ffn_projection_role;
 
 typedef struct ffn_projection_plan {
   int family;    /* ffn_kernel_family                                          */
   int tile_rows; /* activation rows per tile (the MMA's N); 0 for CUDA cores   */
   int k_splits;  /* K ranges whose fp32 partial sums are added afterwards in a
-                    fixed order (1 = no split)                                 */
+                    fixed order (1 = no split); for the persistent down
+                    projection, the most ranges any output tile is cut into  */
   int grid;      /* CTAs of the projection kernel                              */
 } ffn_projection_plan;
 
 ffn_status ffn_nvfp4_projection_plan(int64_t m, int64_t n, int64_t k, ffn_act_format format,
-                                     int gate_up, ffn_projection_plan* out);
+                                     int role, ffn_projection_plan* out);
+
+/* Measured dense tensor-core throughput of the current GPU, in TFLOP/s, for
+ * the MMA kinds the library issues: kind = 0, tcgen05 kind::f16 (bf16 x bf16,
+ * fp32 accumulate, M128 N256 K16, operands in shared memory); kind = 1,
+ * kind::mxf4nvf4 with UE4M3 scales per 16 elements (E2M1 x E2M1, M128 N128
+ * K64).  One CTA per SM, `issuers` (1 or 2) threads per CTA each issuing
+ * `iters` MMAs back to back into its own accumulator; timed with CUDA events
+ * on a private stream after a short warm-up launch.  A roofline denominator
+ * for the kernels (no library exposes the block-scaled FP4 MMA), not part of
+ * the FFN path.  Allocates 4 bytes of device memory for an error flag and
+ * synchronises.  Returns FFN_ERR_CUDA if a wait gave up. */
+ffn_status ffn_nvfp4_tensor_peak(int kind, int issuers, int iters, double* tflops);
 
 /* Device-side error bits.  Kernels that wait on asynchronous copies or on
  * tensor-core completion give up after about two seconds instead of hanging,

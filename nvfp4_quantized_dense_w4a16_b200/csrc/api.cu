@@ -71,7 +71,7 @@ int num_sms() {
 // GEMV.  FFN_NVFP4_W4A16_PATH=gemv|tc overrides (read once) for measurements.
 enum class Path { kTc, kGemv };
 
-Path w4a16_path(int64_t m) {
+int w4a16_forced() {
   static int forced = [] {
     const char* v = getenv("FFN_NVFP4_W4A16_PATH");
     if (!v) return 0;
@@ -79,11 +79,18 @@ Path w4a16_path(int64_t m) {
     if (!strcmp(v, "tc")) return 2;
     return 0;
   }();
-  if (forced == 1) return Path::kGemv;
-  if (forced == 2) return Path::kTc;
+  return forced;
+}
+
+Path w4a16_path(int64_t m) {
+  if (w4a16_forced() == 1) return Path::kGemv;
   (void)m;
   return Path::kTc;
 }
+
+// The FFN layer for few rows runs as two persistent launches (see
+// plan_persist) unless FFN_NVFP4_W4A16_PATH forces a projection family.
+bool w4a16_persistent(int64_t m) { return w4a16_forced() == 0 && m <= ffn::kPersistMaxRows; }
 
 // Fixed format: the block-scaled FP4 tensor-core kernel, or the CUDA-core one
 // (FFN_NVFP4_W4A4_PATH=gemv).  Either choice is made once per process and does
@@ -100,8 +107,9 @@ Path w4a4_path() {
 // 256-byte aligned): [h bf16 m*inter] [xq codes m*hidden/2] [xq scales
 // m*hidden/16] [hq codes m*inter/2] [hq scales m*inter/16].
 struct Carve {
-  size_t h = 0, xq_c = 0, xq_s = 0, hq_c = 0, hq_s = 0, part = 0, total = 0;
+  size_t h = 0, xq_c = 0, xq_s = 0, hq_c = 0, hq_s = 0, part = 0, cnt = 0, total = 0;
   ffn::TcPlan gate_up, down;
+  ffn::PersistPlan persist;
 };
 
 // Workspace of the fixed format on the tensor-core path: quantised x and h
@@ -131,7 +139,13 @@ Carve carve_ffn(int64_t m, int64_t hidden, int64_t inter, ffn_act_format f) {
   size_t off = 0;
   c.h = off;
   off += round_up((size_t)m * inter * 2, 256);
-  if (f == FFN_ACT_BF16 && m > 0 && w4a16_path(m) == Path::kTc) {
+  if (f == FFN_ACT_BF16 && m > 0 && w4a16_persistent(m)) {
+    c.persist = ffn::plan_persist(m, hidden, inter, num_sms());
+    c.part = off;
+    off += round_up(c.persist.partial_bytes, 256);
+    c.cnt = off;
+    off += round_up(c.persist.counter_bytes, 256);
+  } else if (f == FFN_ACT_BF16 && m > 0 && w4a16_path(m) == Path::kTc) {
     const int sms = num_sms();
     c.gate_up = ffn::plan_tc(m, 2 * inter, hidden, true, sms);
     c.down = ffn::plan_tc(m, hidden, inter, false, sms);
@@ -385,7 +399,10 @@ ffn_status ffn_nvfp4_forward(const void* x, int64_t m, int64_t hidden, int64_t i
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   void* h = ws + c.h;
   cudaError_t e;
-  if (format == FFN_ACT_BF16 && w4a16_path(m) == Path::kTc) {
+  if (format == FFN_ACT_BF16 && w4a16_persistent(m)) {
+    e = ffn::launch_persist_ffn(x, m, gate_up->tc(), down->tc(), c.persist, h, ws + c.part,
+                                reinterpret_cast<int*>(ws + c.cnt), out, s);
+  } else if (format == FFN_ACT_BF16 && w4a16_path(m) == Path::kTc) {
     void* part = ws + c.part;
     e = ffn::launch_tc_w4a16(x, m, gate_up->tc(), true, c.gate_up, h, part, s);
     if (e == cudaSuccess) e = ffn::launch_tc_w4a16(h, m, down->tc(), false, c.down, out, part, s);
@@ -412,14 +429,25 @@ ffn_status ffn_nvfp4_forward(const void* x, int64_t m, int64_t hidden, int64_t i
 }
 
 ffn_status ffn_nvfp4_projection_plan(int64_t m, int64_t n, int64_t k, ffn_act_format format,
-                                     int gate_up, ffn_projection_plan* out) {
-  if (!out || m < 0 || n <= 0) return FFN_ERR_INVALID_ARG;
+                                     int role, ffn_projection_plan* out) {
+  if (!out || m < 0 || n <= 0 || role < 0 || role > 2) return FFN_ERR_INVALID_ARG;
   if (format != FFN_ACT_BF16 && format != FFN_ACT_NVFP4_FIXED) return FFN_ERR_INVALID_ARG;
+  const int gate_up = role == FFN_ROLE_GATE_UP;
   if (!valid_k(k) || (gate_up && n % 2)) return FFN_ERR_SHAPE;
   *out = ffn_projection_plan{FFN_KERNEL_NONE, 0, 1, 0};
   if (m == 0) return FFN_OK;
   const int ncols = (int)(gate_up ? n / 2 : n);
-  if (format == FFN_ACT_BF16 && w4a16_path(m) == Path::kTc) {
+  if (format == FFN_ACT_BF16 && role != FFN_ROLE_LINEAR && w4a16_persistent(m)) {
+    // gate+up: n = 2 * inter, k = hidden; down: n = hidden, k = inter
+    const ffn::PersistPlan p = gate_up ? ffn::plan_persist(m, k, n / 2, num_sms())
+                                       : ffn::plan_persist(m, n, k, num_sms());
+    *out = gate_up ? ffn_projection_plan{FFN_KERNEL_TC_W4A16_PERSISTENT, p.bn, 1, p.gu_grid}
+                   : ffn_projection_plan{FFN_KERNEL_TC_W4A16_PERSISTENT, p.bn, 0, p.dn_grid};
+    if (!gate_up) {  // K ranges per output tile: at most ceil(kc / (tiles*kc/grid)) + 1
+      const int64_t W = (int64_t)p.dn_tiles * p.dn_kc;
+      out->k_splits = (int)(((int64_t)p.dn_kc * p.dn_grid + W - 1) / W + 1);
+    }
+  } else if (format == FFN_ACT_BF16 && w4a16_path(m) == Path::kTc) {
     const ffn::TcPlan p = ffn::plan_tc(m, n, k, gate_up != 0, num_sms());
     *out = ffn_projection_plan{FFN_KERNEL_TC_W4A16, p.bn, p.splits, p.xtiles * p.wtiles * p.splits};
   } else if (format == FFN_ACT_BF16) {

@@ -43,6 +43,21 @@ cudaError_t launch_tile_weight(const uint8_t* codes, const uint8_t* scales, int6
                                bool gate_up, bool for_w4a16, uint8_t* out, cudaStream_t s);
 cudaError_t launch_tc_w4a16(const void* x, int64_t m, const TcWeight& w, bool silu_mul,
                             const TcPlan& p, void* y, void* partials, cudaStream_t s);
+// Few-row FFN layer (m <= 64): two persistent launches, one CTA per SM --
+// gate+up over whole tiles dealt round-robin (SiLU*mul epilogue into h), then
+// down over equal contiguous (tile, K chunk) ranges with the split-K sums
+// added in K order by the CTA that completes each tile.
+constexpr int64_t kPersistMaxRows = 64;
+struct PersistPlan {
+  int bn = 0;
+  int gu_tiles = 0, gu_kc = 0, gu_grid = 0;
+  int dn_tiles = 0, dn_kc = 0, dn_grid = 0;
+  size_t partial_bytes = 0, counter_bytes = 0;
+};
+PersistPlan plan_persist(int64_t m, int64_t hidden, int64_t inter, int num_sms);
+cudaError_t launch_persist_ffn(const void* x, int64_t m, const TcWeight& gate_up, const TcWeight& down,
+                               const PersistPlan& p, void* h, void* partials, int* counters, void* out,
+                               cudaStream_t s);
 // Fixed-format (W4A4) projection on the block-scaled FP4 tensor core.  The
 // plan depends on (n, k) only (plus the number of 128-row activation tiles).
 TcPlan plan_w4a4(int64_t m, int64_t n, int64_t k, bool gate_up, int num_sms);

@@ -507,6 +507,397 @@ tc_w4a16_kernel(const __grid_constant__ CUtensorMap xmap, const TcArgs a) {
 }
 
 // ---------------------------------------------------------------------------
+// Persistent narrow-tile W4A16 projection (m <= 64, one activation tile): the
+// two projections of an FFN layer for few rows, each one launch.  Every CTA
+// walks a list of segments -- (weight tile, range of 64-element K chunks) --
+// with its pipelines running straight through from one segment to the next
+// (the rings are indexed by the CTA's global unit count), so the weight
+// stream never stops at a tile boundary and each CTA pays its prologue once.
+//  * kModeTiles (the fused gate+up weight): the tiles are dealt round-robin
+//    to the CTAs, each whole (all K chunks); the epilogue of each tile writes
+//    h = bf16(silu(bf16 g) * bf16 u).  After its griddep_wait the kernel also
+//    zeroes the tile counters of the projection that follows it in the
+//    stream (the down projection of the same layer).
+//  * kModeRanges (the down projection, K = inter deep, few tiles): the
+//    (tile, chunk) space is cut into one contiguous, equal range per CTA;
+//    each segment's fp32 partial sums go to the workspace, slot (CTA + tile),
+//    and the CTA whose segment completes a tile's count (an atomic counter,
+//    zeroed by the preceding gate+up kernel) adds that tile's partials in K
+//    order -- a fixed order, whichever CTA finishes last -- and writes
+//    out = bf16(gs * sum).  No separate reduction launch.
+// ---------------------------------------------------------------------------
+enum : int { kModeTiles = 0, kModeRanges = 1 };
+
+struct PArgs {
+  const uint8_t* wt;   // tiled weight [ntiles][kc][4608] (W4A16 code arrangement)
+  const float* gs;     // tensor scale(s)
+  uint16_t* out;       // bf16 [m, ldo]
+  int m, n_out, ldo, kc, ntiles, x_box_rows;
+  float* partials;     // kModeRanges: [gridDim.x + ntiles][m][128]
+  int* counters;       // kModeRanges: [ntiles], zero on entry
+  int* zero_ptr;       // kModeTiles: counters of the next projection (or null)
+  int zero_count;
+};
+
+struct Seg {
+  int tile, c0, nk;
+};
+
+// Segment j of this CTA; false once there are no more.  kModeRanges needs
+// ntiles * kc >= gridDim.x (the host sizes the grid so).
+template <int MODE>
+__device__ __forceinline__ bool cta_segment(const PArgs& a, int j, Seg& s) {
+  const int G = gridDim.x, g = blockIdx.x;
+  if (MODE == kModeTiles) {
+    const int t = g + j * G;
+    if (t >= a.ntiles) return false;
+    s.tile = t;
+    s.c0 = 0;
+    s.nk = a.kc;
+    return true;
+  }
+  const int64_t W = (int64_t)a.ntiles * a.kc;
+  const int64_t lo = W * g / G, hi = W * (g + 1) / G;
+  const int t = (int)(lo / a.kc) + j;
+  const int64_t b = lo > (int64_t)t * a.kc ? lo : (int64_t)t * a.kc;
+  const int64_t e = hi < (int64_t)(t + 1) * a.kc ? hi : (int64_t)(t + 1) * a.kc;
+  if (b >= e) return false;
+  s.tile = t;
+  s.c0 = (int)(b - (int64_t)t * a.kc);
+  s.nk = (int)(e - b);
+  return true;
+}
+
+// kModeRanges: the CTA that owns unit u of the flattened (tile, chunk) space.
+__device__ __forceinline__ int range_owner(int64_t u, int64_t W, int G) {
+  return (int)(((u + 1) * G - 1) / W);
+}
+
+// Shared-memory layout of the persistent kernel: the rings (as TcCfg), the
+// barriers, then DQG epilogue buffers of 8 KB that do not alias the rings
+// (the epilogue of a segment runs while the next segment streams in).
+template <int BN, int SXS, int XC, int SWS, int SA, int DQG, int NI>
+struct PCfg {
+  using C = TcCfg<BN, SXS, XC, SWS, SA, DQG, 1, NI, false>;
+  static constexpr int kBarBytes = (C::kNumBars + 1) * 8 + 32;  // + accfree; TMEM slot, flags
+  static constexpr int kEpiOff = (C::kSmemRings + kBarBytes + 127) / 128 * 128;
+  static constexpr int kSmemAlloc = kEpiOff + DQG * 8192 + 1024;
+  static_assert(kSmemAlloc <= 232448, "shared memory budget");
+  static_assert(BN <= 64, "one activation tile of at most 64 rows");
+};
+
+template <int BN, int SXS, int XC, int SWS, int SA, int DQG, int NI, int MODE>
+__global__ void __launch_bounds__(TcCfg<BN, SXS, XC, SWS, SA, DQG, 1, NI, false>::kThreads, 1)
+tc_w4a16_persistent_kernel(const __grid_constant__ CUtensorMap xmap, const PArgs a) {
+  using C = TcCfg<BN, SXS, XC, SWS, SA, DQG, 1, NI, false>;
+  using PC = PCfg<BN, SXS, XC, SWS, SA, DQG, NI>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  uint8_t* xs = smem;
+  uint8_t* wsm = smem + C::kSmemW;
+  uint64_t* xfull = reinterpret_cast<uint64_t*>(smem + C::kSmemBar);
+  uint64_t* xempty = xfull + SXS;
+  uint64_t* wfull = xempty + SXS;
+  uint64_t* wempty = wfull + SWS;
+  uint64_t* afull = wempty + SWS;
+  uint64_t* aempty = afull + SA;
+  uint64_t* accfull = aempty + SA;        // NI barriers: one per MMA thread
+  uint64_t* accfree = accfull + NI;       // 1 barrier: the epilogue has read the accumulators
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(accfree + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  volatile int* last_flag = reinterpret_cast<volatile int*>(tmem_slot + 2);
+  int* err = &g_ffn_device_error;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  // units (= chunks) of this CTA over all its segments
+  int total = 0, nseg = 0;
+  {
+    Seg sg;
+    while (cta_segment<MODE>(a, nseg, sg)) {
+      total += sg.nk;
+      ++nseg;
+    }
+  }
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < SXS; ++s) {
+      mbar_init(&xfull[s], 1);
+      mbar_init(&xempty[s], NI);
+    }
+    for (int s = 0; s < SWS; ++s) {
+      mbar_init(&wfull[s], 1);
+      mbar_init(&wempty[s], 4 * DQG);
+    }
+    for (int s = 0; s < SA; ++s) {
+      mbar_init(&afull[s], 4);
+      mbar_init(&aempty[s], 1);
+    }
+    for (int j = 0; j < NI; ++j) mbar_init(&accfull[j], 1);
+    mbar_init(accfree, 4 * DQG);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 2) {
+    tmem_alloc(tmem_slot, C::kTmemCols);
+    tmem_relinquish();
+  }
+  if (warp == 3 && lane == 0) tma_prefetch_desc(&xmap);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  griddep_launch_dependents();
+
+  if (warp == 0) {
+    // ------------------------------------------------- weight producer
+    if (lane == 0) {
+      int u = 0, issued_rounds = 0;
+      bool ok = true;
+      Seg sg;
+      for (int j = 0; ok && cta_segment<MODE>(a, j, sg); ++j) {
+        const uint8_t* src = a.wt + ((size_t)sg.tile * a.kc + sg.c0) * kChunkBytes;
+        for (int c = 0; c < sg.nk; ++c, ++u) {
+          const int r = u / DQG, slot = u % DQG, st = r % SWS;
+          if (slot == 0) {
+            if (r >= SWS && !mbar_wait(&wempty[st], ((r / SWS) - 1) & 1, abort_flag, err, 1)) {
+              ok = false;
+              break;
+            }
+            mbar_arrive_expect_tx(&wfull[st], min(DQG, total - u) * kChunkBytes);
+            ++issued_rounds;
+          }
+          bulk_load(wsm + st * C::kWStageBytes + slot * kChunkBytes, src + (size_t)c * kChunkBytes,
+                    kChunkBytes, &wfull[st]);
+        }
+      }
+      for (int r = max(0, issued_rounds - SWS); r < issued_rounds; ++r)
+        wait_drain(&wfull[r % SWS], (r / SWS) & 1);
+    }
+  } else if (warp == 3) {
+    // --------------------------------------------- activation producer
+    if (lane == 0) {
+      griddep_wait();  // x (or h) comes from the previous kernel
+      if (MODE == kModeTiles)
+        for (int i = blockIdx.x; i < a.zero_count; i += gridDim.x) a.zero_ptr[i] = 0;
+      int u = 0, issued = 0;
+      bool ok = true;
+      Seg sg;
+      for (int j = 0; ok && cta_segment<MODE>(a, j, sg); ++j) {
+        for (int c = 0; c < sg.nk; ++c, ++u) {
+          const int t = u / XC, pos = u % XC, st = t % SXS;
+          if (pos == 0) {
+            if (t >= SXS && !mbar_wait(&xempty[st], ((t / SXS) - 1) & 1, abort_flag, err, 1)) {
+              ok = false;
+              break;
+            }
+            mbar_arrive_expect_tx(&xfull[st], min(XC, total - u) * a.x_box_rows * 128);
+            ++issued;
+          }
+          tma_load_2d(xs + st * C::kXStageBytes + pos * BN * 128, &xmap, (sg.c0 + c) * kChunkK, 0,
+                      &xfull[st]);
+        }
+      }
+      for (int t = max(0, issued - SXS); t < issued; ++t) wait_drain(&xfull[t % SXS], (t / SXS) & 1);
+    }
+  } else if (warp == 1 || (NI == 2 && warp == 2)) {
+    // -------------------------------------------------- MMA issuer(s)
+    if (lane == 0) {
+      const int jt = warp - 1;  // units u with u % NI == jt
+      const uint32_t idesc = idesc_bf16_f32(kTileRows, BN);
+      const uint32_t d = tmem + jt * BN;
+      int u = 0;
+      bool ok = true;
+      Seg sg;
+      for (int j = 0; ok && cta_segment<MODE>(a, j, sg); ++j) {
+        if (j > 0 && !mbar_wait(accfree, (j - 1) & 1, abort_flag, err, 2)) break;
+        tc_fence_after();
+        bool first = true;
+        for (int c = 0; c < sg.nk; ++c, ++u) {
+          if (u % NI != jt) continue;
+          const int t = u / XC, sx = t % SXS, sa = u % SA;
+          if (u % XC == jt && !mbar_wait(&xfull[sx], (t / SXS) & 1, abort_flag, err, 2)) {
+            ok = false;
+            break;
+          }
+          if (!mbar_wait(&afull[sa], (u / SA) & 1, abort_flag, err, 2)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t a_base = tmem + C::kAColBase + C::kSlotCols * sa;
+          const uint64_t b_base = smem_desc_sw128(smem_u32(xs + sx * C::kXStageBytes + (u % XC) * BN * 128));
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk)
+            mma_bf16_ts(d, a_base + 8 * kk, b_base + 2 * kk, idesc, (first && kk == 0) ? 0u : 1u);
+          first = false;
+          mma_commit(&aempty[sa]);
+          if (u + NI >= (t + 1) * XC || u + NI >= total) mma_commit(&xempty[sx]);
+        }
+        mma_commit(&accfull[jt]);  // this segment's MMAs of this thread are complete
+      }
+    }
+  } else if (warp >= 4) {
+    // ------------------------------- dequant, then each segment's epilogue
+    const int g = (warp - 4) >> 2;
+    const int q = warp & 3;
+    const int row = 32 * q + lane;
+    const int tid = threadIdx.x - 128;  // 0 .. 128 * DQG - 1
+    const uint32_t lane_addr = (uint32_t)(32 * q) << 16;
+    const int sf_off = 16 * lane + 4 * q;
+    int u = 0;
+    bool ok = true;
+    bool waited = false;
+    Seg sg;
+    for (int j = 0; ok && cta_segment<MODE>(a, j, sg); ++j) {
+      const int u0 = u;
+      for (int c = 0; c < sg.nk; ++c, ++u) {
+        if (u % DQG != g) continue;
+        const int r = u / DQG, sw = r % SWS, sa = u % SA;
+        if (u >= SA) {
+          const bool okw = mbar_wait(&aempty[sa], ((u / SA) - 1) & 1, abort_flag, err, 4);
+          if (!__all_sync(0xffffffffu, okw)) { ok = false; break; }
+          tc_fence_after();
+        }
+        const bool okw = mbar_wait(&wfull[sw], (r / SWS) & 1, abort_flag, err, 4);
+        if (!__all_sync(0xffffffffu, okw)) { ok = false; break; }
+        const uint8_t* w = wsm + sw * C::kWStageBytes + g * kChunkBytes;
+        const uint4 lo = *reinterpret_cast<const uint4*>(w + 16 * row);
+        const uint4 hi = *reinterpret_cast<const uint4*>(w + 2048 + 16 * row);
+        const uint32_t sc = *reinterpret_cast<const uint32_t*>(w + 4096 + sf_off);
+        uint32_t v[32];
+        dequant64_w4a16(lo, hi, sc, v);
+        tmem_st32(tmem + lane_addr + C::kAColBase + C::kSlotCols * sa, v);
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&wempty[sw]);
+        tmem_st_wait();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&afull[sa]);
+      }
+      if (!ok) break;
+      // ---- epilogue of segment j: accumulators -> h, or partials (+ finalise)
+      bool done = true;
+      for (int jt = 0; jt < NI; ++jt) done = mbar_wait(&accfull[jt], j & 1, abort_flag, err, 8) && done;
+      done = __all_sync(0xffffffffu, done);
+      tc_fence_after();
+      if (!waited) {
+        griddep_wait();  // the previous kernel may still read this kernel's outputs
+        waited = true;
+      }
+      if (!done || *abort_flag) { ok = false; break; }
+      // accumulator jt holds units u0 + i with (u0 + i) % NI == jt, i < nk
+      unsigned used = 0;
+      for (int jt = 0; jt < NI; ++jt)
+        if (((jt - u0) % NI + NI) % NI < sg.nk) used |= 1u << jt;
+      const int cols = min(a.m, BN);
+      if (MODE == kModeTiles) {
+        // gate rows 0..63 and up rows 64..127 of tile t: h[:, 64t + row]
+        float* U = reinterpret_cast<float*>(smem + PC::kEpiOff) + g * 2048;  // [32][64]
+        for (int c = g; c * 32 < cols; c += DQG) {
+          const int jmax = min(32, cols - 32 * c);
+          float acc[32];
+#pragma unroll
+          for (int i = 0; i < 32; ++i) acc[i] = 0.0f;
+          for (int jt = 0; jt < NI; ++jt) {
+            if (!(used >> jt & 1)) continue;
+            uint32_t v0[16], v1[16];
+            tmem_ld16(tmem + lane_addr + jt * BN + 32 * c, v0);
+            if (BN - 32 * c > 16) tmem_ld16(tmem + lane_addr + jt * BN + 32 * c + 16, v1);
+            tmem_ld_wait();
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+              acc[i] += __uint_as_float(v0[i]);
+              if (BN - 32 * c > 16) acc[16 + i] += __uint_as_float(v1[i]);
+            }
+          }
+          // rows 64..127 (up) hand bf16(gs_u * u) to rows 0..63 (gate)
+          if (q >= 2) {
+            const float gsu = a.gs[1] * kW4A16Unscale;
+#pragma unroll
+            for (int i = 0; i < 32; ++i) U[i * 64 + (row - 64)] = bf16_round(gsu * acc[i]);
+          }
+          named_bar_sync(1 + g, 128);
+          if (q < 2) {
+            const float gsg = a.gs[0] * kW4A16Unscale;
+            const int n = 64 * sg.tile + row;
+            if (n < a.n_out) {
+#pragma unroll
+              for (int i = 0; i < 32; ++i) {
+                if (i < jmax) {
+                  const float gv = bf16_round(gsg * acc[i]);
+                  a.out[(size_t)(32 * c + i) * a.ldo + n] = f32_to_bf16_bits(silu_fast(gv) * U[i * 64 + row]);
+                }
+              }
+            }
+          }
+          named_bar_sync(1 + g, 128);
+        }
+      } else {
+        // this segment's partial sums -> slot (CTA + tile), rows [act row][tile row]
+        float* P = a.partials + (size_t)(blockIdx.x + sg.tile) * a.m * kTileRows;
+        for (int c = g; c * 32 < cols; c += DQG) {
+          const int jmax = min(32, cols - 32 * c);
+          float acc[32];
+#pragma unroll
+          for (int i = 0; i < 32; ++i) acc[i] = 0.0f;
+          for (int jt = 0; jt < NI; ++jt) {
+            if (!(used >> jt & 1)) continue;
+            uint32_t v0[16], v1[16];
+            tmem_ld16(tmem + lane_addr + jt * BN + 32 * c, v0);
+            if (BN - 32 * c > 16) tmem_ld16(tmem + lane_addr + jt * BN + 32 * c + 16, v1);
+            tmem_ld_wait();
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+              acc[i] += __uint_as_float(v0[i]);
+              if (BN - 32 * c > 16) acc[16 + i] += __uint_as_float(v1[i]);
+            }
+          }
+#pragma unroll
+          for (int i = 0; i < 32; ++i)
+            if (i < jmax) P[(size_t)(32 * c + i) * kTileRows + row] = acc[i];
+        }
+        __threadfence();
+        named_bar_sync(1 + DQG, 128 * DQG);
+        if (tid == 0) {
+          const int64_t W = (int64_t)a.ntiles * a.kc;
+          const int G = gridDim.x;
+          const int g0 = range_owner((int64_t)sg.tile * a.kc, W, G);
+          const int g1 = range_owner((int64_t)sg.tile * a.kc + a.kc - 1, W, G);
+          *last_flag = atomicAdd(&a.counters[sg.tile], 1) == g1 - g0 ? 1 : 0;
+        }
+        named_bar_sync(1 + DQG, 128 * DQG);
+        if (*last_flag) {
+          __threadfence();
+          const int64_t W = (int64_t)a.ntiles * a.kc;
+          const int G = gridDim.x;
+          const int g0 = range_owner((int64_t)sg.tile * a.kc, W, G);
+          const int g1 = range_owner((int64_t)sg.tile * a.kc + a.kc - 1, W, G);
+          const float gsd = a.gs[0] * kW4A16Unscale;
+          for (int idx = tid; idx < a.m * kTileRows; idx += 128 * DQG) {
+            const int jr = idx / kTileRows, rr = idx % kTileRows;
+            const int n = kTileRows * sg.tile + rr;
+            float sum = 0.0f;
+            for (int gg = g0; gg <= g1; ++gg)
+              sum += __ldcg(a.partials + ((size_t)(gg + sg.tile) * a.m + jr) * kTileRows + rr);
+            if (n < a.n_out) a.out[(size_t)jr * a.ldo + n] = f32_to_bf16_bits(gsd * sum);
+          }
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(accfree);
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 2) {
+    tc_fence_after();
+    tmem_dealloc(tmem, C::kTmemCols);
+  }
+}
+
+// ---------------------------------------------------------------------------
 // Fixed-format (W4A4) projection on the block-scaled FP4 tensor core
 // ("metrale_model_layers/layers/dense_ffn_fixed.rs", forward_fixed: the
 // nvfp4_proj_mx projections).  D[n, r] = sum_k (wq * sw)[n, k] (xq * sx)[r, k]
@@ -806,9 +1197,88 @@ cudaError_t launch_bn(int bn, const CUtensorMap& map, const TcArgs& a, dim3 grid
   }
 }
 
+template <int BN, int SXS, int XC, int SWS, int SA, int DQG, int NI, int MODE>
+cudaError_t launch_persist_cfg(const CUtensorMap& map, const PArgs& a, int grid, cudaStream_t s) {
+  using C = TcCfg<BN, SXS, XC, SWS, SA, DQG, 1, NI, false>;
+  using PC = PCfg<BN, SXS, XC, SWS, SA, DQG, NI>;
+  auto kern = tc_w4a16_persistent_kernel<BN, SXS, XC, SWS, SA, DQG, NI, MODE>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, PC::kSmemAlloc);
+  if (e != cudaSuccess) return e;
+  return launch_pdl(kern, dim3(grid), dim3(C::kThreads), PC::kSmemAlloc, s, map, a);
+}
+
+template <int MODE>
+cudaError_t launch_persist_bn(int bn, const CUtensorMap& map, const PArgs& a, int grid, cudaStream_t s) {
+  switch (bn) {
+    // BN, activation stages, chunks per activation stage, weight stages
+    // (rounds of DQG chunks), TMEM A slots (chunks), dequant warpgroups, MMA
+    // threads.  One CTA per SM: TMEM NI*BN + 32*SA columns of 512.
+    case 16: return launch_persist_cfg<16, 4, 6, 10, 12, 3, 2, MODE>(map, a, grid, s);
+    case 32: return launch_persist_cfg<32, 3, 6, 8, 12, 3, 2, MODE>(map, a, grid, s);
+    default: return launch_persist_cfg<64, 3, 4, 8, 6, 2, 2, MODE>(map, a, grid, s);
+  }
+}
+
 }  // namespace
 
 int tc_tile_bytes_per_row_chunk() { return kChunkBytes; }
+
+PersistPlan plan_persist(int64_t m, int64_t hidden, int64_t inter, int num_sms) {
+  PersistPlan p;
+  p.bn = m <= 16 ? 16 : m <= 32 ? 32 : 64;
+  p.gu_tiles = (int)((inter + 63) / 64);
+  p.gu_kc = (int)((hidden + kChunkK - 1) / kChunkK);
+  p.gu_grid = p.gu_tiles < num_sms ? p.gu_tiles : num_sms;
+  p.dn_tiles = (int)((hidden + kTileRows - 1) / kTileRows);
+  p.dn_kc = (int)((inter + kChunkK - 1) / kChunkK);
+  const int64_t W = (int64_t)p.dn_tiles * p.dn_kc;
+  p.dn_grid = (int)(W < num_sms ? W : num_sms);
+  p.partial_bytes = (size_t)(p.dn_grid + p.dn_tiles) * m * kTileRows * sizeof(float);
+  p.counter_bytes = (size_t)p.dn_tiles * sizeof(int);
+  return p;
+}
+
+cudaError_t launch_persist_ffn(const void* x, int64_t m, const TcWeight& gate_up, const TcWeight& down,
+                               const PersistPlan& p, void* h, void* partials, int* counters, void* out,
+                               cudaStream_t s) {
+  const int box_rows = (int)m;
+  const int64_t inter = gate_up.n / 2, hidden = down.n;
+  CUtensorMap xm, hm;
+  if (!make_x_map(&xm, x, m, gate_up.k, box_rows) || !make_x_map(&hm, h, m, down.k, box_rows))
+    return cudaErrorInvalidValue;
+  PArgs a{};
+  a.wt = gate_up.tiled16;
+  a.gs = gate_up.gs;
+  a.out = static_cast<uint16_t*>(h);
+  a.m = (int)m;
+  a.n_out = (int)inter;
+  a.ldo = (int)inter;
+  a.kc = p.gu_kc;
+  a.ntiles = p.gu_tiles;
+  a.x_box_rows = box_rows;
+  a.zero_ptr = counters;
+  a.zero_count = p.dn_tiles;
+  cudaError_t e;
+  {
+    ProfScope prof(s, "tc_w4a16_gate_up_silu_persistent");
+    e = launch_persist_bn<kModeTiles>(p.bn, xm, a, p.gu_grid, s);
+  }
+  if (e != cudaSuccess) return e;
+  PArgs b{};
+  b.wt = down.tiled16;
+  b.gs = down.gs;
+  b.out = static_cast<uint16_t*>(out);
+  b.m = (int)m;
+  b.n_out = (int)hidden;
+  b.ldo = (int)hidden;
+  b.kc = p.dn_kc;
+  b.ntiles = p.dn_tiles;
+  b.x_box_rows = box_rows;
+  b.partials = static_cast<float*>(partials);
+  b.counters = counters;
+  ProfScope prof(s, "tc_w4a16_down_persistent");
+  return launch_persist_bn<kModeRanges>(p.bn, hm, b, p.dn_grid, s);
+}
 
 int64_t tc_tiled_bytes(int64_t n, int64_t k, bool gate_up) {
   const int64_t tiles = gate_up ? (n / 2 + 63) / 64 : (n + kTileRows - 1) / kTileRows;

@@ -36,7 +36,9 @@ class ProjectionPlan(ctypes.Structure):
                 ("grid", ctypes.c_int)]
 
 
-KERNEL_FAMILIES = {0: "none", 1: "tc_w4a16", 2: "tc_w4a4", 3: "gemv_w4a16", 4: "gemv_w4a4"}
+KERNEL_FAMILIES = {0: "none", 1: "tc_w4a16", 2: "tc_w4a4", 3: "gemv_w4a16", 4: "gemv_w4a4",
+                   5: "tc_w4a16_persistent"}
+ROLES = {"linear": 0, "gate_up": 1, "down": 2}
 
 
 class KernelTime(ctypes.Structure):
@@ -67,6 +69,8 @@ def _load() -> ctypes.CDLL:
         "ffn_nvfp4_linear_noalloc": (ctypes.c_int, [vp, i64, vp, vp, vp]),
         "ffn_nvfp4_projection_plan": (ctypes.c_int, [i64, i64, i64, ctypes.c_int, ctypes.c_int,
                                                      P(ProjectionPlan)]),
+        "ffn_nvfp4_tensor_peak": (ctypes.c_int, [ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                                 P(ctypes.c_double)]),
         "ffn_nvfp4_profile_begin": (ctypes.c_int, []),
         "ffn_nvfp4_device_error": (ctypes.c_int, [P(ctypes.c_int), ctypes.c_int]),
         "ffn_nvfp4_profile_end": (ctypes.c_int, [P(KernelTime), ctypes.c_int, P(ctypes.c_int)]),
@@ -294,10 +298,20 @@ def ffn_nvfp4_linear_noalloc(x: torch.Tensor, w: Weight, y=None, stream=None) ->
     return y
 
 
-def ffn_nvfp4_projection_plan(m: int, n: int, k: int, fmt="bf16", gate_up: bool = False) -> dict:
-    """The kernel configuration a projection of m rows selects (nothing launched)."""
+def ffn_nvfp4_projection_plan(m: int, n: int, k: int, fmt="bf16", role: str = "linear") -> dict:
+    """The kernel configuration a projection of m rows selects (nothing
+    launched); role: 'linear', or the forward's 'gate_up' / 'down'."""
     p = ProjectionPlan()
-    _check("ffn_nvfp4_projection_plan", lib.ffn_nvfp4_projection_plan(m, n, k, _fmt(fmt), int(gate_up),
+    _check("ffn_nvfp4_projection_plan", lib.ffn_nvfp4_projection_plan(m, n, k, _fmt(fmt), ROLES[role],
                                                                       ctypes.byref(p)))
     return {"family": KERNEL_FAMILIES.get(p.family, str(p.family)), "tile_rows": p.tile_rows,
             "k_splits": p.k_splits, "grid": p.grid}
+
+
+def ffn_nvfp4_tensor_peak(kind: str = "bf16", issuers: int = 1, iters: int = 20000) -> float:
+    """Measured dense tensor-core TFLOP/s of the current GPU for the MMA kind
+    the library issues ('bf16': kind::f16; 'nvfp4': kind::mxf4nvf4)."""
+    out = ctypes.c_double()
+    _check("ffn_nvfp4_tensor_peak", lib.ffn_nvfp4_tensor_peak({"bf16": 0, "nvfp4": 1}[kind], issuers, iters,
+                                                              ctypes.byref(out)))
+    return out.value

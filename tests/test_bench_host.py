@@ -89,7 +89,9 @@ def test_traffic_reported_only_for_the_captured_sources():
 def test_roofline_bound_uses_each_formats_own_peak(layers):
     peaks = {"hbm_gbs": 6557.8, "bf16_tflops": 1671.7, "bf16_tflops_sustained": 1402.4}
     assert bench.tensor_peak(peaks, "bf16")[0] == 1671.7
-    assert bench.tensor_peak(peaks, "nvfp4_fixed")[0] == 1671.7 * 4
+    assert bench.tensor_peak(peaks, "nvfp4_fixed")[0] == 1671.7 * 4   # nominal fallback
+    assert bench.tensor_peak(dict(peaks, fp4_tflops=6000.0), "nvfp4_fixed")[0] == 6000.0
+    assert "probe" in bench.tensor_peak(dict(peaks, fp4_tflops=6000.0), "nvfp4_fixed")[1]
     dec = layers["decode"][0]
     bound, units = dec.kernel_units("tc_w4a16_gate_up_silu", peaks)
     assert bound == "hbm" and units == bench.nvfp4_bytes(2 * 17408, 5120) + 5120 * 2 + 17408 * 2

@@ -128,3 +128,58 @@ def test_w4a4_exact_inputs_bit_exact(native, m, n, k, splits):
     bad = np.argwhere(got != ref)
     assert bad.size == 0, f"{len(bad)} mismatches, first at {bad[:3].tolist()}"
     assert native.ffn_nvfp4_device_error(clear=False) == 0
+
+
+def exact_ffn_inputs(rng, m, H, I, down_nonzeros=4):
+    """An FFN whose every intermediate is exact, so the whole layer must match
+    the oracle bit for bit (all tensor scales 1):
+      x in {1, 2};  gate: non-negative codes, scales 2^-3..2^0, so every
+      g = x . w_g is a positive dyadic sum, here >= 32 (asserted), where
+      silu(g) = g / (1 + e^-g) equals g in fp32 and rounds like g in fp64;
+      up: one non-zero code (+-1 or +-2) per row in a block of scale 2^-4,
+      so u = +-2^e and h = bf16(silu(g) * u) = bf16(g) * u exactly;
+      down: `down_nonzeros` codes per row, scales 1, so each output is a
+      short sum of exact products below 2^16 with at least 2^-7 resolution."""
+    x = rng.integers(1, 3, (m, H)).astype(np.float32)
+    mag = rng.integers(1, 8, (I, H)).astype(np.uint8)            # sign bit 0
+    gc = (mag[:, 0::2] | (mag[:, 1::2] << 4)).astype(np.uint8)
+    gsc = rng.choice(POW2_SCALES, (I, H // 16)).astype(np.uint8)
+    un = np.zeros((I, H), np.uint8)
+    cols = rng.integers(0, H, I)
+    un[np.arange(I), cols] = rng.choice(np.array([0x2, 0xA, 0x4, 0xC], np.uint8), I)
+    uc = (un[:, 0::2] | (un[:, 1::2] << 4)).astype(np.uint8)
+    usc = np.full((I, H // 16), 0x18, np.uint8)                  # 2^-4
+    dn = np.zeros((H, I), np.uint8)
+    for r in range(H):
+        dn[r, rng.choice(I, down_nonzeros, replace=False)] = rng.integers(1, 16, down_nonzeros)
+    dc = (dn[:, 0::2] | (dn[:, 1::2] << 4)).astype(np.uint8)
+    dsc = np.full((H, I // 16), 0x38, np.uint8)                  # 1
+    one = np.float32(1.0)
+    g = O.round_to_bf16(O.project_w4a16(x.astype(np.float64), gc, gsc, one))
+    assert g.min() >= 32.0, g.min()
+    return x, (gc, gsc, one), (uc, usc, one), (dc, dsc, one)
+
+
+FFN_EXACT_CASES = [
+    # (m, hidden, inter): few-row persistent kernels for m <= 64 (tile widths
+    # 16/32/64; down K ranges that cut tiles, inter % 64 == 32), per-tile
+    # kernels with split-K and the SiLU*mul reduction for wider m
+    (1, 512, 1536), (5, 1024, 4096), (16, 512, 800), (33, 512, 1536), (64, 1024, 2048),
+    (100, 512, 1536), (300, 512, 800),
+]
+
+
+@pytest.mark.parametrize("m,H,I", FFN_EXACT_CASES)
+def test_ffn_exact_inputs_bit_exact(native, m, H, I):
+    rng = np.random.default_rng(3000 + m + H + I)
+    x, qg, qu, qd = exact_ffn_inputs(rng, m, H, I)
+    ref = O.ffn_w4a16(x.astype(np.float64), qg, qu, qd)
+    hs = [make_handle(native, q[0], q[1]) for q in (qg, qu, qd)]
+    gate_up = native.ffn_nvfp4_weight_create_gate_up(hs[0], hs[1])
+    out = native.ffn_nvfp4_forward(torch.from_numpy(x).cuda().to(torch.bfloat16), gate_up, hs[2], "bf16")
+    torch.cuda.synchronize()
+    got = bf16_to_f64(out)
+    bad = np.argwhere(got != ref)
+    plan = native.ffn_nvfp4_projection_plan(m, H, I, "bf16", role="down")
+    assert bad.size == 0, f"{plan}: {len(bad)} mismatches, first at {bad[:3].tolist()}"
+    assert native.ffn_nvfp4_device_error(clear=False) == 0
