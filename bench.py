@@ -234,7 +234,7 @@ class Workload:
             self.sets = int(math.ceil(4 * L2_BYTES / self.weight_bytes))
         self.handles = []
         for _ in range(self.sets):
-            g, u, d = (native.ffn_nvfp4_weight_create(*t) for t in q)
+            g, u, d = (native.ffn_nvfp4_weight_create(*t, formats=fmt) for t in q)
             self.handles.append((native.ffn_nvfp4_weight_create_gate_up(g, u), d))
             del g, u
         del q

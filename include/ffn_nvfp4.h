@@ -113,20 +113,39 @@ ffn_status ffn_nvfp4_quantize_activations(const void* x_bf16, int64_t m, int64_t
                                           void* codes, void* block_scales,
                                           void* stream);
 
+/* Activation formats a weight handle is built for (bit set). */
+typedef enum ffn_weight_formats {
+  FFN_FORMAT_BF16 = 1,         /* serves FFN_ACT_BF16 (W4A16)         */
+  FFN_FORMAT_NVFP4_FIXED = 2,  /* serves FFN_ACT_NVFP4_FIXED (W4A4)   */
+  FFN_FORMAT_ALL = 3
+} ffn_weight_formats;
+
 /* Build a weight handle from NVFP4 tensors of logical shape [n, k] (codes,
- * block_scales as above, global_scale one device float).  Copies the data
- * (the caller keeps ownership of its buffers) and builds the kernel layouts.
- * Allocates device memory; enqueues copies on `stream`; the handle is usable
- * by later work on `stream` (other streams: synchronise first).
- * Errors: FFN_ERR_SHAPE unless n > 0 and k is a positive multiple of 32. */
+ * block_scales as above, global_scale one device float) for the activation
+ * formats in `formats` (FFN_FORMAT_* bits, not 0).  Reads the caller's
+ * buffers (which it may free afterwards) and builds, per format, one
+ * re-tiled copy in the layout that format's kernels stream: 0.5625 bytes per
+ * weight and format, plus tile padding -- the canonical copy is not kept.
+ * Allocates device memory; enqueues its work on `stream`; the handle is
+ * usable by later work on `stream` (other streams: synchronise first).
+ * Errors: FFN_ERR_SHAPE unless n > 0 and k is a positive multiple of 32;
+ * FFN_ERR_INVALID_ARG for formats outside FFN_FORMAT_ALL or 0.  Using a
+ * handle with a format it was not built for returns FFN_ERR_UNSUPPORTED. */
+ffn_status ffn_nvfp4_weight_create_ex(const void* codes, const void* block_scales,
+                                      const float* global_scale, int64_t n, int64_t k,
+                                      unsigned formats, void* stream, ffn_nvfp4_weight** out);
+
+/* ffn_nvfp4_weight_create_ex with FFN_FORMAT_ALL (both activation formats). */
 ffn_status ffn_nvfp4_weight_create(const void* codes, const void* block_scales,
                                    const float* global_scale, int64_t n, int64_t k,
                                    void* stream, ffn_nvfp4_weight** out);
 
 /* Fused gate+up handle of logical shape [2*inter, hidden]: rows [0, inter)
  * are `gate`, rows [inter, 2*inter) are `up`, byte for byte, each keeping its
- * own tensor scale.  `gate` and `up` must share (n, k) and stay owned by the
- * caller (they may be destroyed afterwards). */
+ * own tensor scale; built for the formats both parts serve (re-tiled from
+ * their tiles; FFN_ERR_UNSUPPORTED if they share none).  `gate` and `up` must
+ * share (n, k) and device and stay owned by the caller (they may be destroyed
+ * afterwards). */
 ffn_status ffn_nvfp4_weight_create_gate_up(const ffn_nvfp4_weight* gate,
                                            const ffn_nvfp4_weight* up, void* stream,
                                            ffn_nvfp4_weight** out);
@@ -138,6 +157,11 @@ ffn_status ffn_nvfp4_weight_destroy(ffn_nvfp4_weight* w);
 /* Logical dims of a handle; *is_gate_up = 1 for a fused gate+up handle. */
 ffn_status ffn_nvfp4_weight_dims(const ffn_nvfp4_weight* w, int64_t* n, int64_t* k,
                                  int* is_gate_up);
+
+/* The FFN_FORMAT_* bits a handle serves and the device bytes it holds
+ * (either pointer may be NULL). */
+ffn_status ffn_nvfp4_weight_info(const ffn_nvfp4_weight* w, unsigned* formats,
+                                 size_t* device_bytes);
 
 /* Workspace bytes ffn_nvfp4_forward needs for (m, hidden, inter, format). */
 ffn_status ffn_nvfp4_workspace_size(int64_t m, int64_t hidden, int64_t inter,

@@ -15,11 +15,13 @@ struct ffn_nvfp4_weight {
   int64_t n = 0, k = 0;
   int gate_up = 0;
   int device = 0;
-  uint8_t* codes = nullptr;   // [n, k/2] canonical
-  uint8_t* scales = nullptr;  // [n, k/16] canonical
+  unsigned formats = 0;       // FFN_FORMAT_* bits the handle serves
+  size_t bytes = 0;           // device bytes held
+  uint8_t* codes = nullptr;   // [n, k/2] canonical (only for a forced CUDA-core arm)
+  uint8_t* scales = nullptr;  // [n, k/16] canonical (likewise)
   float* gs = nullptr;        // 1 float, or 2 (gate, up) for a fused handle
-  uint8_t* tiled = nullptr;   // tensor-core layout (see tc_gemm.cu), natural codes
-  uint8_t* tiled16 = nullptr; // the same tiles with the W4A16 code-bit arrangement
+  uint8_t* tiled = nullptr;   // tensor-core layout (see tc_gemm.cu), natural codes: fixed format
+  uint8_t* tiled16 = nullptr; // the same tiles with the W4A16 code-bit arrangement: bf16
   WeightView view() const { return WeightView{codes, scales, gs, n, k}; }
   ffn::TcWeight tc() const { return ffn::TcWeight{tiled, tiled16, gs, n, k}; }
 };
@@ -101,6 +103,19 @@ Path w4a4_path() {
     return (v && !strcmp(v, "gemv")) ? Path::kGemv : Path::kTc;
   }();
   return p;
+}
+
+// The canonical NVFP4 copy is read only by the CUDA-core arms, which run
+// only when forced by environment; otherwise handles keep just the tiled
+// copies their formats need (0.5625 B per weight and format, plus tile padding).
+bool keep_canonical() { return w4a16_forced() == 1 || w4a4_path() == Path::kGemv; }
+
+// The handle holds what `format` reads on the path that will run.
+bool serves(const ffn_nvfp4_weight* w, ffn_act_format f) {
+  const unsigned bit = f == FFN_ACT_BF16 ? FFN_FORMAT_BF16 : FFN_FORMAT_NVFP4_FIXED;
+  if (!(w->formats & bit)) return false;
+  const bool gemv = f == FFN_ACT_BF16 ? w4a16_forced() == 1 : w4a4_path() == Path::kGemv;
+  return gemv ? w->codes != nullptr : (f == FFN_ACT_BF16 ? w->tiled16 : w->tiled) != nullptr;
 }
 
 // Workspace layout of ffn_nvfp4_forward / ffn_nvfp4_linear (each region
@@ -185,12 +200,13 @@ Carve carve_linear(int64_t m, int64_t n, int64_t k, ffn_act_format f) {
 }
 
 template <class T>
-ffn_status alloc(T** p, size_t bytes) {
+ffn_status alloc(T** p, size_t bytes, size_t* total = nullptr) {
   if (cudaMalloc(reinterpret_cast<void**>(p), bytes) != cudaSuccess) {
     cudaGetLastError();
     *p = nullptr;
     return FFN_ERR_OOM;
   }
+  if (total) *total += bytes;
   return FFN_OK;
 }
 
@@ -256,12 +272,13 @@ ffn_status ffn_nvfp4_quantize_activations(const void* x_bf16, int64_t m, int64_t
       ffn::launch_quantize_activations(x_bf16, m, k, codes, block_scales, as_stream(stream)));
 }
 
-ffn_status ffn_nvfp4_weight_create(const void* codes, const void* block_scales,
-                                   const float* global_scale, int64_t n, int64_t k,
-                                   void* stream, ffn_nvfp4_weight** out) {
+ffn_status ffn_nvfp4_weight_create_ex(const void* codes, const void* block_scales,
+                                      const float* global_scale, int64_t n, int64_t k,
+                                      unsigned formats, void* stream, ffn_nvfp4_weight** out) {
   if (!out) return FFN_ERR_INVALID_ARG;
   *out = nullptr;
   if (!codes || !block_scales || !global_scale) return FFN_ERR_INVALID_ARG;
+  if (formats == 0 || (formats & ~(unsigned)FFN_FORMAT_ALL)) return FFN_ERR_INVALID_ARG;
   if (n <= 0 || !valid_k(k)) return FFN_ERR_SHAPE;
   if (!aligned16(codes) || !aligned16(block_scales)) return FFN_ERR_ALIGNMENT;
   if (ffn_status st = precheck()) return st;
@@ -269,28 +286,41 @@ ffn_status ffn_nvfp4_weight_create(const void* codes, const void* block_scales,
   if (!w) return FFN_ERR_OOM;
   w->n = n;
   w->k = k;
+  w->formats = formats;
   cudaGetDevice(&w->device);
   const cudaStream_t s = as_stream(stream);
   ffn_status st = FFN_OK;
-  if ((st = alloc(&w->codes, (size_t)n * k / 2)) || (st = alloc(&w->scales, (size_t)n * k / 16)) ||
-      (st = alloc(&w->gs, 2 * sizeof(float)))) {
+  if ((st = alloc(&w->gs, 2 * sizeof(float), &w->bytes))) {
     free_weight(w);
     return st;
   }
-  cudaError_t e = cudaMemcpyAsync(w->codes, codes, (size_t)n * k / 2, cudaMemcpyDeviceToDevice, s);
-  if (e == cudaSuccess)
-    e = cudaMemcpyAsync(w->scales, block_scales, (size_t)n * k / 16, cudaMemcpyDeviceToDevice, s);
-  if (e == cudaSuccess)
-    e = cudaMemcpyAsync(w->gs, global_scale, sizeof(float), cudaMemcpyDeviceToDevice, s);
-  if (e == cudaSuccess) {
-    const size_t tb = (size_t)ffn::tc_tiled_bytes(n, k, false);
-    if ((st = alloc(&w->tiled, tb)) || (st = alloc(&w->tiled16, tb))) {
+  cudaError_t e = cudaMemcpyAsync(w->gs, global_scale, sizeof(float), cudaMemcpyDeviceToDevice, s);
+  if (e == cudaSuccess && keep_canonical()) {
+    if ((st = alloc(&w->codes, (size_t)n * k / 2, &w->bytes)) ||
+        (st = alloc(&w->scales, (size_t)n * k / 16, &w->bytes))) {
       free_weight(w);
       return st;
     }
-    e = ffn::launch_tile_weight(w->codes, w->scales, n, k, false, false, w->tiled, s);
+    e = cudaMemcpyAsync(w->codes, codes, (size_t)n * k / 2, cudaMemcpyDeviceToDevice, s);
     if (e == cudaSuccess)
-      e = ffn::launch_tile_weight(w->codes, w->scales, n, k, false, true, w->tiled16, s);
+      e = cudaMemcpyAsync(w->scales, block_scales, (size_t)n * k / 16, cudaMemcpyDeviceToDevice, s);
+  }
+  const size_t tb = (size_t)ffn::tc_tiled_bytes(n, k, false);
+  const auto* c8 = static_cast<const uint8_t*>(codes);
+  const auto* s8 = static_cast<const uint8_t*>(block_scales);
+  if (e == cudaSuccess && (formats & FFN_FORMAT_NVFP4_FIXED)) {
+    if ((st = alloc(&w->tiled, tb, &w->bytes))) {
+      free_weight(w);
+      return st;
+    }
+    e = ffn::launch_tile_weight(c8, s8, n, k, false, false, w->tiled, s);
+  }
+  if (e == cudaSuccess && (formats & FFN_FORMAT_BF16)) {
+    if ((st = alloc(&w->tiled16, tb, &w->bytes))) {
+      free_weight(w);
+      return st;
+    }
+    e = ffn::launch_tile_weight(c8, s8, n, k, false, true, w->tiled16, s);
   }
   if (e != cudaSuccess) {
     cudaGetLastError();
@@ -299,6 +329,13 @@ ffn_status ffn_nvfp4_weight_create(const void* codes, const void* block_scales,
   }
   *out = w;
   return FFN_OK;
+}
+
+ffn_status ffn_nvfp4_weight_create(const void* codes, const void* block_scales,
+                                   const float* global_scale, int64_t n, int64_t k,
+                                   void* stream, ffn_nvfp4_weight** out) {
+  return ffn_nvfp4_weight_create_ex(codes, block_scales, global_scale, n, k, FFN_FORMAT_ALL, stream,
+                                    out);
 }
 
 ffn_status ffn_nvfp4_weight_create_gate_up(const ffn_nvfp4_weight* gate,
@@ -310,6 +347,8 @@ ffn_status ffn_nvfp4_weight_create_gate_up(const ffn_nvfp4_weight* gate,
   if (gate->gate_up || up->gate_up) return FFN_ERR_INVALID_ARG;
   if (gate->n != up->n || gate->k != up->k) return FFN_ERR_SHAPE;
   if (gate->device != up->device) return FFN_ERR_INVALID_ARG;
+  const unsigned formats = gate->formats & up->formats;
+  if (!formats) return FFN_ERR_UNSUPPORTED;
   if (ffn_status st = check_device(gate)) return st;
   if (ffn_status st = precheck()) return st;
   const int64_t I = gate->n, H = gate->k;
@@ -318,30 +357,42 @@ ffn_status ffn_nvfp4_weight_create_gate_up(const ffn_nvfp4_weight* gate,
   w->n = 2 * I;
   w->k = H;
   w->gate_up = 1;
+  w->formats = formats;
   cudaGetDevice(&w->device);
   const cudaStream_t s = as_stream(stream);
   ffn_status st = FFN_OK;
-  const size_t cb = (size_t)I * H / 2, sb = (size_t)I * H / 16;
-  if ((st = alloc(&w->codes, 2 * cb)) || (st = alloc(&w->scales, 2 * sb)) ||
-      (st = alloc(&w->gs, 2 * sizeof(float)))) {
+  if ((st = alloc(&w->gs, 2 * sizeof(float), &w->bytes))) {
     free_weight(w);
     return st;
   }
-  cudaError_t e = cudaMemcpyAsync(w->codes, gate->codes, cb, cudaMemcpyDeviceToDevice, s);
-  if (e == cudaSuccess) e = cudaMemcpyAsync(w->codes + cb, up->codes, cb, cudaMemcpyDeviceToDevice, s);
-  if (e == cudaSuccess) e = cudaMemcpyAsync(w->scales, gate->scales, sb, cudaMemcpyDeviceToDevice, s);
-  if (e == cudaSuccess) e = cudaMemcpyAsync(w->scales + sb, up->scales, sb, cudaMemcpyDeviceToDevice, s);
-  if (e == cudaSuccess) e = cudaMemcpyAsync(w->gs, gate->gs, sizeof(float), cudaMemcpyDeviceToDevice, s);
+  cudaError_t e = cudaMemcpyAsync(w->gs, gate->gs, sizeof(float), cudaMemcpyDeviceToDevice, s);
   if (e == cudaSuccess) e = cudaMemcpyAsync(w->gs + 1, up->gs, sizeof(float), cudaMemcpyDeviceToDevice, s);
-  if (e == cudaSuccess) {
-    const size_t tb = (size_t)ffn::tc_tiled_bytes(2 * I, H, true);
-    if ((st = alloc(&w->tiled, tb)) || (st = alloc(&w->tiled16, tb))) {
+  if (e == cudaSuccess && gate->codes && up->codes) {
+    const size_t cb = (size_t)I * H / 2, sb = (size_t)I * H / 16;
+    if ((st = alloc(&w->codes, 2 * cb, &w->bytes)) || (st = alloc(&w->scales, 2 * sb, &w->bytes))) {
       free_weight(w);
       return st;
     }
-    e = ffn::launch_tile_weight(w->codes, w->scales, 2 * I, H, true, false, w->tiled, s);
-    if (e == cudaSuccess)
-      e = ffn::launch_tile_weight(w->codes, w->scales, 2 * I, H, true, true, w->tiled16, s);
+    e = cudaMemcpyAsync(w->codes, gate->codes, cb, cudaMemcpyDeviceToDevice, s);
+    if (e == cudaSuccess) e = cudaMemcpyAsync(w->codes + cb, up->codes, cb, cudaMemcpyDeviceToDevice, s);
+    if (e == cudaSuccess) e = cudaMemcpyAsync(w->scales, gate->scales, sb, cudaMemcpyDeviceToDevice, s);
+    if (e == cudaSuccess) e = cudaMemcpyAsync(w->scales + sb, up->scales, sb, cudaMemcpyDeviceToDevice, s);
+  }
+  // the fused tiles are re-tiled from the parts' tiled copies, byte for byte
+  const size_t tb = (size_t)ffn::tc_tiled_bytes(2 * I, H, true);
+  if (e == cudaSuccess && (formats & FFN_FORMAT_NVFP4_FIXED)) {
+    if ((st = alloc(&w->tiled, tb, &w->bytes))) {
+      free_weight(w);
+      return st;
+    }
+    e = ffn::launch_retile_gate_up(gate->tiled, up->tiled, I, H, w->tiled, s);
+  }
+  if (e == cudaSuccess && (formats & FFN_FORMAT_BF16)) {
+    if ((st = alloc(&w->tiled16, tb, &w->bytes))) {
+      free_weight(w);
+      return st;
+    }
+    e = ffn::launch_retile_gate_up(gate->tiled16, up->tiled16, I, H, w->tiled16, s);
   }
   if (e != cudaSuccess) {
     cudaGetLastError();
@@ -368,6 +419,13 @@ ffn_status ffn_nvfp4_weight_dims(const ffn_nvfp4_weight* w, int64_t* n, int64_t*
   return FFN_OK;
 }
 
+ffn_status ffn_nvfp4_weight_info(const ffn_nvfp4_weight* w, unsigned* formats, size_t* device_bytes) {
+  if (!w) return FFN_ERR_INVALID_ARG;
+  if (formats) *formats = w->formats;
+  if (device_bytes) *device_bytes = w->bytes;
+  return FFN_OK;
+}
+
 ffn_status ffn_nvfp4_workspace_size(int64_t m, int64_t hidden, int64_t inter,
                                     ffn_act_format format, size_t* bytes) {
   if (!bytes || m < 0) return FFN_ERR_INVALID_ARG;
@@ -391,6 +449,7 @@ ffn_status ffn_nvfp4_forward(const void* x, int64_t m, int64_t hidden, int64_t i
   if (!x || !out) return FFN_ERR_INVALID_ARG;
   if (ffn_status st = check_device(gate_up)) return st;
   if (ffn_status st = check_device(down)) return st;
+  if (!serves(gate_up, format) || !serves(down, format)) return FFN_ERR_UNSUPPORTED;
   const Carve c = carve_ffn(m, hidden, inter, format);
   if (!workspace || workspace_bytes < c.total) return FFN_ERR_WORKSPACE;
   if (!aligned16(x) || !aligned16(out) || !aligned16(workspace)) return FFN_ERR_ALIGNMENT;
@@ -488,6 +547,7 @@ ffn_status ffn_nvfp4_linear(const void* x, int64_t m, const ffn_nvfp4_weight* w,
   if (m == 0) return FFN_OK;
   if (!x || !y) return FFN_ERR_INVALID_ARG;
   if (ffn_status st = check_device(w)) return st;
+  if (!serves(w, format)) return FFN_ERR_UNSUPPORTED;
   const Carve c = carve_linear(m, w->n, w->k, format);
   if (c.total && (!workspace || workspace_bytes < c.total)) return FFN_ERR_WORKSPACE;
   if (!aligned16(x) || !aligned16(y) || (c.total && !aligned16(workspace)))

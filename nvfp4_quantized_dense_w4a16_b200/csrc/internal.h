@@ -39,6 +39,9 @@ struct TcPlan {
 
 TcPlan plan_tc(int64_t m, int64_t n, int64_t k, bool gate_up, int num_sms);
 int64_t tc_tiled_bytes(int64_t n, int64_t k, bool gate_up);
+// Fused gate+up tiles from the gate and up handles' tiles of the same kind.
+cudaError_t launch_retile_gate_up(const uint8_t* gate_tiled, const uint8_t* up_tiled, int64_t inter,
+                                  int64_t k, uint8_t* out, cudaStream_t s);
 cudaError_t launch_tile_weight(const uint8_t* codes, const uint8_t* scales, int64_t n, int64_t k,
                                bool gate_up, bool for_w4a16, uint8_t* out, cudaStream_t s);
 cudaError_t launch_tc_w4a16(const void* x, int64_t m, const TcWeight& w, bool silu_mul,

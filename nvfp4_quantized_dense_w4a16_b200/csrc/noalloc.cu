@@ -106,7 +106,7 @@ extern "C" ffn_status ffn_nvfp4_linear_noalloc(const void* x, int64_t m,
   ffn::TcWeight tw;
   bool gate_up = false;
   ffn::handle_tc_view(w, &tw, &gate_up);
-  if (gate_up) return FFN_ERR_UNSUPPORTED;
+  if (gate_up || !tw.tiled16) return FFN_ERR_UNSUPPORTED;
   if (m == 0) return FFN_OK;
   if (!x || !y) return FFN_ERR_INVALID_ARG;
   if (ffn_status st = ffn::handle_check_device(w)) return st;

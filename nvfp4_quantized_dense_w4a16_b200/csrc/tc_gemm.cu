@@ -1123,6 +1123,33 @@ __global__ void tile_weight_kernel(const uint8_t* __restrict__ codes,
   *reinterpret_cast<uint32_t*>(base + 4096 + 16 * (r & 31) + 4 * (r >> 5)) = sc;
 }
 
+// Fused gate+up tiles from two plain tiled weights [inter, k] of the same
+// kind: fused tile t, row r < 64 is gate row 64t + r, row r >= 64 is up row
+// 64t + r - 64 (zero past inter); codes and scale bytes are moved unchanged.
+__global__ void retile_gate_up_kernel(const uint8_t* __restrict__ gate, const uint8_t* __restrict__ up,
+                                      int64_t inter, int kc, int ntiles, uint8_t* __restrict__ out) {
+  const int64_t idx = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;
+  if (idx >= (int64_t)ntiles * kc * kTileRows) return;
+  const int r = (int)(idx % kTileRows);
+  const int64_t tj = idx / kTileRows;
+  const int j = (int)(tj % kc);
+  const int t = (int)(tj / kc);
+  const int64_t i = 64 * (int64_t)t + (r & 63);
+  uint4 lo = make_uint4(0, 0, 0, 0), hi = lo;
+  uint32_t sc = 0;
+  if (i < inter) {
+    const int sr = (int)(i % kTileRows);
+    const uint8_t* src = (r < 64 ? gate : up) + ((i / kTileRows) * kc + j) * kChunkBytes;
+    lo = *reinterpret_cast<const uint4*>(src + 16 * sr);
+    hi = *reinterpret_cast<const uint4*>(src + 2048 + 16 * sr);
+    sc = *reinterpret_cast<const uint32_t*>(src + 4096 + 16 * (sr & 31) + 4 * (sr >> 5));
+  }
+  uint8_t* dst = out + ((int64_t)t * kc + j) * kChunkBytes;
+  *reinterpret_cast<uint4*>(dst + 16 * r) = lo;
+  *reinterpret_cast<uint4*>(dst + 2048 + 16 * r) = hi;
+  *reinterpret_cast<uint32_t*>(dst + 4096 + 16 * (r & 31) + 4 * (r >> 5)) = sc;
+}
+
 // ----------------------------------------------------------------- host side
 
 PFN_cuTensorMapEncodeTiled_v12000 get_encode() {
@@ -1294,6 +1321,16 @@ cudaError_t launch_tile_weight(const uint8_t* codes, const uint8_t* scales, int6
   const int64_t total = (int64_t)ntiles * kc * kTileRows;
   tile_weight_kernel<<<(unsigned)((total + 255) / 256), 256, 0, s>>>(codes, scales, n, k, half, ntiles,
                                                                    kc, for_w4a16, out);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_retile_gate_up(const uint8_t* gate_tiled, const uint8_t* up_tiled, int64_t inter,
+                                  int64_t k, uint8_t* out, cudaStream_t s) {
+  const int ntiles = (int)((inter + 63) / 64);
+  const int kc = (int)((k + kChunkK - 1) / kChunkK);
+  const int64_t total = (int64_t)ntiles * kc * kTileRows;
+  retile_gate_up_kernel<<<(unsigned)((total + 255) / 256), 256, 0, s>>>(gate_tiled, up_tiled, inter, kc,
+                                                                       ntiles, out);
   return cudaGetLastError();
 }
 

@@ -20,6 +20,8 @@ HEADER = os.path.join(os.path.dirname(PKG), "include", "ffn_nvfp4.h")
 
 FFN_ACT_BF16 = 0
 FFN_ACT_NVFP4_FIXED = 1
+# weight handle formats (FFN_FORMAT_* bits)
+_WEIGHT_FORMATS = {"bf16": 1, "w4a16": 1, "nvfp4_fixed": 2, "w4a4": 2, "all": 3}
 _FORMATS = {"bf16": FFN_ACT_BF16, "w4a16": FFN_ACT_BF16,
             "nvfp4_fixed": FFN_ACT_NVFP4_FIXED, "w4a4": FFN_ACT_NVFP4_FIXED}
 
@@ -59,6 +61,8 @@ def _load() -> ctypes.CDLL:
         "ffn_nvfp4_quantize_weights": (ctypes.c_int, [vp, i64, i64, vp, vp, vp, vp]),
         "ffn_nvfp4_quantize_activations": (ctypes.c_int, [vp, i64, i64, vp, vp, vp]),
         "ffn_nvfp4_weight_create": (ctypes.c_int, [vp, vp, vp, i64, i64, vp, P(vp)]),
+        "ffn_nvfp4_weight_create_ex": (ctypes.c_int, [vp, vp, vp, i64, i64, ctypes.c_uint, vp, P(vp)]),
+        "ffn_nvfp4_weight_info": (ctypes.c_int, [vp, P(ctypes.c_uint), P(sz)]),
         "ffn_nvfp4_weight_create_gate_up": (ctypes.c_int, [vp, vp, vp, P(vp)]),
         "ffn_nvfp4_weight_destroy": (ctypes.c_int, [vp]),
         "ffn_nvfp4_weight_dims": (ctypes.c_int, [vp, P(i64), P(i64), P(ctypes.c_int)]),
@@ -172,6 +176,9 @@ class Weight:
         _check("ffn_nvfp4_weight_dims", lib.ffn_nvfp4_weight_dims(
             self._h, ctypes.byref(n), ctypes.byref(k), ctypes.byref(gu)))
         self.n, self.k, self.is_gate_up = n.value, k.value, bool(gu.value)
+        f, b = ctypes.c_uint(), ctypes.c_size_t()
+        _check("ffn_nvfp4_weight_info", lib.ffn_nvfp4_weight_info(self._h, ctypes.byref(f), ctypes.byref(b)))
+        self.formats, self.device_bytes = f.value, b.value
 
     @property
     def handle(self):
@@ -190,15 +197,18 @@ class Weight:
 
 
 def ffn_nvfp4_weight_create(codes: torch.Tensor, block_scales: torch.Tensor,
-                            global_scale: torch.Tensor, stream=None) -> Weight:
+                            global_scale: torch.Tensor, stream=None, formats="all") -> Weight:
+    """Handle for the activation formats 'bf16', 'nvfp4_fixed' or 'all'
+    (one tiled copy of the weight per format)."""
     _need(codes, "codes", torch.uint8)
     n, half_k = codes.shape
     k = 2 * half_k
     _need(block_scales, "block_scales", torch.uint8, (n, k // 16))
     _need(global_scale, "global_scale", torch.float32, (1,))
     h = ctypes.c_void_p()
-    _check("ffn_nvfp4_weight_create", lib.ffn_nvfp4_weight_create(
-        _ptr(codes), _ptr(block_scales), _ptr(global_scale), n, k, _stream(stream), ctypes.byref(h)))
+    f = formats if isinstance(formats, int) else _WEIGHT_FORMATS[formats]
+    _check("ffn_nvfp4_weight_create_ex", lib.ffn_nvfp4_weight_create_ex(
+        _ptr(codes), _ptr(block_scales), _ptr(global_scale), n, k, f, _stream(stream), ctypes.byref(h)))
     return Weight(h)
 
 

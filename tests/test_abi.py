@@ -95,3 +95,13 @@ def test_projection_plan_m_dispatch(native):
     assert L.ffn_nvfp4_projection_plan(4, 129, 64, 0, 1, ctypes.byref(p)) == 2    # odd gate+up n
     assert L.ffn_nvfp4_projection_plan(-1, 128, 64, 0, 0, ctypes.byref(p)) == 1
     assert L.ffn_nvfp4_projection_plan(4, 128, 64, 0, 0, None) == 1
+
+
+def test_weight_create_ex_rejects_bad_formats(native):
+    L = native.lib
+    fake = ctypes.c_void_p(256)
+    h = ctypes.c_void_p()
+    assert L.ffn_nvfp4_weight_create_ex(fake, fake, fake, 4, 64, 0, None, ctypes.byref(h)) == 1
+    assert L.ffn_nvfp4_weight_create_ex(fake, fake, fake, 4, 64, 4, None, ctypes.byref(h)) == 1
+    assert L.ffn_nvfp4_weight_create_ex(fake, fake, fake, 4, 40, 1, None, ctypes.byref(h)) == 2
+    assert L.ffn_nvfp4_weight_info(None, None, None) == 1

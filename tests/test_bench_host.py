@@ -40,7 +40,7 @@ def fake_native(calls):
     counter = iter(range(10**6))
     return types.SimpleNamespace(
         ffn_nvfp4_quantize_weights=lambda w: (w, w, w),
-        ffn_nvfp4_weight_create=lambda c, s, g: ("w", next(counter)),
+        ffn_nvfp4_weight_create=lambda c, s, g, formats="all": ("w", next(counter)),
         ffn_nvfp4_weight_create_gate_up=lambda g, u: ("gu", g, u),
         ffn_nvfp4_workspace_size=lambda m, H, I, f: 1024,
         ffn_nvfp4_forward=lambda x, gu, d, f, out=None, workspace=None: calls.append((gu, d)))

@@ -213,3 +213,30 @@ def test_cuda_core_paths_match_oracle_in_subprocess(native, env, fmt):
 def test_device_error_word_is_clear(native, tiny):
     tiny.forward("bf16")
     assert native.ffn_nvfp4_device_error(clear=False) == 0
+
+
+def test_handles_hold_one_tiled_copy_per_format(native):
+    # a bf16-only handle holds ~0.5625 B per weight (tiles pad n to 128 rows
+    # and k to 64); the fused gate+up serves what both parts serve; a format
+    # the handle was not built for is refused, not silently recomputed
+    n, k = 512, 1024
+    bits = synth.random_bf16((n, k), 7, std=0.02)
+    c, s, g = native.ffn_nvfp4_quantize_weights(to_dev_bf16(bits))
+    w16 = native.ffn_nvfp4_weight_create(c, s, g, formats="bf16")
+    w4 = native.ffn_nvfp4_weight_create(c, s, g, formats="nvfp4_fixed")
+    wall = native.ffn_nvfp4_weight_create(c, s, g)
+    assert w16.formats == 1 and w4.formats == 2 and wall.formats == 3
+    assert w16.device_bytes <= 0.6 * n * k and w4.device_bytes <= 0.6 * n * k
+    assert wall.device_bytes <= 1.2 * n * k
+    x = to_dev_bf16(synth.random_bf16((3, k), 8))
+    ref = O.round_to_bf16(O.project_w4a16(synth.bf16_bits_to_f32(synth.f32_to_bf16_bits(
+        x.float().cpu().numpy())).astype(np.float64), *oracle_weight(bits)))
+    assert_close(bf16_to_f64(native.ffn_nvfp4_linear(x, w16, "bf16")), ref)
+    with pytest.raises(native.FfnError) as e:
+        native.ffn_nvfp4_linear(x, w16, "nvfp4_fixed")
+    assert e.value.status_name == "FFN_ERR_UNSUPPORTED"
+    gu = native.ffn_nvfp4_weight_create_gate_up(w16, wall)
+    assert gu.formats == 1 and gu.device_bytes <= 0.6 * 2 * n * k
+    with pytest.raises(native.FfnError) as e:
+        native.ffn_nvfp4_weight_create_gate_up(w16, w4)
+    assert e.value.status_name == "FFN_ERR_UNSUPPORTED"
