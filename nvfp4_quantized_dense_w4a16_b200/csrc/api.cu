@@ -105,6 +105,17 @@ Path w4a4_path() {
   return p;
 }
 
+// The fixed format quantises h inside the gate+up epilogue when that
+// projection runs unsplit; FFN_NVFP4_W4A4_FUSE_HQ=0 keeps the separate
+// quantiser launch (read once; for comparisons).
+bool w4a4_fuse_hq() {
+  static const bool on = [] {
+    const char* v = getenv("FFN_NVFP4_W4A4_FUSE_HQ");
+    return !(v && !strcmp(v, "0"));
+  }();
+  return on;
+}
+
 // The canonical NVFP4 copy is read only by the CUDA-core arms, which run
 // only when forced by environment; otherwise handles keep just the tiled
 // copies their formats need (0.5625 B per weight and format, plus tile padding).
@@ -472,8 +483,14 @@ ffn_status ffn_nvfp4_forward(const void* x, int64_t m, int64_t hidden, int64_t i
     uint8_t *xq = ws + c.xq_c, *xs = ws + c.xq_s, *hq = ws + c.hq_c, *hs = ws + c.hq_s;
     void* part = ws + c.part;
     e = ffn::launch_quantize_activations_blocked(x, m, hidden, xq, xs, s);
-    if (e == cudaSuccess) e = ffn::launch_tc_w4a4(xq, xs, m, gate_up->tc(), true, c.gate_up, h, part, s);
-    if (e == cudaSuccess) e = ffn::launch_quantize_activations_blocked(h, m, inter, hq, hs, s);
+    if (c.gate_up.splits == 1 && w4a4_fuse_hq()) {
+      // h is quantised in the gate+up epilogue, bit for bit as the quantiser would
+      if (e == cudaSuccess)
+        e = ffn::launch_tc_w4a4(xq, xs, m, gate_up->tc(), true, c.gate_up, h, part, s, hq, hs);
+    } else {
+      if (e == cudaSuccess) e = ffn::launch_tc_w4a4(xq, xs, m, gate_up->tc(), true, c.gate_up, h, part, s);
+      if (e == cudaSuccess) e = ffn::launch_quantize_activations_blocked(h, m, inter, hq, hs, s);
+    }
     if (e == cudaSuccess) e = ffn::launch_tc_w4a4(hq, hs, m, down->tc(), false, c.down, out, part, s);
   } else {
     uint8_t *xq = ws + c.xq_c, *xs = ws + c.xq_s, *hq = ws + c.hq_c, *hs = ws + c.hq_s;
@@ -513,7 +530,8 @@ ffn_status ffn_nvfp4_projection_plan(int64_t m, int64_t n, int64_t k, ffn_act_fo
     *out = ffn_projection_plan{FFN_KERNEL_GEMV_W4A16, 0, 1, ffn::gemv_grid(ncols)};
   } else if (w4a4_path() == Path::kTc) {
     const ffn::TcPlan p = ffn::plan_w4a4(m, n, k, gate_up != 0, num_sms());
-    *out = ffn_projection_plan{FFN_KERNEL_TC_W4A4, p.bn, p.splits, p.xtiles * p.wtiles * p.splits};
+    const int xt = ffn::w4a4_tiles_per_cta(p.xtiles);
+    *out = ffn_projection_plan{FFN_KERNEL_TC_W4A4, p.bn, p.splits, (p.xtiles + xt - 1) / xt * p.wtiles * p.splits};
   } else {
     *out = ffn_projection_plan{FFN_KERNEL_GEMV_W4A4, 0, 1, ffn::gemv_grid(ncols)};
   }

@@ -38,6 +38,28 @@ __device__ __forceinline__ float e4m3_decode(uint32_t b) {
   return __uint_as_float(((e + 120u) << 23) | (m << 20));
 }
 
+// Codes of one 16-element block under the decoded scale sdec (fp32 IEEE
+// division per element); all zero when `zero`.  Element i in nibble i.
+__device__ __forceinline__ uint2 e2m1_encode_block16(const float (&v)[16], float sdec, bool zero) {
+  uint32_t lo = 0, hi = 0;
+  if (!zero) {
+#pragma unroll
+    for (int i = 0; i < 8; ++i) lo |= e2m1_encode(__fdiv_rn(v[i], sdec)) << (4 * i);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) hi |= e2m1_encode(__fdiv_rn(v[8 + i], sdec)) << (4 * i);
+  }
+  return make_uint2(lo, hi);
+}
+
+// Scale-factor byte position of (row r, 16-element block kb) in the blocked
+// layout the block-scaled FP4 kernel copies to TMEM: one 512-byte block per
+// 128 rows and 64 elements (kc such blocks per 128 rows), row r's four scales
+// at 16 * (r % 32) + 4 * ((r % 128) / 32).
+__host__ __device__ __forceinline__ int64_t sf_blocked_offset(int64_t r, int64_t kb, int64_t kc) {
+  const int rr = (int)(r & 127);
+  return ((r >> 7) * kc + kb / 4) * 512 + 16 * (rr & 31) + 4 * (rr >> 5) + (kb & 3);
+}
+
 // E2M1 magnitude of a 3-bit index as fp32 (exact).
 __device__ __forceinline__ float e2m1_mag(uint32_t i) {
   // 0, .5, 1, 1.5, 2, 3, 4, 6 = (i < 2 ? 0.5*i : 2^(e-1)*(1+m/2)) with e = i>>1

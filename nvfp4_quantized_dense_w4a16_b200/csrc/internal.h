@@ -64,10 +64,17 @@ cudaError_t launch_persist_ffn(const void* x, int64_t m, const TcWeight& gate_up
 // Fixed-format (W4A4) projection on the block-scaled FP4 tensor core.  The
 // plan depends on (n, k) only (plus the number of 128-row activation tiles).
 TcPlan plan_w4a4(int64_t m, int64_t n, int64_t k, bool gate_up, int num_sms);
+// Activation tiles of 128 rows each CTA of the W4A4 kernel multiplies with
+// one weight stage (1 or 2; changes no result bit).
+int w4a4_tiles_per_cta(int xtiles);
 size_t w4a4_sf_block_bytes(int64_t m, int64_t k);
+// With silu_mul, no K split and hq_codes/hq_sf given, the epilogue writes the
+// per-row NVFP4 quantisation of h (codes [m, n/4], blocked scales) instead
+// of h itself.
 cudaError_t launch_tc_w4a4(const uint8_t* xcodes, const uint8_t* xsf_blocks, int64_t m,
                            const TcWeight& w, bool silu_mul, const TcPlan& p, void* y,
-                           void* partials, cudaStream_t s);
+                           void* partials, cudaStream_t s, uint8_t* hq_codes = nullptr,
+                           uint8_t* hq_sf = nullptr);
 // Activation quantiser that also writes the scales as 512-byte blocks per
 // 128 rows and 64 elements (the W4A4 kernel's scale-factor layout).
 cudaError_t launch_quantize_activations_blocked(const void* x, int64_t m, int64_t k, void* codes,

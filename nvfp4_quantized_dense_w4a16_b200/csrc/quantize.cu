@@ -10,6 +10,7 @@
 // s = E4M3(block amax / 6), code = E2M1(x / E4M3value(s)).
 #include "common.cuh"
 #include "internal.h"
+#include "launch.cuh"
 #include "profile.h"
 
 namespace ffn {
@@ -36,14 +37,7 @@ __device__ __forceinline__ void load_block16(const uint16_t* src, Block16& b) {
 
 // Encode a block whose decoded scale is sdec (0 => all codes 0).
 __device__ __forceinline__ uint2 encode_block16(const Block16& b, float sdec, bool zero) {
-  uint32_t lo = 0, hi = 0;
-  if (!zero) {
-#pragma unroll
-    for (int i = 0; i < 8; ++i) lo |= e2m1_encode(__fdiv_rn(b.v[i], sdec)) << (4 * i);
-#pragma unroll
-    for (int i = 0; i < 8; ++i) hi |= e2m1_encode(__fdiv_rn(b.v[8 + i], sdec)) << (4 * i);
-  }
-  return make_uint2(lo, hi);
+  return e2m1_encode_block16(b.v, sdec, zero);
 }
 
 __global__ void amax_bf16_kernel(const uint16_t* __restrict__ w, int64_t count8,
@@ -112,6 +106,9 @@ __global__ void quantize_act_blocked_kernel(const uint16_t* __restrict__ x, int6
                                             int64_t kb_per_row, int kc,
                                             uint8_t* __restrict__ codes,
                                             uint8_t* __restrict__ sf_blocks) {
+  // x comes from the previous kernel (with programmatic dependent launch)
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   const int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;
   if (i >= nblocks) return;
   Block16 b;
@@ -119,9 +116,7 @@ __global__ void quantize_act_blocked_kernel(const uint16_t* __restrict__ x, int6
   const uint32_t s8 = e4m3_encode_satfinite(__fdiv_rn(b.amax, 6.0f));
   const uint2 c = encode_block16(b, e4m3_decode(s8), s8 == 0);
   reinterpret_cast<uint2*>(codes)[i] = c;
-  const int64_t r = i / kb_per_row, kb = i % kb_per_row;
-  const int rr = (int)(r & 127);
-  sf_blocks[((r >> 7) * kc + kb / 4) * 512 + 16 * (rr & 31) + 4 * (rr >> 5) + (kb & 3)] = (uint8_t)s8;
+  sf_blocks[sf_blocked_offset(i / kb_per_row, i % kb_per_row, kc)] = (uint8_t)s8;
 }
 
 cudaError_t launch_quantize_activations_blocked(const void* x, int64_t m, int64_t k, void* codes,
@@ -131,9 +126,9 @@ cudaError_t launch_quantize_activations_blocked(const void* x, int64_t m, int64_
   const int threads = 256;
   const int kc = (int)((k + 63) / 64);
   ProfScope prof(s, "quantize_activations");
-  quantize_act_blocked_kernel<<<(unsigned)((nblocks + threads - 1) / threads), threads, 0, s>>>(
-      (const uint16_t*)x, nblocks, k / 16, kc, (uint8_t*)codes, (uint8_t*)sf_blocks);
-  return cudaGetLastError();
+  return launch_pdl(quantize_act_blocked_kernel, dim3((unsigned)((nblocks + threads - 1) / threads)),
+                    dim3(threads), 0, s, (const uint16_t*)x, nblocks, (int64_t)(k / 16), kc,
+                    (uint8_t*)codes, (uint8_t*)sf_blocks);
 }
 
 cudaError_t launch_quantize_weights(const void* w, int64_t n, int64_t k, void* codes,

@@ -31,12 +31,14 @@
 // Pipelines are mbarrier-driven; every wait is bounded and, on timeout, sets
 // a device error bit and lets the CTA free its TMEM and exit.
 #include <cudaTypedefs.h>
+#include <stdlib.h>
 
 #include <mutex>
 #include <utility>
 
 #include "common.cuh"
 #include "internal.h"
+#include "launch.cuh"
 #include "profile.h"
 #include "sm100.cuh"
 
@@ -52,7 +54,7 @@ constexpr int kChunkK = 64;        // K elements per stage
 constexpr int kTileRows = 128;     // weight rows per tile = TMEM lanes
 constexpr int kChunkBytes = 4608;  // 128 x (16 + 16 + 4) bytes
 
-enum : int { kEpiStore = 0, kEpiSiluMul = 1, kEpiPartial = 2 };
+enum : int { kEpiStore = 0, kEpiSiluMul = 1, kEpiPartial = 2, kEpiSiluMulQuant = 3 };
 
 // Pipeline shape.  The K range of a CTA is a sequence of 64-element chunks,
 // grouped into units of UA consecutive chunks; unit u is dequantised by
@@ -123,6 +125,12 @@ struct TcArgs {
   // stale data, which only reaches accumulator columns of rows >= m -- MMA
   // columns are independent and those columns are never stored.
   int x_box_rows;
+  // kEpiSiluMulQuant: h is quantised per row to NVFP4 as it is produced
+  // (the fixed format's input of the down projection): codes [m, n_out/2]
+  // and scale bytes in the blocked layout with q_kc 64-element chunks per row.
+  uint8_t* q_codes = nullptr;
+  uint8_t* q_sf = nullptr;
+  int q_kc = 0;
 };
 
 __device__ __forceinline__ uint32_t bmul2(uint32_t a, uint32_t b) {
@@ -244,8 +252,11 @@ __device__ __forceinline__ bool wait_drain(uint64_t* bar, uint32_t parity) {
 // y = bf16(gs * acc); kEpiSiluMul (rows 0-63 gate, 64-127 the matching up rows)
 // writes h = bf16(silu(bf16(gs_g * g)) * bf16(gs_u * u)); kEpiPartial writes
 // fp32 split-K partials (gs_mul: a power of two folded into the operands,
-// applied with gs).  Stores are staged through shared memory (ebuf,
-// 16 KB per warpgroup) so that global writes are 16-byte and row-contiguous.
+// applied with gs); kEpiSiluMulQuant computes h like kEpiSiluMul and writes
+// its per-row NVFP4 quantisation instead (per 16-block: s = E4M3(amax/6),
+// codes = E2M1(h / s), the same arithmetic as the activation quantiser).
+// Stores are staged through shared memory (ebuf, 16 KB per warpgroup) so that
+// global writes are 16-byte and row-contiguous.
 template <int BN, int EPI, int NG, int NACC = 1>
 __device__ __forceinline__ void epilogue_tile(const TcArgs& a, uint32_t tmem, int q, int lane,
                                               int g, uint8_t* ebuf, int xtile, int wtile,
@@ -316,12 +327,31 @@ __device__ __forceinline__ void epilogue_tile(const TcArgs& a, uint32_t tmem, in
       }
       named_bar_sync(1 + g, 128);
       const int n0 = 64 * wtile;
-      for (int idx = et; idx < 32 * 8; idx += 128) {
-        const int j = idx >> 3, ch = idx & 7;
-        const int r = r0 + j, n = n0 + 8 * ch;
-        if (j < jmax && r < a.m && n < a.n_out)
-          *reinterpret_cast<uint4*>(static_cast<uint16_t*>(a.out) + (size_t)r * a.ldo + n) =
-              *reinterpret_cast<const uint4*>(Hs + j * 64 + 8 * ch);
+      if (EPI == kEpiSiluMulQuant) {
+        // thread et: activation row j = et / 4 of this chunk, 16-block b = et % 4
+        const int j = et >> 2, b = et & 3;
+        const int r = r0 + j, n = n0 + 16 * b;
+        if (j < jmax && r < a.m && n < a.n_out) {
+          float hv[16];
+          float amax = 0.0f;
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            hv[i] = bf16_bits_to_float(Hs[j * 64 + 16 * b + i]);
+            amax = fmaxf(amax, fabsf(hv[i]));
+          }
+          const uint32_t s8 = e4m3_encode_satfinite(__fdiv_rn(amax, 6.0f));
+          const uint2 c = e2m1_encode_block16(hv, e4m3_decode(s8), s8 == 0);
+          *reinterpret_cast<uint2*>(a.q_codes + (size_t)r * (a.n_out / 2) + n / 2) = c;
+          a.q_sf[sf_blocked_offset(r, n / 16, a.q_kc)] = (uint8_t)s8;
+        }
+      } else {
+        for (int idx = et; idx < 32 * 8; idx += 128) {
+          const int j = idx >> 3, ch = idx & 7;
+          const int r = r0 + j, n = n0 + 8 * ch;
+          if (j < jmax && r < a.m && n < a.n_out)
+            *reinterpret_cast<uint4*>(static_cast<uint16_t*>(a.out) + (size_t)r * a.ldo + n) =
+                *reinterpret_cast<const uint4*>(Hs + j * 64 + 8 * ch);
+        }
       }
       named_bar_sync(1 + g, 128);
     }
@@ -917,54 +947,63 @@ tc_w4a16_persistent_kernel(const __grid_constant__ CUtensorMap xmap, const PArgs
 // ---------------------------------------------------------------------------
 constexpr int kW4BN = 128;        // activation rows per tile (fixed)
 constexpr int kW4Chunks = 4;      // 64-element chunks per stage
-constexpr int kW4Stages = 5;
 
+// XT activation tiles per CTA share each weight stage (one MMA per tile and
+// chunk, an accumulator each): the weights cross L2 once per XT tiles.  Every
+// activation row is still the N column of a 128-row MMA with the same K
+// order, so XT changes no result bit.
+template <int XT>
 struct W4Cfg {
+  static constexpr int kStages = XT == 1 ? 5 : 4;
   static constexpr int kWBytes = kW4Chunks * kChunkBytes;  // 18432
   static constexpr int kXBytes = kW4BN * 128;              // 16384 (128 rows x 256 elements)
   static constexpr int kSfbBytes = kW4Chunks * 512;        // 2048
-  static constexpr int kStageBytes = kWBytes + kXBytes + kSfbBytes;  // 36864 = 36 KB
-  static constexpr int kSmemEpi = kW4Stages * kStageBytes;
-  static constexpr int kSmemBar = kSmemEpi + 16384;
-  static constexpr int kSmemBytes = kSmemBar + (2 * kW4Stages + 1) * 8 + 16;
+  static constexpr int kStageBytes = kWBytes + XT * (kXBytes + kSfbBytes);
+  static constexpr int kSmemEpi = kStages * kStageBytes;
+  static constexpr int kSmemBar = kSmemEpi + (kSmemEpi >= 16384 ? 0 : 16384);
+  static constexpr int kSmemBytes = kSmemBar + (2 * kStages + 1) * 8 + 16;
   static constexpr int kSmemAlloc = kSmemBytes + 1024;
-  static constexpr int kSfaCol = kW4BN;                                  // TMEM columns
-  static constexpr int kSfbCol = kSfaCol + 4 * kW4Chunks * kW4Stages;
+  static constexpr int kSfaCol = XT * kW4BN;                             // TMEM columns
+  static constexpr int kSfbCol = kSfaCol + 4 * kW4Chunks * kStages;     // + 4 * kW4Chunks * kStages per tile
   static constexpr int kTmemCols = 512;
-  static_assert(kSfbCol + 4 * kW4Chunks * kW4Stages <= kTmemCols, "TMEM budget");
+  static_assert(kSfbCol + XT * 4 * kW4Chunks * kStages <= kTmemCols, "TMEM budget");
   static_assert(kStageBytes % 1024 == 0, "stage alignment");
   static_assert(kSmemAlloc <= 232448, "shared memory budget");
+  static_assert(kSmemEpi >= 16384, "the epilogue buffer aliases the rings");
 };
 
 struct W4Args {
   TcArgs t;
   const uint8_t* sfb;   // activation scale blocks [ceil(m/128)][kc][512]
+  int xtiles;           // activation tiles of 128 rows
 };
 
-template <int EPI>
+template <int EPI, int XT>
 __global__ void __launch_bounds__(256, 1)
 tc_w4a4_kernel(const __grid_constant__ CUtensorMap xmap, const W4Args w4) {
-  using C = W4Cfg;
+  using C = W4Cfg<XT>;
+  constexpr int S = C::kStages;
   const TcArgs& a = w4.t;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
   uint8_t* epi = smem;  // aliases the rings; used only after the last MMA
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::kSmemBar);
-  uint64_t* empty = full + kW4Stages;
-  uint64_t* accum = empty + kW4Stages;
+  uint64_t* empty = full + S;
+  uint64_t* accum = empty + S;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(accum + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   int* err = &g_ffn_device_error;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int xtile = blockIdx.x, wtile = blockIdx.y;
+  const int xt0 = blockIdx.x * XT, wtile = blockIdx.y;
+  const int nxt = min(XT, w4.xtiles - xt0);                        // activation tiles of this CTA
   const int kc0 = blockIdx.z * a.kc_per_split;
   const int nk = min(a.kc_total, kc0 + a.kc_per_split) - kc0;     // chunks of this CTA
   const int nstage = (nk + kW4Chunks - 1) / kW4Chunks;
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < kW4Stages; ++s) {
+    for (int s = 0; s < S; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
     }
@@ -981,44 +1020,66 @@ tc_w4a4_kernel(const __grid_constant__ CUtensorMap xmap, const W4Args w4) {
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  griddep_launch_dependents();
 
   if (warp == 0) {
     if (lane == 0) {
       const uint8_t* wsrc = a.wt + ((size_t)wtile * a.kc_total + kc0) * kChunkBytes;
-      const uint8_t* ssrc = w4.sfb + ((size_t)xtile * a.kc_total + kc0) * 512;
+      auto stage_bytes = [&](int i) {
+        const int nch = min(kW4Chunks, nk - kW4Chunks * i);
+        return (uint32_t)(nch * kChunkBytes + nxt * (nch * 512 + a.x_box_rows * 128));
+      };
+      // the first ring's weights do not depend on the previous kernel: stream
+      // them before waiting for it (the activation codes and scales do)
+      const int pre = min(nstage, S);
+      for (int i = 0; i < pre; ++i) {
+        const int nch = min(kW4Chunks, nk - kW4Chunks * i);
+        mbar_arrive_expect_tx(&full[i], stage_bytes(i));
+        bulk_load(smem + i * C::kStageBytes, wsrc + (size_t)kW4Chunks * i * kChunkBytes, nch * kChunkBytes,
+                  &full[i]);
+      }
+      griddep_wait();
       int issued = 0;
       for (int i = 0; i < nstage; ++i) {
-        const int s = i % kW4Stages;
+        const int s = i % S;
         const int nch = min(kW4Chunks, nk - kW4Chunks * i);
-        if (i >= kW4Stages && !mbar_wait(&empty[s], ((i / kW4Stages) - 1) & 1, abort_flag, err, 1)) break;
         uint8_t* st = smem + s * C::kStageBytes;
-        mbar_arrive_expect_tx(&full[s], nch * (kChunkBytes + 512) + a.x_box_rows * 128);
-        bulk_load(st, wsrc + (size_t)kW4Chunks * i * kChunkBytes, nch * kChunkBytes, &full[s]);
-        tma_load_2d(st + C::kWBytes, &xmap, 32 * (kc0 + kW4Chunks * i), xtile * kW4BN, &full[s]);
-        bulk_load(st + C::kWBytes + C::kXBytes, ssrc + (size_t)kW4Chunks * i * 512, nch * 512, &full[s]);
+        if (i >= pre) {
+          if (!mbar_wait(&empty[s], ((i / S) - 1) & 1, abort_flag, err, 1)) break;
+          mbar_arrive_expect_tx(&full[s], stage_bytes(i));
+          bulk_load(st, wsrc + (size_t)kW4Chunks * i * kChunkBytes, nch * kChunkBytes, &full[s]);
+        }
+        for (int t = 0; t < nxt; ++t) {
+          uint8_t* xt = st + C::kWBytes + t * (C::kXBytes + C::kSfbBytes);
+          tma_load_2d(xt, &xmap, 32 * (kc0 + kW4Chunks * i), (xt0 + t) * kW4BN, &full[s]);
+          bulk_load(xt + C::kXBytes,
+                    w4.sfb + ((size_t)(xt0 + t) * a.kc_total + kc0 + kW4Chunks * i) * 512, nch * 512, &full[s]);
+        }
         ++issued;
       }
-      for (int i = max(0, issued - kW4Stages); i < issued; ++i)
-        wait_drain(&full[i % kW4Stages], (i / kW4Stages) & 1);
+      for (int i = max(0, issued - S); i < issued; ++i) wait_drain(&full[i % S], (i / S) & 1);
     }
   } else if (warp == 1) {
     if (lane == 0) {
       const uint32_t idesc = idesc_mxf4nvf4(kTileRows, kW4BN);
       for (int i = 0; i < nstage; ++i) {
-        const int s = i % kW4Stages;
+        const int s = i % S;
         const int nch = min(kW4Chunks, nk - kW4Chunks * i);
-        if (!mbar_wait(&full[s], (i / kW4Stages) & 1, abort_flag, err, 2)) break;
+        if (!mbar_wait(&full[s], (i / S) & 1, abort_flag, err, 2)) break;
         tc_fence_after();
         const uint8_t* st = smem + s * C::kStageBytes;
-        const uint64_t b_base = smem_desc_sw128(smem_u32(st + C::kWBytes));
         for (int c = 0; c < nch; ++c) {
           const uint32_t slot = 4 * (s * kW4Chunks + c);
           const uint8_t* wc = st + c * kChunkBytes;
           tmem_cp_32x128b_x4(tmem + C::kSfaCol + slot, smem_desc_interleave(smem_u32(wc + 4096), 16, 128));
-          tmem_cp_32x128b_x4(tmem + C::kSfbCol + slot,
-                             smem_desc_interleave(smem_u32(st + C::kWBytes + C::kXBytes + 512 * c), 16, 128));
-          mma_mxf4nvf4(tmem, smem_desc_interleave(smem_u32(wc), 2048, 128), b_base + 2 * c, idesc,
-                       tmem + C::kSfaCol + slot, tmem + C::kSfbCol + slot, (i | c) != 0 ? 1u : 0u);
+          const uint64_t a_desc = smem_desc_interleave(smem_u32(wc), 2048, 128);
+          for (int t = 0; t < nxt; ++t) {
+            const uint8_t* xt = st + C::kWBytes + t * (C::kXBytes + C::kSfbBytes);
+            const uint32_t sfb = tmem + C::kSfbCol + t * 4 * kW4Chunks * S + slot;
+            tmem_cp_32x128b_x4(sfb, smem_desc_interleave(smem_u32(xt + C::kXBytes + 512 * c), 16, 128));
+            mma_mxf4nvf4(tmem + t * kW4BN, a_desc, smem_desc_sw128(smem_u32(xt)) + 2 * c, idesc,
+                         tmem + C::kSfaCol + slot, sfb, (i | c) != 0 ? 1u : 0u);
+          }
         }
         mma_commit(&empty[s]);
       }
@@ -1028,7 +1089,10 @@ tc_w4a4_kernel(const __grid_constant__ CUtensorMap xmap, const W4Args w4) {
     const int q = warp & 3;
     const bool done = __all_sync(0xffffffffu, wait_drain(accum, 0));
     tc_fence_after();
-    if (done && !*abort_flag) epilogue_tile<kW4BN, EPI, 1>(a, tmem, q, lane, 0, epi, xtile, wtile);
+    griddep_wait();  // the previous kernel may still read this kernel's outputs
+    if (done && !*abort_flag)
+      for (int t = 0; t < nxt; ++t)
+        epilogue_tile<kW4BN, EPI, 1>(a, tmem + t * kW4BN, q, lane, 0, epi, xt0 + t, wtile);
   }
   tc_fence_before();
   __syncthreads();
@@ -1178,26 +1242,6 @@ bool make_x_map(CUtensorMap* map, const void* x, int64_t m, int64_t k, int box_r
              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// Launch with programmatic stream serialisation: the kernel may begin while
-// the previous kernel in the stream finishes (the kernels wait for its
-// results with griddep_wait).  Not while per-kernel timing is recorded: an
-// event between two kernels must not let the second start early.
-template <typename... KArgs, typename... Args>
-cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
-                       Args&&... args) {
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = grid;
-  cfg.blockDim = block;
-  cfg.dynamicSmemBytes = smem;
-  cfg.stream = s;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = profiling() ? 0 : 1;
-  return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
-}
-
 template <int BN, int SXS, int XC, int SWS, int SA, int DQG, int UA, int NI, bool DQX, int EPI>
 cudaError_t launch_cfg(const CUtensorMap& map, const TcArgs& a, dim3 grid, cudaStream_t s) {
   using C = TcCfg<BN, SXS, XC, SWS, SA, DQG, UA, NI, DQX>;
@@ -1209,8 +1253,29 @@ cudaError_t launch_cfg(const CUtensorMap& map, const TcArgs& a, dim3 grid, cudaS
   return launch_pdl(kern, grid, dim3(C::kThreads), C::kSmemAlloc, s, map, a);
 }
 
+// Pipeline variant of the 256-row tile (read once from FFN_NVFP4_WIDE_CFG;
+// 0 = the default): alternatives kept selectable so that they can be timed
+// against each other on the same build.
+int wide_variant() {
+  static const int v = [] {
+    const char* e = getenv("FFN_NVFP4_WIDE_CFG");
+    return e ? atoi(e) : 0;
+  }();
+  return v;
+}
+
 template <int EPI>
 cudaError_t launch_bn(int bn, const CUtensorMap& map, const TcArgs& a, dim3 grid, cudaStream_t s) {
+  if (bn == 256) switch (wide_variant()) {
+    // three dequant warpgroups, 3 two-chunk TMEM slots, the MMA thread waits
+    // for the activation stages itself
+    case 1: return launch_cfg<256, 2, 2, 3, 3, 3, 2, 1, false, EPI>(map, a, grid, s);
+    // three dequant warpgroups, 6 one-chunk TMEM slots
+    case 2: return launch_cfg<256, 2, 2, 6, 6, 3, 1, 1, false, EPI>(map, a, grid, s);
+    // the default with a deeper weight ring
+    case 3: return launch_cfg<256, 2, 2, 5, 4, 2, 2, 1, true, EPI>(map, a, grid, s);
+    default: break;
+  }
   switch (bn) {
     // BN, activation stages, chunks per activation stage, weight stages
     // (rounds), TMEM A slots (units), dequant warpgroups, chunks per unit, MMA
@@ -1397,6 +1462,8 @@ cudaError_t launch_tc_w4a16(const void* x, int64_t m, const TcWeight& w, bool si
                   : launch_bn<kEpiStore>(p.bn, map, a, grid, s);
 }
 
+int w4a4_tiles_per_cta(int xtiles) { return xtiles >= 2 ? 2 : 1; }
+
 TcPlan plan_w4a4(int64_t m, int64_t n, int64_t k, bool gate_up, int num_sms) {
   // Everything but the number of activation tiles depends on (n, k) only.
   TcPlan p;
@@ -1422,7 +1489,7 @@ size_t w4a4_sf_block_bytes(int64_t m, int64_t k) {
 
 cudaError_t launch_tc_w4a4(const uint8_t* xcodes, const uint8_t* xsf_blocks, int64_t m,
                            const TcWeight& w, bool silu_mul, const TcPlan& p, void* y,
-                           void* partials, cudaStream_t s) {
+                           void* partials, cudaStream_t s, uint8_t* hq_codes, uint8_t* hq_sf) {
   auto enc = get_encode();
   if (!enc) return cudaErrorInvalidValue;
   CUtensorMap map;
@@ -1437,6 +1504,7 @@ cudaError_t launch_tc_w4a4(const uint8_t* xcodes, const uint8_t* xsf_blocks, int
       return cudaErrorInvalidValue;
   }
   W4Args a;
+  a.xtiles = p.xtiles;
   a.t.x_box_rows = (int)(m < kW4BN ? m : kW4BN);
   a.t.wt = w.tiled;
   a.t.gs = w.gs;
@@ -1447,38 +1515,45 @@ cudaError_t launch_tc_w4a4(const uint8_t* xcodes, const uint8_t* xsf_blocks, int
   a.t.kc_per_split = p.kc_per_split;
   a.t.n_pad = p.n_pad;
   a.sfb = xsf_blocks;
-  const dim3 grid(p.xtiles, p.wtiles, p.splits);
-  auto launch = [&](auto kern, int) -> cudaError_t {
+  const int xt = w4a4_tiles_per_cta(p.xtiles);
+  const dim3 grid((p.xtiles + xt - 1) / xt, p.wtiles, p.splits);
+  auto launch = [&](auto kern1, auto kern2, int) -> cudaError_t {
     // set on every launch: the attribute belongs to the current device's context
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, W4Cfg::kSmemAlloc);
+    const int smem = xt == 1 ? W4Cfg<1>::kSmemAlloc : W4Cfg<2>::kSmemAlloc;
+    cudaError_t e = xt == 1 ? cudaFuncSetAttribute(kern1, cudaFuncAttributeMaxDynamicSharedMemorySize, smem)
+                            : cudaFuncSetAttribute(kern2, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
-    kern<<<grid, 256, W4Cfg::kSmemAlloc, s>>>(map, a);
-    return cudaGetLastError();
+    return xt == 1 ? launch_pdl(kern1, grid, dim3(256), smem, s, map, a)
+                   : launch_pdl(kern2, grid, dim3(256), smem, s, map, a);
   };
   cudaError_t e;
   if (p.splits > 1) {
     a.t.out = partials;
     {
       ProfScope prof(s, silu_mul ? "tc_w4a4_gate_up_partial" : "tc_w4a4_partial");
-      e = launch(tc_w4a4_kernel<kEpiPartial>, kEpiPartial);
+      e = launch(tc_w4a4_kernel<kEpiPartial, 1>, tc_w4a4_kernel<kEpiPartial, 2>, kEpiPartial);
     }
     if (e != cudaSuccess) return e;
     const int64_t total = m * a.t.n_out;
     ProfScope prof(s, silu_mul ? "splitk_reduce_silu_mul" : "splitk_reduce");
-    if (silu_mul)
-      splitk_reduce_kernel<true><<<(unsigned)((total + 255) / 256), 256, 0, s>>>(
-          (const float*)partials, p.splits, (int)m, p.n_pad, a.t.n_out, w.gs, 1.0f, (uint16_t*)y,
-          a.t.ldo);
-    else
-      splitk_reduce_kernel<false><<<(unsigned)((total + 255) / 256), 256, 0, s>>>(
-          (const float*)partials, p.splits, (int)m, p.n_pad, a.t.n_out, w.gs, 1.0f, (uint16_t*)y,
-          a.t.ldo);
-    return cudaGetLastError();
+    const dim3 rgrid((unsigned)((total + 255) / 256));
+    const float* P = static_cast<const float*>(partials);
+    return silu_mul ? launch_pdl(splitk_reduce_kernel<true>, rgrid, dim3(256), 0, s, P, p.splits, (int)m,
+                                 p.n_pad, a.t.n_out, w.gs, 1.0f, static_cast<uint16_t*>(y), a.t.ldo)
+                    : launch_pdl(splitk_reduce_kernel<false>, rgrid, dim3(256), 0, s, P, p.splits, (int)m,
+                                 p.n_pad, a.t.n_out, w.gs, 1.0f, static_cast<uint16_t*>(y), a.t.ldo);
   }
   a.t.out = y;
+  if (silu_mul && hq_codes && hq_sf) {
+    a.t.q_codes = hq_codes;
+    a.t.q_sf = hq_sf;
+    a.t.q_kc = (int)((a.t.n_out + kChunkK - 1) / kChunkK);
+    ProfScope prof(s, "tc_w4a4_gate_up_silu_quant");
+    return launch(tc_w4a4_kernel<kEpiSiluMulQuant, 1>, tc_w4a4_kernel<kEpiSiluMulQuant, 2>, kEpiSiluMulQuant);
+  }
   ProfScope prof(s, silu_mul ? "tc_w4a4_gate_up_silu" : "tc_w4a4");
-  return silu_mul ? launch(tc_w4a4_kernel<kEpiSiluMul>, kEpiSiluMul)
-                  : launch(tc_w4a4_kernel<kEpiStore>, kEpiStore);
+  return silu_mul ? launch(tc_w4a4_kernel<kEpiSiluMul, 1>, tc_w4a4_kernel<kEpiSiluMul, 2>, kEpiSiluMul)
+                  : launch(tc_w4a4_kernel<kEpiStore, 1>, tc_w4a4_kernel<kEpiStore, 2>, kEpiStore);
 }
 
 cudaError_t read_device_error(int* flags, bool clear) {

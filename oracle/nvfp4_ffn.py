@@ -44,6 +44,15 @@ Readings taken where the pages are silent:
   R7 fused gate+up = concatenation of the separately quantised gate and up,
      each with its own tensor scale.
   R8 relative error = sum|out - ref| / sum|ref|.
+  R13 LoRA adapters (page "metrale_model_layers/layers/dense_ffn_overlays.rs",
+     set_lora_weights / apply_lora_gate_up / apply_lora_down): a projection's
+     adapter is a pair A [r, in], B [out, r] of bf16 values, its delta is
+     (x A^T) B^T, with the rank-r product x A^T rounded to bf16 (the pages
+     keep it in an activation buffer), the second product summed exactly and
+     added to the projection's bf16 output, rounded once more to bf16 (the
+     pages add in place into the bf16 gate/up/output buffers).  Gate and up
+     deltas are added before the activation, the down delta after the down
+     projection.  No separate scaling factor appears (it is folded into B).
 
 Precision: the decisions that produce integer codes are taken in fp32 (the
 precision the encoding steps are defined in, and the kernel's), so the codes
@@ -60,7 +69,7 @@ __all__ = [
     "f64_to_bf16_bits", "silu",
     "quantize_weight", "quantize_activation", "pack_nibbles", "unpack_nibbles",
     "dequantize", "project_w4a16", "project_w4a4",
-    "ffn_w4a16", "ffn_w4a4", "fuse_gate_up", "error_stats",
+    "ffn_w4a16", "ffn_w4a4", "fuse_gate_up", "error_stats", "lora_delta", "ffn_w4a16_lora",
     "WEIGHT_SCALE_DIVISOR",
 ]
 
@@ -306,6 +315,35 @@ def ffn_w4a4(x, gate, up, down, return_h: bool = False):
     """Fixed-format FFN: as ``ffn_w4a16`` with x and h quantised per row to
     NVFP4 before their projections."""
     out, h = _ffn(x, gate, up, down, project_w4a4)
+    return (out, h) if return_h else out
+
+
+def lora_delta(x, a, b) -> np.ndarray:
+    """Low-rank delta (x A^T) B^T of one projection (reading R13): the rank-r
+    product rounded to bf16, the second product in fp64 (not rounded).
+
+    x: [m, in] (bf16 values); a: [r, in]; b: [out, r] (bf16 values)."""
+    xa = round_to_bf16(np.asarray(x, dtype=np.float64) @ np.asarray(a, dtype=np.float64).T)
+    return xa @ np.asarray(b, dtype=np.float64).T
+
+
+def ffn_w4a16_lora(x, gate, up, down, lora, return_h: bool = False):
+    """The W4A16 FFN with LoRA adapters (reading R13).
+
+    lora: dict with optional keys 'gate', 'up', 'down', each an (A, B) pair.
+    g = bf16(bf16(x Wg^T) + delta_g), u likewise, h = bf16(silu(g) * u),
+    out = bf16(bf16(h Wd^T) + delta_d)."""
+    x = np.asarray(x, dtype=np.float64)
+
+    def proj(inp, w, key):
+        y = round_to_bf16(project_w4a16(inp, *w))
+        if lora.get(key) is not None:
+            y = round_to_bf16(y + lora_delta(inp, *lora[key]))
+        return y
+    g = proj(x, gate, "gate")
+    u = proj(x, up, "up")
+    h = round_to_bf16(silu(g) * u)
+    out = proj(h, down, "down")
     return (out, h) if return_h else out
 
 

@@ -113,6 +113,36 @@ def _transposed_activation(O):
     O.project_w4a16 = project_w4a16
 
 
+def _lora_xa_unrounded(O):
+    def lora_delta(x, a, b):
+        return (np.asarray(x, np.float64) @ np.asarray(a, np.float64).T) @ np.asarray(b, np.float64).T
+    O.lora_delta = lora_delta
+
+
+def _lora_gate_delta_after_activation(O):
+    def ffn_w4a16_lora(x, gate, up, down, lora, return_h=False):
+        x = np.asarray(x, dtype=np.float64)
+        g = O.round_to_bf16(O.project_w4a16(x, *gate))
+        u = O.round_to_bf16(O.project_w4a16(x, *up))
+        if lora.get("up") is not None:
+            u = O.round_to_bf16(u + O.lora_delta(x, *lora["up"]))
+        h = O.round_to_bf16(O.silu(g) * u)
+        if lora.get("gate") is not None:
+            h = O.round_to_bf16(h + O.lora_delta(x, *lora["gate"]))
+        out = O.round_to_bf16(O.project_w4a16(h, *down))
+        if lora.get("down") is not None:
+            out = O.round_to_bf16(out + O.lora_delta(h, *lora["down"]))
+        return (out, h) if return_h else out
+    O.ffn_w4a16_lora = ffn_w4a16_lora
+
+
+def _lora_adapter_transposed(O):
+    def lora_delta(x, a, b):
+        xa = O.round_to_bf16(np.asarray(x, np.float64) @ np.asarray(a, np.float64)[:, ::-1].T)
+        return xa @ np.asarray(b, np.float64).T
+    O.lora_delta = lora_delta
+
+
 MUTATIONS = {
     "dropped_h_rounding": _dropped_h_rounding,
     "swapped_silu_operands": _swapped_silu_operands,
@@ -126,6 +156,9 @@ MUTATIONS = {
     "activation_scale_amax_over_4": _activation_scale_amax_over_4,
     "projection_drops_tensor_scale": _projection_drops_tensor_scale,
     "transposed_activation": _transposed_activation,
+    "lora_xa_unrounded": _lora_xa_unrounded,
+    "lora_gate_delta_after_activation": _lora_gate_delta_after_activation,
+    "lora_adapter_transposed": _lora_adapter_transposed,
 }
 
 

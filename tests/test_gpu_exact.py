@@ -104,6 +104,8 @@ W4A4_CASES = [
     (1, 384, 256, 1), (1, 128, 4096, 8),
     (130, 384, 256, 1), (130, 128, 4096, 8),
     (7, 256, 1024, None), (64, 640, 2048, None),
+    # three activation tiles: CTAs of two tiles and a last CTA of one
+    (300, 256, 512, None), (300, 128, 4096, 8),
 ]
 
 

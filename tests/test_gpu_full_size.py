@@ -73,3 +73,26 @@ def test_prefill_m4096_full_sampled_rows(native):
     assert_close(out[rows], case.oracle("bf16", rows=rows), "prefill m=4096")
     assert np.all(np.isfinite(out))
     assert native.ffn_nvfp4_device_error(clear=False) == 0
+
+
+def test_w4a4_fused_h_quantisation_is_bit_identical_in_subprocess(native):
+    # the fixed format quantises h inside the gate+up epilogue; the layer
+    # output must be bit for bit what the separate quantiser launch gives
+    import os
+    import subprocess
+    import sys
+    code = (
+        "import sys, hashlib; sys.path.insert(0, 'tests'); sys.path.insert(0, '.');"
+        "from gpu_helpers import FfnCase;"
+        "from nvfp4_quantized_dense_w4a16_b200 import native as N, synth;"
+        "c = FfnCase(N, synth.make_inputs('w4a4', m=64), check_quant=False);"
+        "o = c.forward('nvfp4_fixed').view(__import__('torch').int16).cpu().numpy();"
+        "print('sha', hashlib.sha1(o.tobytes()).hexdigest())")
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    outs = []
+    for fuse in ("1", "0"):
+        r = subprocess.run([sys.executable, "-c", code], cwd=root, capture_output=True, text=True, timeout=900,
+                           env=dict(os.environ, FFN_NVFP4_W4A4_FUSE_HQ=fuse))
+        assert r.returncode == 0, r.stdout + r.stderr
+        outs.append([l for l in r.stdout.splitlines() if l.startswith("sha")][-1])
+    assert outs[0] == outs[1]

@@ -3,7 +3,8 @@
 way, a wrong E4M3 bias, a bf16 with one bit too many, scales on transposed
 blocks, swapped nibbles, a wrong E2M1 table entry, swapped SiLU operands, a
 wrong tensor- or activation-scale convention, a dropped tensor scale, a
-reversed activation operand) is planted in a child pytest process that runs
+reversed activation operand; for the LoRA adapters an unrounded rank-r
+product, a gate delta added after the activation, a mirrored adapter) is planted in a child pytest process that runs
 the oracle's pin tests, and that run must fail.  CPU only."""
 import os
 import subprocess
@@ -15,7 +16,8 @@ from oracle_mutations import MUTATIONS
 
 HERE = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(HERE)
-PINS = ["tests/test_oracle_codecs.py", "tests/test_oracle_quant.py", "tests/test_oracle_ffn.py"]
+PINS = ["tests/test_oracle_codecs.py", "tests/test_oracle_quant.py", "tests/test_oracle_ffn.py",
+        "tests/test_oracle_lora.py"]
 
 
 def _run(mutation):
