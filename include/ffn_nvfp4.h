@@ -193,6 +193,44 @@ ffn_status ffn_nvfp4_forward(const void* x, int64_t m, int64_t hidden, int64_t i
                              ffn_act_format format, void* out, void* workspace,
                              size_t workspace_bytes, void* stream);
 
+/* LoRA adapters on the layer ("metrale_model_layers/layers/
+ * dense_ffn_overlays.rs", set_lora_weights, apply_lora_gate_up,
+ * apply_lora_down): for each of gate, up and down an optional pair A [r, in],
+ * B [out, r] of bf16 (row-major; in/out = hidden/inter for gate and up,
+ * inter/hidden for down), the delta of a projection being (x A^T) B^T.
+ * Numerics: xa = bf16(x A^T) (fp32 sums), then each output
+ * y = bf16(bf16(projection) + sum_i xa_i * B[n, i]) (fp32 sum, i ascending);
+ * gate and up deltas are added before SiLU*mul, the down delta after the
+ * down projection.  No scaling factor is applied (fold it into B).
+ * A missing adapter is a NULL pair (both NULL); at least one must be given.
+ * Copies the matrices to device memory the handle owns (the caller may free
+ * its buffers once the stream has run the copies).  1 <= rank <=
+ * FFN_LORA_MAX_RANK, else FFN_ERR_UNSUPPORTED; FFN_ERR_SHAPE unless hidden
+ * and inter are multiples of 32; a half-given pair is FFN_ERR_INVALID_ARG. */
+#define FFN_LORA_MAX_RANK 256
+typedef struct ffn_lora ffn_lora;
+ffn_status ffn_nvfp4_lora_create(int64_t rank, int64_t hidden, int64_t inter,
+                                 const void* gate_a, const void* gate_b,
+                                 const void* up_a, const void* up_b,
+                                 const void* down_a, const void* down_b,
+                                 void* stream, ffn_lora** out);
+/* Synchronises the device, then frees the adapter's memory.  NULL is accepted. */
+ffn_status ffn_nvfp4_lora_destroy(ffn_lora* lora);
+
+/* ffn_nvfp4_forward with adapters (lora NULL: exactly ffn_nvfp4_forward).
+ * Bf16 activations only (FFN_ERR_UNSUPPORTED for the fixed format, whose
+ * page-defined path has no adapters); the handle must match hidden/inter
+ * (FFN_ERR_SHAPE) and the current device (FFN_ERR_INVALID_ARG).  Two small
+ * extra launches compute the rank-r products; the projections' epilogues add
+ * the deltas.  Workspace: ffn_nvfp4_workspace_size_lora bytes. */
+ffn_status ffn_nvfp4_workspace_size_lora(int64_t m, int64_t hidden, int64_t inter,
+                                         ffn_act_format format, const ffn_lora* lora,
+                                         size_t* bytes);
+ffn_status ffn_nvfp4_forward_lora(const void* x, int64_t m, int64_t hidden, int64_t inter,
+                                  const ffn_nvfp4_weight* gate_up, const ffn_nvfp4_weight* down,
+                                  const ffn_lora* lora, ffn_act_format format, void* out,
+                                  void* workspace, size_t workspace_bytes, void* stream);
+
 /* One projection y[m, n] = bf16(gs * sum_k x[m, k] * w[n, k]) for a plain
  * (not gate+up) handle of shape [n, k]; in FFN_ACT_NVFP4_FIXED x is quantised
  * per row first.  Workspace: ffn_nvfp4_linear_workspace_size bytes. */

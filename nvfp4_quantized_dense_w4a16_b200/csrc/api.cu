@@ -133,7 +133,7 @@ bool serves(const ffn_nvfp4_weight* w, ffn_act_format f) {
 // 256-byte aligned): [h bf16 m*inter] [xq codes m*hidden/2] [xq scales
 // m*hidden/16] [hq codes m*inter/2] [hq scales m*inter/16].
 struct Carve {
-  size_t h = 0, xq_c = 0, xq_s = 0, hq_c = 0, hq_s = 0, part = 0, cnt = 0, total = 0;
+  size_t h = 0, xq_c = 0, xq_s = 0, hq_c = 0, hq_s = 0, part = 0, cnt = 0, xa_gu = 0, xa_d = 0, total = 0;
   ffn::TcPlan gate_up, down;
   ffn::PersistPlan persist;
 };
@@ -160,11 +160,17 @@ void carve_w4a4_tc(Carve& c, size_t& off, int64_t m, int64_t hidden, int64_t int
   off += round_up(pb, 256);
 }
 
-Carve carve_ffn(int64_t m, int64_t hidden, int64_t inter, ffn_act_format f) {
+Carve carve_ffn(int64_t m, int64_t hidden, int64_t inter, ffn_act_format f, int64_t lora_rank = 0) {
   Carve c;
   size_t off = 0;
   c.h = off;
   off += round_up((size_t)m * inter * 2, 256);
+  if (lora_rank > 0) {  // the adapters' rank-r products, bf16
+    c.xa_gu = off;
+    off += round_up((size_t)m * 2 * lora_rank * 2, 256);
+    c.xa_d = off;
+    off += round_up((size_t)m * lora_rank * 2, 256);
+  }
   if (f == FFN_ACT_BF16 && m > 0 && w4a16_persistent(m)) {
     c.persist = ffn::plan_persist(m, hidden, inter, num_sms());
     c.part = off;
@@ -446,11 +452,16 @@ ffn_status ffn_nvfp4_workspace_size(int64_t m, int64_t hidden, int64_t inter,
   return FFN_OK;
 }
 
-ffn_status ffn_nvfp4_forward(const void* x, int64_t m, int64_t hidden, int64_t inter,
-                             const ffn_nvfp4_weight* gate_up, const ffn_nvfp4_weight* down,
-                             ffn_act_format format, void* out, void* workspace,
-                             size_t workspace_bytes, void* stream) {
+ffn_status ffn_nvfp4_forward_lora(const void* x, int64_t m, int64_t hidden, int64_t inter,
+                                  const ffn_nvfp4_weight* gate_up, const ffn_nvfp4_weight* down,
+                                  const ffn_lora* lora, ffn_act_format format, void* out,
+                                  void* workspace, size_t workspace_bytes, void* stream) {
   if (m < 0 || !gate_up || !down) return FFN_ERR_INVALID_ARG;
+  const ffn::LoraView lv = ffn::lora_view(lora);
+  if (lora) {
+    if (format != FFN_ACT_BF16 || w4a16_forced() == 1) return FFN_ERR_UNSUPPORTED;
+    if (ffn::lora_dims_mismatch(lora, hidden, inter)) return FFN_ERR_SHAPE;
+  }
   if (format != FFN_ACT_BF16 && format != FFN_ACT_NVFP4_FIXED) return FFN_ERR_INVALID_ARG;
   if (!valid_k(hidden) || !valid_k(inter)) return FFN_ERR_SHAPE;
   if (!gate_up->gate_up || down->gate_up) return FFN_ERR_INVALID_ARG;
@@ -461,7 +472,15 @@ ffn_status ffn_nvfp4_forward(const void* x, int64_t m, int64_t hidden, int64_t i
   if (ffn_status st = check_device(gate_up)) return st;
   if (ffn_status st = check_device(down)) return st;
   if (!serves(gate_up, format) || !serves(down, format)) return FFN_ERR_UNSUPPORTED;
-  const Carve c = carve_ffn(m, hidden, inter, format);
+  if (lora) {
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess) {
+      cudaGetLastError();
+      return FFN_ERR_CUDA;
+    }
+    if (dev != lv.device) return FFN_ERR_INVALID_ARG;
+  }
+  const Carve c = carve_ffn(m, hidden, inter, format, lv.rank);
   if (!workspace || workspace_bytes < c.total) return FFN_ERR_WORKSPACE;
   if (!aligned16(x) || !aligned16(out) || !aligned16(workspace)) return FFN_ERR_ALIGNMENT;
   if (ffn_status st = precheck()) return st;
@@ -471,11 +490,29 @@ ffn_status ffn_nvfp4_forward(const void* x, int64_t m, int64_t hidden, int64_t i
   cudaError_t e;
   if (format == FFN_ACT_BF16 && w4a16_persistent(m)) {
     e = ffn::launch_persist_ffn(x, m, gate_up->tc(), down->tc(), c.persist, h, ws + c.part,
-                                reinterpret_cast<int*>(ws + c.cnt), out, s);
+                                reinterpret_cast<int*>(ws + c.cnt), out, s, lv, ws + c.xa_gu, ws + c.xa_d);
   } else if (format == FFN_ACT_BF16 && w4a16_path(m) == Path::kTc) {
     void* part = ws + c.part;
-    e = ffn::launch_tc_w4a16(x, m, gate_up->tc(), true, c.gate_up, h, part, s);
-    if (e == cudaSuccess) e = ffn::launch_tc_w4a16(h, m, down->tc(), false, c.down, out, part, s);
+    ffn::LoraArgs lg, ld;
+    e = cudaSuccess;
+    if (lv.rank > 0 && lv.a_gu) {
+      e = ffn::launch_lora_xa(x, m, hidden, lv.a_gu, 2 * lv.rank, ws + c.xa_gu, s);
+      lg.xa = reinterpret_cast<const uint16_t*>(ws + c.xa_gu);
+      lg.xa_ld = 2 * lv.rank;
+      lg.b0 = lv.b_g;
+      lg.b1 = lv.b_u;
+      lg.off1 = lv.rank;
+      lg.r = lv.rank;
+    }
+    if (e == cudaSuccess) e = ffn::launch_tc_w4a16(x, m, gate_up->tc(), true, c.gate_up, h, part, s, lg);
+    if (e == cudaSuccess && lv.rank > 0 && lv.a_d) {
+      e = ffn::launch_lora_xa(h, m, inter, lv.a_d, lv.rank, ws + c.xa_d, s);
+      ld.xa = reinterpret_cast<const uint16_t*>(ws + c.xa_d);
+      ld.xa_ld = lv.rank;
+      ld.b0 = lv.b_d;
+      ld.r = lv.rank;
+    }
+    if (e == cudaSuccess) e = ffn::launch_tc_w4a16(h, m, down->tc(), false, c.down, out, part, s, ld);
   } else if (format == FFN_ACT_BF16) {
     e = ffn::launch_gemv_w4a16(x, m, gate_up->view(), Epilogue::kSiluMul, h, s);
     if (e == cudaSuccess) e = ffn::launch_gemv_w4a16(h, m, down->view(), Epilogue::kStore, out, s);
@@ -535,6 +572,23 @@ ffn_status ffn_nvfp4_projection_plan(int64_t m, int64_t n, int64_t k, ffn_act_fo
   } else {
     *out = ffn_projection_plan{FFN_KERNEL_GEMV_W4A4, 0, 1, ffn::gemv_grid(ncols)};
   }
+  return FFN_OK;
+}
+
+ffn_status ffn_nvfp4_forward(const void* x, int64_t m, int64_t hidden, int64_t inter,
+                             const ffn_nvfp4_weight* gate_up, const ffn_nvfp4_weight* down,
+                             ffn_act_format format, void* out, void* workspace,
+                             size_t workspace_bytes, void* stream) {
+  return ffn_nvfp4_forward_lora(x, m, hidden, inter, gate_up, down, nullptr, format, out, workspace,
+                                workspace_bytes, stream);
+}
+
+ffn_status ffn_nvfp4_workspace_size_lora(int64_t m, int64_t hidden, int64_t inter,
+                                         ffn_act_format format, const ffn_lora* lora, size_t* bytes) {
+  if (!bytes || m < 0) return FFN_ERR_INVALID_ARG;
+  if (format != FFN_ACT_BF16 && format != FFN_ACT_NVFP4_FIXED) return FFN_ERR_INVALID_ARG;
+  if (!valid_k(hidden) || !valid_k(inter)) return FFN_ERR_SHAPE;
+  *bytes = carve_ffn(m, hidden, inter, format, ffn::lora_view(lora).rank).total;
   return FFN_OK;
 }
 

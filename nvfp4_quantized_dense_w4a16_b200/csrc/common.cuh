@@ -6,6 +6,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include "lora_args.h"
+
 namespace ffn {
 
 // ---------------------------------------------------------------------------
@@ -77,6 +79,22 @@ __device__ __forceinline__ float bf16_round(float v) {
 __device__ __forceinline__ uint16_t f32_to_bf16_bits(float v) {
   __nv_bfloat16 b = __float2bfloat16_rn(v);
   return *reinterpret_cast<uint16_t*>(&b);
+}
+
+__device__ __forceinline__ float lora_dot(const uint16_t* xa_row, const uint16_t* b_row, int r) {
+  float d = 0.0f;
+  for (int i = 0; i < r; ++i)
+    d = fmaf(__uint_as_float((uint32_t)xa_row[i] << 16), __uint_as_float((uint32_t)b_row[i] << 16), d);
+  return d;
+}
+
+// y (a bf16 value as fp32) + delta of output n for activation row j, rounded
+// to bf16; unchanged without an adapter.
+__device__ __forceinline__ float lora_add(float y, const uint16_t* b, int off, const LoraArgs& l, int64_t j,
+                                          int64_t n) {
+  if (!b) return y;
+  const float d = lora_dot(l.xa + j * l.xa_ld + off, b + n * l.r, l.r);
+  return __bfloat162float(__float2bfloat16_rn(y + d));
 }
 
 // SiLU in fp32: z / (1 + exp(-z)).

@@ -5,6 +5,7 @@
 #include <stdint.h>
 
 #include "ffn_nvfp4.h"
+#include "lora_args.h"
 
 namespace ffn {
 
@@ -37,6 +38,21 @@ struct TcPlan {
   size_t partial_bytes = 0;  // fp32 split-K partials needed in the workspace
 };
 
+// LoRA adapters of one layer (device copies; see lora.cu).
+struct LoraView {
+  int rank = 0, device = 0;
+  const uint16_t* a_gu = nullptr;  // [2r, hidden]: gate rows then up rows
+  const uint16_t* a_d = nullptr;   // [r, inter]
+  const uint16_t* b_g = nullptr;   // [inter, r]
+  const uint16_t* b_u = nullptr;
+  const uint16_t* b_d = nullptr;   // [hidden, r]
+};
+LoraView lora_view(const ffn_lora* l);
+bool lora_dims_mismatch(const ffn_lora* l, int64_t hidden, int64_t inter);
+// xa[j, i] = bf16(x[j, :] . a[i, :]) for i < rows (x [m, k], a [rows, k]).
+cudaError_t launch_lora_xa(const void* x, int64_t m, int64_t k, const uint16_t* a, int rows, void* xa,
+                           cudaStream_t s);
+
 TcPlan plan_tc(int64_t m, int64_t n, int64_t k, bool gate_up, int num_sms);
 int64_t tc_tiled_bytes(int64_t n, int64_t k, bool gate_up);
 // Fused gate+up tiles from the gate and up handles' tiles of the same kind.
@@ -45,7 +61,8 @@ cudaError_t launch_retile_gate_up(const uint8_t* gate_tiled, const uint8_t* up_t
 cudaError_t launch_tile_weight(const uint8_t* codes, const uint8_t* scales, int64_t n, int64_t k,
                                bool gate_up, bool for_w4a16, uint8_t* out, cudaStream_t s);
 cudaError_t launch_tc_w4a16(const void* x, int64_t m, const TcWeight& w, bool silu_mul,
-                            const TcPlan& p, void* y, void* partials, cudaStream_t s);
+                            const TcPlan& p, void* y, void* partials, cudaStream_t s,
+                            const LoraArgs& lora = LoraArgs());
 // Few-row FFN layer (m <= 64): two persistent launches, one CTA per SM --
 // gate+up over whole tiles dealt round-robin (SiLU*mul epilogue into h), then
 // down over equal contiguous (tile, K chunk) ranges with the split-K sums
@@ -58,9 +75,13 @@ struct PersistPlan {
   size_t partial_bytes = 0, counter_bytes = 0;
 };
 PersistPlan plan_persist(int64_t m, int64_t hidden, int64_t inter, int num_sms);
+// With LoRA adapters (lv.rank > 0): xa_gu [m, 2r] and xa_d [m, r] workspace
+// buffers receive the rank-r products, computed by lora_xa launches before
+// each projection, and the projections' epilogues add the deltas.
 cudaError_t launch_persist_ffn(const void* x, int64_t m, const TcWeight& gate_up, const TcWeight& down,
                                const PersistPlan& p, void* h, void* partials, int* counters, void* out,
-                               cudaStream_t s);
+                               cudaStream_t s, const LoraView& lv = LoraView(), void* xa_gu = nullptr,
+                               void* xa_d = nullptr);
 // Fixed-format (W4A4) projection on the block-scaled FP4 tensor core.  The
 // plan depends on (n, k) only (plus the number of 128-row activation tiles).
 TcPlan plan_w4a4(int64_t m, int64_t n, int64_t k, bool gate_up, int num_sms);

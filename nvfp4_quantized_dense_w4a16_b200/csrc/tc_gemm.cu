@@ -131,6 +131,7 @@ struct TcArgs {
   uint8_t* q_codes = nullptr;
   uint8_t* q_sf = nullptr;
   int q_kc = 0;
+  LoraArgs lora;  // adapter deltas added to the bf16 outputs (store / SiLU*mul)
 };
 
 __device__ __forceinline__ uint32_t bmul2(uint32_t a, uint32_t b) {
@@ -296,8 +297,14 @@ __device__ __forceinline__ void epilogue_tile(const TcArgs& a, uint32_t tmem, in
     } else if (EPI == kEpiStore) {
       uint16_t* T = reinterpret_cast<uint16_t*>(ebuf);  // [32][128] bf16
       const float gs = a.gs[0] * gs_mul;
+      const int64_t nrow = (int64_t)kTileRows * wtile + row;
+      const bool lv = a.lora.b0 != nullptr && nrow < a.n_out;
 #pragma unroll
-      for (int j = 0; j < 32; ++j) T[j * 128 + row] = f32_to_bf16_bits(gs * __uint_as_float(v[j]));
+      for (int j = 0; j < 32; ++j) {
+        float y = gs * __uint_as_float(v[j]);
+        if (lv && r0 + j < a.m) y = lora_add(bf16_round(y), a.lora.b0, a.lora.off0, a.lora, r0 + j, nrow);
+        T[j * 128 + row] = f32_to_bf16_bits(y);
+      }
       named_bar_sync(1 + g, 128);
       const int n0 = kTileRows * wtile;
       for (int idx = et; idx < 32 * 16; idx += 128) {
@@ -313,15 +320,24 @@ __device__ __forceinline__ void epilogue_tile(const TcArgs& a, uint32_t tmem, in
       uint16_t* Hs = reinterpret_cast<uint16_t*>(ebuf + 8192);    // [32][64] bf16
       if (q >= 2) {
         const float gsu = a.gs[1] * gs_mul;
+        const int64_t nu = 64 * (int64_t)wtile + row - 64;
+        const bool lv = a.lora.b1 != nullptr && nu < a.n_out;
 #pragma unroll
-        for (int j = 0; j < 32; ++j) U[j * 64 + (row - 64)] = bf16_round(gsu * __uint_as_float(v[j]));
+        for (int j = 0; j < 32; ++j) {
+          float uv = bf16_round(gsu * __uint_as_float(v[j]));
+          if (lv && r0 + j < a.m) uv = lora_add(uv, a.lora.b1, a.lora.off1, a.lora, r0 + j, nu);
+          U[j * 64 + (row - 64)] = uv;
+        }
       }
       named_bar_sync(1 + g, 128);
       if (q < 2) {
         const float gsg = a.gs[0] * gs_mul;
+        const int64_t ng = 64 * (int64_t)wtile + row;
+        const bool lv = a.lora.b0 != nullptr && ng < a.n_out;
 #pragma unroll
         for (int j = 0; j < 32; ++j) {
-          const float gv = bf16_round(gsg * __uint_as_float(v[j]));
+          float gv = bf16_round(gsg * __uint_as_float(v[j]));
+          if (lv && r0 + j < a.m) gv = lora_add(gv, a.lora.b0, a.lora.off0, a.lora, r0 + j, ng);
           Hs[j * 64 + row] = f32_to_bf16_bits(silu_fast(gv) * U[j * 64 + row]);
         }
       }
@@ -567,6 +583,7 @@ struct PArgs {
   int* counters;       // kModeRanges: [ntiles], zero on entry
   int* zero_ptr;       // kModeTiles: counters of the next projection (or null)
   int zero_count;
+  LoraArgs lora;       // adapter deltas added to the bf16 outputs
 };
 
 struct Seg {
@@ -844,8 +861,14 @@ tc_w4a16_persistent_kernel(const __grid_constant__ CUtensorMap xmap, const PArgs
           // rows 64..127 (up) hand bf16(gs_u * u) to rows 0..63 (gate)
           if (q >= 2) {
             const float gsu = a.gs[1] * kW4A16Unscale;
+            const int nu = 64 * sg.tile + row - 64;
+            const bool lv = a.lora.b1 != nullptr && nu < a.n_out;
 #pragma unroll
-            for (int i = 0; i < 32; ++i) U[i * 64 + (row - 64)] = bf16_round(gsu * acc[i]);
+            for (int i = 0; i < 32; ++i) {
+              float uv = bf16_round(gsu * acc[i]);
+              if (lv && i < jmax) uv = lora_add(uv, a.lora.b1, a.lora.off1, a.lora, 32 * c + i, nu);
+              U[i * 64 + (row - 64)] = uv;
+            }
           }
           named_bar_sync(1 + g, 128);
           if (q < 2) {
@@ -855,7 +878,8 @@ tc_w4a16_persistent_kernel(const __grid_constant__ CUtensorMap xmap, const PArgs
 #pragma unroll
               for (int i = 0; i < 32; ++i) {
                 if (i < jmax) {
-                  const float gv = bf16_round(gsg * acc[i]);
+                  float gv = bf16_round(gsg * acc[i]);
+                  if (a.lora.b0) gv = lora_add(gv, a.lora.b0, a.lora.off0, a.lora, 32 * c + i, n);
                   a.out[(size_t)(32 * c + i) * a.ldo + n] = f32_to_bf16_bits(silu_fast(gv) * U[i * 64 + row]);
                 }
               }
@@ -910,7 +934,11 @@ tc_w4a16_persistent_kernel(const __grid_constant__ CUtensorMap xmap, const PArgs
             float sum = 0.0f;
             for (int gg = g0; gg <= g1; ++gg)
               sum += __ldcg(a.partials + ((size_t)(gg + sg.tile) * a.m + jr) * kTileRows + rr);
-            if (n < a.n_out) a.out[(size_t)jr * a.ldo + n] = f32_to_bf16_bits(gsd * sum);
+            if (n < a.n_out) {
+              float y = gsd * sum;
+              if (a.lora.b0) y = lora_add(bf16_round(y), a.lora.b0, a.lora.off0, a.lora, jr, n);
+              a.out[(size_t)jr * a.ldo + n] = f32_to_bf16_bits(y);
+            }
           }
         }
       }
@@ -1106,7 +1134,7 @@ tc_w4a4_kernel(const __grid_constant__ CUtensorMap xmap, const W4Args w4) {
 template <bool kGateUp>
 __global__ void splitk_reduce_kernel(const float* __restrict__ P, int splits, int m, int n_pad,
                                      int n_out, const float* __restrict__ gs, float gs_mul,
-                                     uint16_t* __restrict__ out, int ldo) {
+                                     uint16_t* __restrict__ out, int ldo, const LoraArgs lora) {
   griddep_wait();  // the partial sums come from the previous kernel
   griddep_launch_dependents();
   const int64_t idx = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;
@@ -1120,12 +1148,15 @@ __global__ void splitk_reduce_kernel(const float* __restrict__ P, int splits, in
       g += P[z * plane + (size_t)r * n_pad + gcol];
       u += P[z * plane + (size_t)r * n_pad + ucol];
     }
-    const float gb = bf16_round(gs[0] * gs_mul * g), ub = bf16_round(gs[1] * gs_mul * u);
+    const float gb = lora_add(bf16_round(gs[0] * gs_mul * g), lora.b0, lora.off0, lora, r, n);
+    const float ub = lora_add(bf16_round(gs[1] * gs_mul * u), lora.b1, lora.off1, lora, r, n);
     out[(size_t)r * ldo + n] = f32_to_bf16_bits(silu_fast(gb) * ub);
   } else {
     float acc = 0.0f;
     for (int z = 0; z < splits; ++z) acc += P[z * plane + (size_t)r * n_pad + n];
-    out[(size_t)r * ldo + n] = f32_to_bf16_bits(gs[0] * gs_mul * acc);
+    float y = gs[0] * gs_mul * acc;
+    if (lora.b0) y = lora_add(bf16_round(y), lora.b0, lora.off0, lora, r, n);
+    out[(size_t)r * ldo + n] = f32_to_bf16_bits(y);
   }
 }
 
@@ -1332,7 +1363,7 @@ PersistPlan plan_persist(int64_t m, int64_t hidden, int64_t inter, int num_sms) 
 
 cudaError_t launch_persist_ffn(const void* x, int64_t m, const TcWeight& gate_up, const TcWeight& down,
                                const PersistPlan& p, void* h, void* partials, int* counters, void* out,
-                               cudaStream_t s) {
+                               cudaStream_t s, const LoraView& lv, void* xa_gu, void* xa_d) {
   const int box_rows = (int)m;
   const int64_t inter = gate_up.n / 2, hidden = down.n;
   CUtensorMap xm, hm;
@@ -1350,12 +1381,27 @@ cudaError_t launch_persist_ffn(const void* x, int64_t m, const TcWeight& gate_up
   a.x_box_rows = box_rows;
   a.zero_ptr = counters;
   a.zero_count = p.dn_tiles;
-  cudaError_t e;
+  cudaError_t e = cudaSuccess;
+  if (lv.rank > 0 && lv.a_gu) {
+    e = launch_lora_xa(x, m, gate_up.k, lv.a_gu, 2 * lv.rank, xa_gu, s);
+    a.lora.xa = static_cast<const uint16_t*>(xa_gu);
+    a.lora.xa_ld = 2 * lv.rank;
+    a.lora.b0 = lv.b_g;
+    a.lora.b1 = lv.b_u;
+    a.lora.off0 = 0;
+    a.lora.off1 = lv.rank;
+    a.lora.r = lv.rank;
+  }
+  if (e != cudaSuccess) return e;
   {
     ProfScope prof(s, "tc_w4a16_gate_up_silu_persistent");
     e = launch_persist_bn<kModeTiles>(p.bn, xm, a, p.gu_grid, s);
   }
   if (e != cudaSuccess) return e;
+  if (lv.rank > 0 && lv.a_d) {
+    e = launch_lora_xa(h, m, down.k, lv.a_d, lv.rank, xa_d, s);
+    if (e != cudaSuccess) return e;
+  }
   PArgs b{};
   b.wt = down.tiled16;
   b.gs = down.gs;
@@ -1368,6 +1414,12 @@ cudaError_t launch_persist_ffn(const void* x, int64_t m, const TcWeight& gate_up
   b.x_box_rows = box_rows;
   b.partials = static_cast<float*>(partials);
   b.counters = counters;
+  if (lv.rank > 0 && lv.a_d) {
+    b.lora.xa = static_cast<const uint16_t*>(xa_d);
+    b.lora.xa_ld = lv.rank;
+    b.lora.b0 = lv.b_d;
+    b.lora.r = lv.rank;
+  }
   ProfScope prof(s, "tc_w4a16_down_persistent");
   return launch_persist_bn<kModeRanges>(p.bn, hm, b, p.dn_grid, s);
 }
@@ -1422,7 +1474,8 @@ TcPlan plan_tc(int64_t m, int64_t n, int64_t k, bool gate_up, int num_sms) {
 }
 
 cudaError_t launch_tc_w4a16(const void* x, int64_t m, const TcWeight& w, bool silu_mul,
-                            const TcPlan& p, void* y, void* partials, cudaStream_t s) {
+                            const TcPlan& p, void* y, void* partials, cudaStream_t s,
+                            const LoraArgs& lora) {
   CUtensorMap map;
   const int box_rows = (int)(m < p.bn ? m : p.bn);
   if (!make_x_map(&map, x, m, w.k, box_rows)) return cudaErrorInvalidValue;
@@ -1436,6 +1489,7 @@ cudaError_t launch_tc_w4a16(const void* x, int64_t m, const TcWeight& w, bool si
   a.kc_total = p.kc;
   a.kc_per_split = p.kc_per_split;
   a.n_pad = p.n_pad;
+  a.lora = lora;
   const dim3 grid(p.xtiles, p.wtiles, p.splits);
   cudaError_t e;
   if (p.splits > 1) {
@@ -1451,10 +1505,10 @@ cudaError_t launch_tc_w4a16(const void* x, int64_t m, const TcWeight& w, bool si
     const float* P = static_cast<const float*>(partials);
     return silu_mul ? launch_pdl(splitk_reduce_kernel<true>, rgrid, dim3(256), 0, s, P, p.splits,
                                  (int)m, p.n_pad, a.n_out, w.gs, kW4A16Unscale,
-                                 static_cast<uint16_t*>(y), a.ldo)
+                                 static_cast<uint16_t*>(y), a.ldo, lora)
                     : launch_pdl(splitk_reduce_kernel<false>, rgrid, dim3(256), 0, s, P, p.splits,
                                  (int)m, p.n_pad, a.n_out, w.gs, kW4A16Unscale,
-                                 static_cast<uint16_t*>(y), a.ldo);
+                                 static_cast<uint16_t*>(y), a.ldo, lora);
   }
   a.out = y;
   ProfScope prof(s, silu_mul ? "tc_w4a16_gate_up_silu" : "tc_w4a16");
@@ -1539,9 +1593,9 @@ cudaError_t launch_tc_w4a4(const uint8_t* xcodes, const uint8_t* xsf_blocks, int
     const dim3 rgrid((unsigned)((total + 255) / 256));
     const float* P = static_cast<const float*>(partials);
     return silu_mul ? launch_pdl(splitk_reduce_kernel<true>, rgrid, dim3(256), 0, s, P, p.splits, (int)m,
-                                 p.n_pad, a.t.n_out, w.gs, 1.0f, static_cast<uint16_t*>(y), a.t.ldo)
+                                 p.n_pad, a.t.n_out, w.gs, 1.0f, static_cast<uint16_t*>(y), a.t.ldo, LoraArgs())
                     : launch_pdl(splitk_reduce_kernel<false>, rgrid, dim3(256), 0, s, P, p.splits, (int)m,
-                                 p.n_pad, a.t.n_out, w.gs, 1.0f, static_cast<uint16_t*>(y), a.t.ldo);
+                                 p.n_pad, a.t.n_out, w.gs, 1.0f, static_cast<uint16_t*>(y), a.t.ldo, LoraArgs());
   }
   a.t.out = y;
   if (silu_mul && hq_codes && hq_sf) {

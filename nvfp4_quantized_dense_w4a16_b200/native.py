@@ -68,6 +68,10 @@ def _load() -> ctypes.CDLL:
         "ffn_nvfp4_weight_dims": (ctypes.c_int, [vp, P(i64), P(i64), P(ctypes.c_int)]),
         "ffn_nvfp4_workspace_size": (ctypes.c_int, [i64, i64, i64, ctypes.c_int, P(sz)]),
         "ffn_nvfp4_forward": (ctypes.c_int, [vp, i64, i64, i64, vp, vp, ctypes.c_int, vp, vp, sz, vp]),
+        "ffn_nvfp4_forward_lora": (ctypes.c_int, [vp, i64, i64, i64, vp, vp, vp, ctypes.c_int, vp, vp, sz, vp]),
+        "ffn_nvfp4_workspace_size_lora": (ctypes.c_int, [i64, i64, i64, ctypes.c_int, vp, P(sz)]),
+        "ffn_nvfp4_lora_create": (ctypes.c_int, [i64, i64, i64, vp, vp, vp, vp, vp, vp, vp, P(vp)]),
+        "ffn_nvfp4_lora_destroy": (ctypes.c_int, [vp]),
         "ffn_nvfp4_linear_workspace_size": (ctypes.c_int, [i64, i64, i64, ctypes.c_int, P(sz)]),
         "ffn_nvfp4_linear": (ctypes.c_int, [vp, i64, vp, ctypes.c_int, vp, vp, sz, vp]),
         "ffn_nvfp4_linear_noalloc": (ctypes.c_int, [vp, i64, vp, vp, vp]),
@@ -240,18 +244,70 @@ def _workspace(nbytes: int, device, workspace):
     return workspace
 
 
+class Lora:
+    """Owning wrapper of an ``ffn_lora*`` adapter handle."""
+
+    def __init__(self, handle: ctypes.c_void_p, rank: int):
+        self._h, self.rank = handle, rank
+
+    @property
+    def handle(self):
+        return self._h
+
+    def close(self):
+        if self._h:
+            _check("ffn_nvfp4_lora_destroy", lib.ffn_nvfp4_lora_destroy(self._h))
+            self._h = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+
+def ffn_nvfp4_lora_create(rank: int, hidden: int, inter: int, gate=None, up=None, down=None,
+                          stream=None) -> Lora:
+    """Adapters for a layer: each of gate/up/down an (A, B) pair of bf16
+    tensors (A [rank, in], B [out, rank]) or None."""
+    ptrs = []
+    for name, pair, n_in, n_out in (("gate", gate, hidden, inter), ("up", up, hidden, inter),
+                                    ("down", down, inter, hidden)):
+        if pair is None:
+            ptrs += [None, None]
+            continue
+        a, b = pair
+        _need(a, name + "_a", torch.bfloat16, (rank, n_in))
+        _need(b, name + "_b", torch.bfloat16, (n_out, rank))
+        ptrs += [_ptr(a), _ptr(b)]
+    h = ctypes.c_void_p()
+    _check("ffn_nvfp4_lora_create", lib.ffn_nvfp4_lora_create(rank, hidden, inter, *ptrs, _stream(stream),
+                                                              ctypes.byref(h)))
+    return Lora(h, rank)
+
+
 def ffn_nvfp4_forward(x: torch.Tensor, gate_up: Weight, down: Weight, fmt="bf16", out=None,
-                      workspace=None, stream=None) -> torch.Tensor:
-    """out[m, hidden] = down(silu(gate(x)) * up(x)) through the C ABI."""
+                      workspace=None, stream=None, lora: Lora | None = None) -> torch.Tensor:
+    """out[m, hidden] = down(silu(gate(x)) * up(x)) through the C ABI (with
+    the adapters' deltas when `lora` is given)."""
     _need(x, "x", torch.bfloat16)
     m, hidden = x.shape
     inter = down.k
     out = torch.empty((m, hidden), dtype=torch.bfloat16, device=x.device) if out is None else out
     _need(out, "out", torch.bfloat16, (m, hidden))
-    nbytes = ffn_nvfp4_workspace_size(m, hidden, inter, fmt)
-    workspace = _workspace(nbytes, x.device, workspace)
-    _check("ffn_nvfp4_forward", lib.ffn_nvfp4_forward(
-        _ptr(x), m, hidden, inter, gate_up.handle, down.handle, _fmt(fmt), _ptr(out),
+    if lora is None:
+        nbytes = ffn_nvfp4_workspace_size(m, hidden, inter, fmt)
+        workspace = _workspace(nbytes, x.device, workspace)
+        _check("ffn_nvfp4_forward", lib.ffn_nvfp4_forward(
+            _ptr(x), m, hidden, inter, gate_up.handle, down.handle, _fmt(fmt), _ptr(out),
+            _ptr(workspace), workspace.numel(), _stream(stream)))
+        return out
+    nb = ctypes.c_size_t()
+    _check("ffn_nvfp4_workspace_size_lora", lib.ffn_nvfp4_workspace_size_lora(
+        m, hidden, inter, _fmt(fmt), lora.handle, ctypes.byref(nb)))
+    workspace = _workspace(nb.value, x.device, workspace)
+    _check("ffn_nvfp4_forward_lora", lib.ffn_nvfp4_forward_lora(
+        _ptr(x), m, hidden, inter, gate_up.handle, down.handle, lora.handle, _fmt(fmt), _ptr(out),
         _ptr(workspace), workspace.numel(), _stream(stream)))
     return out
 

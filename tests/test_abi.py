@@ -105,3 +105,18 @@ def test_weight_create_ex_rejects_bad_formats(native):
     assert L.ffn_nvfp4_weight_create_ex(fake, fake, fake, 4, 64, 4, None, ctypes.byref(h)) == 1
     assert L.ffn_nvfp4_weight_create_ex(fake, fake, fake, 4, 40, 1, None, ctypes.byref(h)) == 2
     assert L.ffn_nvfp4_weight_info(None, None, None) == 1
+
+
+def test_lora_create_host_checks(native):
+    L = native.lib
+    fake = ctypes.c_void_p(256)
+    h = ctypes.c_void_p()
+    assert L.ffn_nvfp4_lora_create(0, 256, 512, fake, fake, None, None, None, None, None, ctypes.byref(h)) == 4
+    assert L.ffn_nvfp4_lora_create(257, 256, 512, fake, fake, None, None, None, None, None, ctypes.byref(h)) == 4
+    assert L.ffn_nvfp4_lora_create(4, 250, 512, fake, fake, None, None, None, None, None, ctypes.byref(h)) == 2
+    assert L.ffn_nvfp4_lora_create(4, 256, 512, fake, None, None, None, None, None, None, ctypes.byref(h)) == 1
+    assert L.ffn_nvfp4_lora_create(4, 256, 512, None, None, None, None, None, None, None, ctypes.byref(h)) == 1
+    assert L.ffn_nvfp4_lora_destroy(None) == 0
+    sz = ctypes.c_size_t()
+    assert L.ffn_nvfp4_workspace_size_lora(4, 256, 512, 0, None, ctypes.byref(sz)) == 0
+    assert sz.value == native.ffn_nvfp4_workspace_size(4, 256, 512, "bf16")
