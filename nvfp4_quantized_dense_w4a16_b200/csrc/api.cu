@@ -79,6 +79,7 @@ int w4a16_forced() {
     if (!v) return 0;
     if (!strcmp(v, "gemv")) return 1;
     if (!strcmp(v, "tc")) return 2;
+    if (!strcmp(v, "persistent")) return 3;
     return 0;
   }();
   return forced;
@@ -90,9 +91,12 @@ Path w4a16_path(int64_t m) {
   return Path::kTc;
 }
 
-// The FFN layer for few rows runs as two persistent launches (see
-// plan_persist) unless FFN_NVFP4_W4A16_PATH forces a projection family.
-bool w4a16_persistent(int64_t m) { return w4a16_forced() == 0 && m <= ffn::kPersistMaxRows; }
+// The two persistent launches for few rows (see plan_persist) run only when
+// FFN_NVFP4_W4A16_PATH=persistent: measured on B200 at m = 1..64 they were
+// slower than the per-tile kernels (one CTA per SM halves the MMA-issuing
+// threads per SM, which bound these narrow tiles), so the default keeps the
+// per-tile kernels.
+bool w4a16_persistent(int64_t m) { return w4a16_forced() == 3 && m <= ffn::kPersistMaxRows; }
 
 // Fixed format: the block-scaled FP4 tensor-core kernel, or the CUDA-core one
 // (FFN_NVFP4_W4A4_PATH=gemv).  Either choice is made once per process and does

@@ -185,3 +185,21 @@ def test_ffn_exact_inputs_bit_exact(native, m, H, I):
     plan = native.ffn_nvfp4_projection_plan(m, H, I, "bf16", role="down")
     assert bad.size == 0, f"{plan}: {len(bad)} mismatches, first at {bad[:3].tolist()}"
     assert native.ffn_nvfp4_device_error(clear=False) == 0
+
+
+def test_persistent_path_bit_exact_in_subprocess(native):
+    # the persistent few-row kernels (selectable, not the default) keep the
+    # bit-exact property on the exactly representable layer
+    import os
+    import subprocess
+    import sys
+    code = (
+        "import sys; sys.path.insert(0, 'tests'); sys.path.insert(0, '.');"
+        "import test_gpu_exact as T; from nvfp4_quantized_dense_w4a16_b200 import native as N;"
+        "assert N.ffn_nvfp4_projection_plan(5, 1024, 4096, role='down')['family'] == 'tc_w4a16_persistent';"
+        "[T.test_ffn_exact_inputs_bit_exact(N, *c) for c in [(1, 512, 1536), (5, 1024, 4096), (16, 512, 800),"
+        " (33, 512, 1536), (64, 1024, 2048)]]; print('persistent-ok')")
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    r = subprocess.run([sys.executable, "-c", code], cwd=root, capture_output=True, text=True, timeout=900,
+                       env=dict(os.environ, FFN_NVFP4_W4A16_PATH="persistent"))
+    assert r.returncode == 0 and "persistent-ok" in r.stdout, r.stdout + r.stderr
