@@ -224,6 +224,9 @@ class Workload:
             q.append(native.ffn_nvfp4_quantize_weights(w))
             del w
         self.weight_bytes = nvfp4_bytes(2 * I, H) + nvfp4_bytes(H, I)
+        # weight layouts the handles hold: the few-row bf16 workloads also keep
+        # the natural tiles, which the block-scaled FP4 path for m <= 8 streams
+        self.layouts = "all" if (fmt == "bf16" and name in ("decode", "smallm")) else fmt
         # A step that reads less than twice the L2 would find part of its
         # weights still cached from earlier steps: such layers rotate through R
         # copies of their weights (R x weight bytes >= 4 x L2), so every step
@@ -234,7 +237,7 @@ class Workload:
             self.sets = int(math.ceil(4 * L2_BYTES / self.weight_bytes))
         self.handles = []
         for _ in range(self.sets):
-            g, u, d = (native.ffn_nvfp4_weight_create(*t, formats=fmt) for t in q)
+            g, u, d = (native.ffn_nvfp4_weight_create(*t, formats=self.layouts) for t in q)
             self.handles.append((native.ffn_nvfp4_weight_create_gate_up(g, u), d))
             del g, u
         del q
@@ -354,7 +357,7 @@ def run_ours(args, rank, world, dist):
            "h2d_bytes_per_step": wl.m * wl.H * 2, "d2h_bytes_per_step": wl.m * wl.H * 2,
            "ms_per_step": round(e2e_ms / e2e_steps, 4)}
 
-    l2_note = wl.l2_note
+    l2_note, layouts = wl.l2_note, wl.layouts
     extra = {}
     if not args.no_extra and args.workload == "prefill":
         del wl, x_dev
@@ -370,7 +373,7 @@ def run_ours(args, rank, world, dist):
         "value": round(value, 3), "ms_per_step": round(ms_step, 4), "roofline": roof,
         "kernels": kernels, "gpu_launches": gpu_launches, "clocks": clk, "e2e": e2e,
         "workload": args.workload, "m": args.m or WORKLOADS[args.workload][1], "extra": extra,
-        "l2": l2_note,
+        "l2": l2_note, "layouts": layouts,
     }
 
 
@@ -571,7 +574,7 @@ def main():
         "dtype": "bf16 x nvfp4 (fp32 accumulate)" if fmt == "bf16" else "nvfp4 x nvfp4 (fp32 accumulate)",
         "data": "synthetic (seeded numpy draws; random-init weights)",
         "config": {"workload": args.workload, "m": res["m"], "hidden": H, "inter": I, "act_format": fmt,
-                   "parallelism": f"replicas x{world}", "l2": res["l2"],
+                   "parallelism": f"replicas x{world}", "l2": res["l2"], "weight_layouts": res["layouts"],
                    "launch": ("eager launches" if args.eager else
                               "the K timed steps captured in one CUDA graph, replayed once; "
                               "kernel durations from a second replay with an event pair per kernel")},

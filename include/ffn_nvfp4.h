@@ -281,9 +281,21 @@ typedef enum ffn_kernel_family {
   FFN_KERNEL_TC_W4A4 = 2,    /* tcgen05 block-scaled FP4 MMA (kind::mxf4nvf4)   */
   FFN_KERNEL_GEMV_W4A16 = 3, /* CUDA-core projection, bf16 activations          */
   FFN_KERNEL_GEMV_W4A4 = 4,  /* CUDA-core projection, fixed activation format   */
-  FFN_KERNEL_TC_W4A16_PERSISTENT = 5 /* few-row FFN layer: persistent tcgen05
+  FFN_KERNEL_TC_W4A16_PERSISTENT = 5, /* few-row FFN layer: persistent tcgen05
                                 kernels, one CTA per SM, gate+up over whole tiles,
-                                down over equal K ranges reduced in-kernel       */
+                                down over equal K ranges reduced in-kernel
+                                (only with FFN_NVFP4_W4A16_PATH=persistent)     */
+  FFN_KERNEL_TC_PLANES = 6   /* FFN layer for m <= 8 with bf16 activations when
+                                both handles hold the natural tiled layout
+                                (built for the fixed format too, e.g.
+                                FFN_FORMAT_ALL): the NVFP4 weights go to the
+                                block-scaled FP4 MMA as stored and each
+                                activation row as 8 or 16 NVFP4 residual planes
+                                (N = 8m or 16 columns, exact for bf16 rows of
+                                normal spread); equal K ranges per CTA, two
+                                CTAs per SM, split-K sums added in-kernel.
+                                tile_rows reports the MMA's N.  Without the
+                                natural layout the layer takes FFN_KERNEL_TC_W4A16. */
 } ffn_kernel_family;
 
 typedef enum ffn_projection_role {

@@ -80,6 +80,7 @@ int w4a16_forced() {
     if (!strcmp(v, "gemv")) return 1;
     if (!strcmp(v, "tc")) return 2;
     if (!strcmp(v, "persistent")) return 3;
+    if (!strcmp(v, "planes")) return 4;
     return 0;
   }();
   return forced;
@@ -97,6 +98,16 @@ Path w4a16_path(int64_t m) {
 // threads per SM, which bound these narrow tiles), so the default keeps the
 // per-tile kernels.
 bool w4a16_persistent(int64_t m) { return w4a16_forced() == 3 && m <= ffn::kPersistMaxRows; }
+
+// Few rows (m <= 8) with both weights in the natural tiled layout (handles
+// built for the fixed format too, e.g. FFN_FORMAT_ALL): the block-scaled FP4
+// path with activation planes, unless FFN_NVFP4_W4A16_PATH forces another.
+bool w4a16_planes(int64_t m, int64_t hidden, int64_t inter, const ffn_nvfp4_weight* gu,
+                  const ffn_nvfp4_weight* dn) {
+  const int f = w4a16_forced();
+  return (f == 0 || f == 4) && ffn::planes_for_rows(m) > 0 && hidden <= 24576 && inter <= 24576 &&
+         gu && dn && gu->tiled && dn->tiled;
+}
 
 // Fixed format: the block-scaled FP4 tensor-core kernel, or the CUDA-core one
 // (FFN_NVFP4_W4A4_PATH=gemv).  Either choice is made once per process and does
@@ -138,8 +149,10 @@ bool serves(const ffn_nvfp4_weight* w, ffn_act_format f) {
 // m*hidden/16] [hq codes m*inter/2] [hq scales m*inter/16].
 struct Carve {
   size_t h = 0, xq_c = 0, xq_s = 0, hq_c = 0, hq_s = 0, part = 0, cnt = 0, xa_gu = 0, xa_d = 0, total = 0;
+  size_t xg = 0, hg = 0;  // plane factors
   ffn::TcPlan gate_up, down;
   ffn::PersistPlan persist;
+  ffn::PlanesPlan planes;
 };
 
 // Workspace of the fixed format on the tensor-core path: quantised x and h
@@ -164,7 +177,8 @@ void carve_w4a4_tc(Carve& c, size_t& off, int64_t m, int64_t hidden, int64_t int
   off += round_up(pb, 256);
 }
 
-Carve carve_ffn(int64_t m, int64_t hidden, int64_t inter, ffn_act_format f, int64_t lora_rank = 0) {
+Carve carve_ffn(int64_t m, int64_t hidden, int64_t inter, ffn_act_format f, int64_t lora_rank = 0,
+                bool planes = false) {
   Carve c;
   size_t off = 0;
   c.h = off;
@@ -175,7 +189,20 @@ Carve carve_ffn(int64_t m, int64_t hidden, int64_t inter, ffn_act_format f, int6
     c.xa_d = off;
     off += round_up((size_t)m * lora_rank * 2, 256);
   }
-  if (f == FFN_ACT_BF16 && m > 0 && w4a16_persistent(m)) {
+  if (f == FFN_ACT_BF16 && m > 0 && planes) {
+    // plane codes [m*P, k/2], scale blocks [kc][512], factors [m][P], split-K
+    // partials and tile counters
+    c.planes = ffn::plan_planes(m, hidden, inter, num_sms());
+    const size_t rows = (size_t)m * c.planes.planes;
+    c.xq_c = off; off += round_up(rows * hidden / 2, 256);
+    c.xq_s = off; off += round_up((size_t)((hidden + 63) / 64) * 512, 256);
+    c.hq_c = off; off += round_up(rows * inter / 2, 256);
+    c.hq_s = off; off += round_up((size_t)((inter + 63) / 64) * 512, 256);
+    c.xg = off; off += round_up(rows * sizeof(float), 256);
+    c.hg = off; off += round_up(rows * sizeof(float), 256);
+    c.part = off; off += round_up(c.planes.partial_bytes, 256);
+    c.cnt = off; off += round_up((size_t)c.planes.counter_count * sizeof(int), 256);
+  } else if (f == FFN_ACT_BF16 && m > 0 && w4a16_persistent(m)) {
     c.persist = ffn::plan_persist(m, hidden, inter, num_sms());
     c.part = off;
     off += round_up(c.persist.partial_bytes, 256);
@@ -200,6 +227,19 @@ Carve carve_ffn(int64_t m, int64_t hidden, int64_t inter, ffn_act_format f, int6
   }
   c.total = off;
   return c;
+}
+
+// Workspace bytes for the path forward will take, which can depend on the
+// handles' layouts: the larger of the two few-row candidates.
+size_t ffn_workspace_bytes(int64_t m, int64_t hidden, int64_t inter, ffn_act_format f, int64_t lora_rank) {
+  size_t b = carve_ffn(m, hidden, inter, f, lora_rank, false).total;
+  const int forced = w4a16_forced();
+  if (f == FFN_ACT_BF16 && (forced == 0 || forced == 4) && ffn::planes_for_rows(m) > 0 && hidden <= 24576 &&
+      inter <= 24576) {
+    const size_t bp = carve_ffn(m, hidden, inter, f, lora_rank, true).total;
+    if (bp > b) b = bp;
+  }
+  return b;
 }
 
 Carve carve_linear(int64_t m, int64_t n, int64_t k, ffn_act_format f) {
@@ -452,7 +492,7 @@ ffn_status ffn_nvfp4_workspace_size(int64_t m, int64_t hidden, int64_t inter,
   if (!bytes || m < 0) return FFN_ERR_INVALID_ARG;
   if (format != FFN_ACT_BF16 && format != FFN_ACT_NVFP4_FIXED) return FFN_ERR_INVALID_ARG;
   if (!valid_k(hidden) || !valid_k(inter)) return FFN_ERR_SHAPE;
-  *bytes = carve_ffn(m, hidden, inter, format).total;
+  *bytes = ffn_workspace_bytes(m, hidden, inter, format, 0);
   return FFN_OK;
 }
 
@@ -484,7 +524,8 @@ ffn_status ffn_nvfp4_forward_lora(const void* x, int64_t m, int64_t hidden, int6
     }
     if (dev != lv.device) return FFN_ERR_INVALID_ARG;
   }
-  const Carve c = carve_ffn(m, hidden, inter, format, lv.rank);
+  const bool planes = format == FFN_ACT_BF16 && w4a16_planes(m, hidden, inter, gate_up, down);
+  const Carve c = carve_ffn(m, hidden, inter, format, lv.rank, planes);
   if (!workspace || workspace_bytes < c.total) return FFN_ERR_WORKSPACE;
   if (!aligned16(x) || !aligned16(out) || !aligned16(workspace)) return FFN_ERR_ALIGNMENT;
   if (ffn_status st = precheck()) return st;
@@ -492,7 +533,21 @@ ffn_status ffn_nvfp4_forward_lora(const void* x, int64_t m, int64_t hidden, int6
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   void* h = ws + c.h;
   cudaError_t e;
-  if (format == FFN_ACT_BF16 && w4a16_persistent(m)) {
+  if (planes) {
+    ffn::PlanesBuffers b;
+    b.h = h;
+    b.x_codes = ws + c.xq_c;
+    b.x_sf = ws + c.xq_s;
+    b.h_codes = ws + c.hq_c;
+    b.h_sf = ws + c.hq_s;
+    b.x_g = reinterpret_cast<float*>(ws + c.xg);
+    b.h_g = reinterpret_cast<float*>(ws + c.hg);
+    b.partials = ws + c.part;
+    b.counters = reinterpret_cast<int*>(ws + c.cnt);
+    b.xa_gu = ws + c.xa_gu;
+    b.xa_d = ws + c.xa_d;
+    e = ffn::launch_planes_ffn(x, m, gate_up->tc(), down->tc(), c.planes, b, out, s, lv);
+  } else if (format == FFN_ACT_BF16 && w4a16_persistent(m)) {
     e = ffn::launch_persist_ffn(x, m, gate_up->tc(), down->tc(), c.persist, h, ws + c.part,
                                 reinterpret_cast<int*>(ws + c.cnt), out, s, lv, ws + c.xa_gu, ws + c.xa_d);
   } else if (format == FFN_ACT_BF16 && w4a16_path(m) == Path::kTc) {
@@ -554,7 +609,15 @@ ffn_status ffn_nvfp4_projection_plan(int64_t m, int64_t n, int64_t k, ffn_act_fo
   *out = ffn_projection_plan{FFN_KERNEL_NONE, 0, 1, 0};
   if (m == 0) return FFN_OK;
   const int ncols = (int)(gate_up ? n / 2 : n);
-  if (format == FFN_ACT_BF16 && role != FFN_ROLE_LINEAR && w4a16_persistent(m)) {
+  const int forced = w4a16_forced();
+  if (format == FFN_ACT_BF16 && role != FFN_ROLE_LINEAR && (forced == 0 || forced == 4) &&
+      ffn::planes_for_rows(m) > 0 && (gate_up ? k : n) <= 24576 && (gate_up ? n / 2 : k) <= 24576) {
+    // (when both handles hold the natural tiled layout; else the tc_w4a16 row)
+    const ffn::PlanesPlan p = gate_up ? ffn::plan_planes(m, k, n / 2, num_sms()) : ffn::plan_planes(m, n, k, num_sms());
+    const int64_t W = gate_up ? (int64_t)p.gu_tiles * p.gu_kc : (int64_t)p.dn_tiles * p.dn_kc;
+    const int grid = gate_up ? p.gu_grid : p.dn_grid, kc = gate_up ? p.gu_kc : p.dn_kc;
+    *out = ffn_projection_plan{FFN_KERNEL_TC_PLANES, p.nt, (int)(((int64_t)kc * grid + W - 1) / W + 1), grid};
+  } else if (format == FFN_ACT_BF16 && role != FFN_ROLE_LINEAR && w4a16_persistent(m)) {
     // gate+up: n = 2 * inter, k = hidden; down: n = hidden, k = inter
     const ffn::PersistPlan p = gate_up ? ffn::plan_persist(m, k, n / 2, num_sms())
                                        : ffn::plan_persist(m, n, k, num_sms());
@@ -592,7 +655,7 @@ ffn_status ffn_nvfp4_workspace_size_lora(int64_t m, int64_t hidden, int64_t inte
   if (!bytes || m < 0) return FFN_ERR_INVALID_ARG;
   if (format != FFN_ACT_BF16 && format != FFN_ACT_NVFP4_FIXED) return FFN_ERR_INVALID_ARG;
   if (!valid_k(hidden) || !valid_k(inter)) return FFN_ERR_SHAPE;
-  *bytes = carve_ffn(m, hidden, inter, format, ffn::lora_view(lora).rank).total;
+  *bytes = ffn_workspace_bytes(m, hidden, inter, format, ffn::lora_view(lora).rank);
   return FFN_OK;
 }
 

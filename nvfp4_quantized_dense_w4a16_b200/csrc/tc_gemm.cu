@@ -1130,6 +1130,274 @@ tc_w4a4_kernel(const __grid_constant__ CUtensorMap xmap, const W4Args w4) {
   }
 }
 
+// ---------------------------------------------------------------------------
+// Few-row W4A16 projection on the block-scaled FP4 tensor core.  The weights
+// go to kind::mxf4nvf4 as stored (natural tiled chunks: codes are the A
+// operand, the chunk's 512-byte scale block is SFA) -- no software
+// dequantisation; the activation rows arrive as P NVFP4 planes per row (see
+// planes.cu), N = m * P columns, with their scale blocks as SFB.  The
+// epilogue folds the planes back, y[j, n] = sum_p g[j, p] * D[n, j*P + p].
+// Work: the (weight tile, 64-element chunk) space cut into one contiguous,
+// equal range per CTA (two CTAs per SM), each range a list of segments (one
+// per tile it touches); stages of up to 4 chunks never cross a segment.  Each
+// segment's fp32 partial sums go to the workspace, slot (CTA + tile); the CTA
+// that completes a tile's count (atomic, zeroed by the plane quantiser that
+// runs before) adds the tile's partials in K order and writes the output:
+// SiLU*mul into h for the fused gate+up weight, or bf16(gs * y) for down,
+// with LoRA deltas when given.  Two accumulators alternate between segments
+// so that a segment's epilogue overlaps the next segment's MMAs.
+// ---------------------------------------------------------------------------
+constexpr int kQChunks = 4;  // 64-element chunks per stage
+
+template <int NT>
+struct QCfg {
+  static constexpr int kXBytes = NT * 128;               // NT plane rows x 256 elements
+  static constexpr int kStageBytes = kW4Chunks * kChunkBytes + kXBytes + kQChunks * 512;
+  static constexpr int kStages = NT <= 32 ? 4 : 3;
+  static constexpr int kSmemBar = kStages * kStageBytes;
+  static constexpr int kNumBars = 2 * kStages + 4;       // full, empty, accfull[2], accfree[2]
+  static constexpr int kSmemAlloc = kSmemBar + kNumBars * 8 + 32 + 1024;
+  static constexpr int kAccCols = 2 * NT;
+  static constexpr int kSfaCol = kAccCols;
+  static constexpr int kSfbCol = kSfaCol + 4 * kQChunks * kStages;
+  static constexpr int kTmemNeed = kSfbCol + 4 * kQChunks * kStages;
+  static constexpr int kTmemCols = kTmemNeed <= 256 ? 256 : 512;
+  static_assert(kStageBytes % 1024 == 0, "stage alignment (128-byte swizzle)");
+  static_assert(2 * (kSmemAlloc + 1024) <= 233472, "two CTAs per SM");
+  static_assert(kTmemCols == 256, "two CTAs per SM share the 512 TMEM columns");
+  static_assert(NT % 16 == 0 && NT >= 16 && NT <= 64, "MMA N");
+};
+
+struct QArgs {
+  const uint8_t* wt;     // natural tiled weight [ntiles][kc][4608]
+  const float* gs;       // tensor scale(s)
+  uint16_t* out;         // bf16 [m, ldo]: h (gate+up) or out (down)
+  int m, n_out, ldo, kc, ntiles, planes;
+  const uint8_t* sfb;    // plane scale blocks [kc][512]
+  const float* g;        // plane factors [m][planes]
+  float* partials;       // [gridDim.x + ntiles][m][128]
+  int* counters;         // [ntiles], zero on entry
+  LoraArgs lora;
+};
+
+// Segment j of this CTA's equal range of the (tile, chunk) space.
+__device__ __forceinline__ bool range_segment(int ntiles, int kc, int j, Seg& s) {
+  const int G = gridDim.x, g = blockIdx.x;
+  const int64_t W = (int64_t)ntiles * kc;
+  const int64_t lo = W * g / G, hi = W * (g + 1) / G;
+  const int t = (int)(lo / kc) + j;
+  const int64_t b = lo > (int64_t)t * kc ? lo : (int64_t)t * kc;
+  const int64_t e = hi < (int64_t)(t + 1) * kc ? hi : (int64_t)(t + 1) * kc;
+  if (b >= e) return false;
+  s.tile = t;
+  s.c0 = (int)(b - (int64_t)t * kc);
+  s.nk = (int)(e - b);
+  return true;
+}
+
+template <int NT, int P, bool kGateUp>
+__global__ void __launch_bounds__(256, 2)
+tc_planes_kernel(const __grid_constant__ CUtensorMap xmap, const QArgs a) {
+  static_assert(NT % P == 0, "whole rows of planes per MMA");
+  constexpr int MR = NT / P;  // activation rows (m <= MR)
+  using C = QCfg<NT>;
+  constexpr int S = C::kStages;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::kSmemBar);
+  uint64_t* empty = full + S;
+  uint64_t* accfull = empty + S;   // [2]
+  uint64_t* accfree = accfull + 2; // [2]
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(accfree + 2);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  volatile int* last_flag = reinterpret_cast<volatile int*>(tmem_slot + 2);
+  int* err = &g_ffn_device_error;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < S; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&accfull[b], 1);
+      mbar_init(&accfree[b], 4);
+    }
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 2) {
+    tmem_alloc(tmem_slot, C::kTmemCols);
+    tmem_relinquish();
+  }
+  if (warp == 0 && lane == 0) tma_prefetch_desc(&xmap);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  griddep_launch_dependents();
+
+  if (warp == 0) {
+    // -------------------------- producer: weights, plane codes, plane scales
+    if (lane == 0) {
+      Seg sg;
+      int st_i = 0;
+      bool ok = true;
+      bool waited = false;
+      for (int j = 0; ok && range_segment(a.ntiles, a.kc, j, sg); ++j) {
+        for (int c = 0; c < sg.nk; c += kQChunks, ++st_i) {
+          const int s = st_i % S, nch = min(kQChunks, sg.nk - c);
+          if (st_i >= S && !mbar_wait(&empty[s], ((st_i / S) - 1) & 1, abort_flag, err, 1)) {
+            ok = false;
+            break;
+          }
+          uint8_t* st = smem + s * C::kStageBytes;
+          const int kchunk = sg.c0 + c;
+          mbar_arrive_expect_tx(&full[s], nch * (kChunkBytes + 512) + NT * 128);
+          bulk_load(st, a.wt + ((size_t)sg.tile * a.kc + kchunk) * kChunkBytes, nch * kChunkBytes, &full[s]);
+          if (!waited) {  // the planes come from the previous kernel
+            griddep_wait();
+            waited = true;
+          }
+          tma_load_2d(st + kW4Chunks * kChunkBytes, &xmap, 32 * kchunk, 0, &full[s]);
+          bulk_load(st + kW4Chunks * kChunkBytes + C::kXBytes, a.sfb + (size_t)kchunk * 512, nch * 512,
+                    &full[s]);
+        }
+      }
+      for (int i = max(0, st_i - S); i < st_i; ++i) wait_drain(&full[i % S], (i / S) & 1);
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      const uint32_t idesc = idesc_mxf4nvf4(kTileRows, NT);
+      Seg sg;
+      int st_i = 0;
+      bool ok = true;
+      for (int j = 0; ok && range_segment(a.ntiles, a.kc, j, sg); ++j) {
+        const int buf = j & 1;
+        if (j >= 2 && !mbar_wait(&accfree[buf], ((j >> 1) - 1) & 1, abort_flag, err, 2)) break;
+        tc_fence_after();
+        for (int c = 0; c < sg.nk; c += kQChunks, ++st_i) {
+          const int s = st_i % S, nch = min(kQChunks, sg.nk - c);
+          if (!mbar_wait(&full[s], (st_i / S) & 1, abort_flag, err, 2)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint8_t* st = smem + s * C::kStageBytes;
+          const uint64_t b_base = smem_desc_sw128(smem_u32(st + kW4Chunks * kChunkBytes));
+          for (int cc = 0; cc < nch; ++cc) {
+            const uint32_t slot = 4 * (s * kQChunks + cc);
+            const uint8_t* wc = st + cc * kChunkBytes;
+            tmem_cp_32x128b_x4(tmem + C::kSfaCol + slot, smem_desc_interleave(smem_u32(wc + 4096), 16, 128));
+            tmem_cp_32x128b_x4(tmem + C::kSfbCol + slot,
+                               smem_desc_interleave(smem_u32(st + kW4Chunks * kChunkBytes + C::kXBytes + 512 * cc),
+                                                    16, 128));
+            mma_mxf4nvf4(tmem + buf * NT, smem_desc_interleave(smem_u32(wc), 2048, 128), b_base + 2 * cc, idesc,
+                         tmem + C::kSfaCol + slot, tmem + C::kSfbCol + slot, (c | cc) != 0 ? 1u : 0u);
+          }
+          mma_commit(&empty[s]);
+        }
+        if (ok) mma_commit(&accfull[buf]);
+      }
+    }
+  } else if (warp >= 4) {
+    // ----------------------- segment epilogues and the split-K finalisation
+    const int q = warp & 3;
+    const int row = 32 * q + lane;
+    const int tid = threadIdx.x - 128;
+    const uint32_t lane_addr = (uint32_t)(32 * q) << 16;
+    bool waited = false;
+    Seg sg;
+    for (int j = 0; range_segment(a.ntiles, a.kc, j, sg); ++j) {
+      const int buf = j & 1;
+      const bool ok = __all_sync(0xffffffffu, wait_drain(&accfull[buf], (j >> 1) & 1));
+      tc_fence_after();
+      if (!waited) {
+        griddep_wait();  // the previous kernel may still read this kernel's outputs
+        waited = true;
+      }
+      if (!ok || *abort_flag) break;
+      uint32_t d[NT];
+#pragma unroll
+      for (int c = 0; c < NT / 16; ++c) {
+        uint32_t v[16];
+        tmem_ld16(tmem + lane_addr + buf * NT + 16 * c, v);
+#pragma unroll
+        for (int i = 0; i < 16; ++i) d[16 * c + i] = v[i];
+      }
+      tmem_ld_wait();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&accfree[buf]);  // the MMAs may reuse the accumulator
+      // fold the planes (p ascending): partial[slot][jr][row] = sum_p g[jr, p] * D[row, jr * P + p]
+      float* Pp = a.partials + (size_t)(blockIdx.x + sg.tile) * a.m * kTileRows;
+#pragma unroll
+      for (int jr = 0; jr < MR; ++jr) {
+        if (jr < a.m) {
+          float y = 0.0f;
+#pragma unroll
+          for (int p = 0; p < P; ++p) y = fmaf(__ldg(a.g + jr * P + p), __uint_as_float(d[jr * P + p]), y);
+          Pp[(size_t)jr * kTileRows + row] = y;
+        }
+      }
+      __threadfence();
+      named_bar_sync(1, 128);
+      if (tid == 0) {
+        const int64_t W = (int64_t)a.ntiles * a.kc;
+        const int G = gridDim.x;
+        const int g0 = range_owner((int64_t)sg.tile * a.kc, W, G);
+        const int g1 = range_owner((int64_t)sg.tile * a.kc + a.kc - 1, W, G);
+        *last_flag = atomicAdd(&a.counters[sg.tile], 1) == g1 - g0 ? 1 : 0;
+      }
+      named_bar_sync(1, 128);
+      if (*last_flag) {
+        __threadfence();
+        const int64_t W = (int64_t)a.ntiles * a.kc;
+        const int G = gridDim.x;
+        const int g0 = range_owner((int64_t)sg.tile * a.kc, W, G);
+        const int g1 = range_owner((int64_t)sg.tile * a.kc + a.kc - 1, W, G);
+        if (kGateUp) {
+          // h[jr, 64t + r] from gate row r and up row r + 64 of the tile
+          for (int idx = tid; idx < a.m * 64; idx += 128) {
+            const int jr = idx / 64, rr = idx % 64;
+            const int n = 64 * sg.tile + rr;
+            if (n >= a.n_out) continue;
+            float gsum = 0.0f, usum = 0.0f;
+            for (int gg = g0; gg <= g1; ++gg) {
+              const float* Pt = a.partials + ((size_t)(gg + sg.tile) * a.m + jr) * kTileRows;
+              gsum += __ldcg(Pt + rr);
+              usum += __ldcg(Pt + rr + 64);
+            }
+            const float gv = lora_add(bf16_round(a.gs[0] * gsum), a.lora.b0, a.lora.off0, a.lora, jr, n);
+            const float uv = lora_add(bf16_round(a.gs[1] * usum), a.lora.b1, a.lora.off1, a.lora, jr, n);
+            a.out[(size_t)jr * a.ldo + n] = f32_to_bf16_bits(silu_fast(gv) * uv);
+          }
+        } else {
+          for (int idx = tid; idx < a.m * kTileRows; idx += 128) {
+            const int jr = idx / kTileRows, rr = idx % kTileRows;
+            const int n = kTileRows * sg.tile + rr;
+            if (n >= a.n_out) continue;
+            float sum = 0.0f;
+            for (int gg = g0; gg <= g1; ++gg)
+              sum += __ldcg(a.partials + ((size_t)(gg + sg.tile) * a.m + jr) * kTileRows + rr);
+            float y = a.gs[0] * sum;
+            if (a.lora.b0) y = lora_add(bf16_round(y), a.lora.b0, a.lora.off0, a.lora, jr, n);
+            a.out[(size_t)jr * a.ldo + n] = f32_to_bf16_bits(y);
+          }
+        }
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 2) {
+    tc_fence_after();
+    tmem_dealloc(tmem, C::kTmemCols);
+  }
+}
+
 // Split-K reduction in a fixed order (z = 0, 1, ...), then the epilogue.
 template <bool kGateUp>
 __global__ void splitk_reduce_kernel(const float* __restrict__ P, int splits, int m, int n_pad,
@@ -1345,9 +1613,127 @@ cudaError_t launch_persist_bn(int bn, const CUtensorMap& map, const PArgs& a, in
   }
 }
 
+template <int NT, int P, bool kGateUp>
+cudaError_t launch_planes_cfg(const CUtensorMap& map, const QArgs& a, int grid, cudaStream_t s) {
+  using C = QCfg<NT>;
+  auto kern = tc_planes_kernel<NT, P, kGateUp>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemAlloc);
+  if (e != cudaSuccess) return e;
+  return launch_pdl(kern, dim3(grid), dim3(256), C::kSmemAlloc, s, map, a);
+}
+
+template <bool kGateUp>
+cudaError_t launch_planes_nt(int nt, int planes, const CUtensorMap& map, const QArgs& a, int grid,
+                             cudaStream_t s) {
+  if (planes == 16) return launch_planes_cfg<16, 16, kGateUp>(map, a, grid, s);
+  if (nt == 16) return launch_planes_cfg<16, 8, kGateUp>(map, a, grid, s);
+  if (nt == 32) return launch_planes_cfg<32, 8, kGateUp>(map, a, grid, s);
+  return launch_planes_cfg<64, 8, kGateUp>(map, a, grid, s);
+}
+
+// 2-D map over plane codes [rows, k/2] bytes with a 128-byte x nt-row box and
+// the 128-byte swizzle (the MMA's B operand layout).
+bool make_planes_map(CUtensorMap* map, const void* codes, int64_t rows, int64_t k, int nt) {
+  auto enc = get_encode();
+  if (!enc) return false;
+  cuuint64_t dims[2] = {(cuuint64_t)(k / 2), (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)(k / 2)};
+  cuuint32_t box[2] = {128, (cuuint32_t)nt};
+  cuuint32_t estr[2] = {1, 1};
+  return enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(codes), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 }  // namespace
 
 int tc_tile_bytes_per_row_chunk() { return kChunkBytes; }
+
+PlanesPlan plan_planes(int64_t m, int64_t hidden, int64_t inter, int num_sms) {
+  PlanesPlan p;
+  p.planes = planes_for_rows(m);
+  if (!p.planes) return p;
+  const int64_t cols = m * p.planes;
+  p.nt = cols <= 16 ? 16 : cols <= 32 ? 32 : 64;
+  p.gu_tiles = (int)((inter + 63) / 64);
+  p.gu_kc = (int)((hidden + kChunkK - 1) / kChunkK);
+  p.dn_tiles = (int)((hidden + kTileRows - 1) / kTileRows);
+  p.dn_kc = (int)((inter + kChunkK - 1) / kChunkK);
+  const int64_t slots = 2LL * num_sms, Wg = (int64_t)p.gu_tiles * p.gu_kc, Wd = (int64_t)p.dn_tiles * p.dn_kc;
+  p.gu_grid = (int)(Wg < slots ? Wg : slots);
+  p.dn_grid = (int)(Wd < slots ? Wd : slots);
+  const size_t pg = (size_t)(p.gu_grid + p.gu_tiles) * m * kTileRows * sizeof(float);
+  const size_t pd = (size_t)(p.dn_grid + p.dn_tiles) * m * kTileRows * sizeof(float);
+  p.partial_bytes = pg > pd ? pg : pd;
+  p.counter_count = p.gu_tiles + p.dn_tiles;
+  return p;
+}
+
+cudaError_t launch_planes_ffn(const void* x, int64_t m, const TcWeight& gate_up, const TcWeight& down,
+                              const PlanesPlan& p, const PlanesBuffers& b, void* out, cudaStream_t s,
+                              const LoraView& lv) {
+  const int64_t hidden = down.n, inter = gate_up.n / 2;
+  const int rows = (int)(m * p.planes);
+  CUtensorMap xm, hm;
+  if (!make_planes_map(&xm, b.x_codes, rows, hidden, p.nt) || !make_planes_map(&hm, b.h_codes, rows, inter, p.nt))
+    return cudaErrorInvalidValue;
+  int* gu_cnt = b.counters;
+  int* dn_cnt = b.counters + p.gu_tiles;
+  cudaError_t e = launch_quantize_planes(x, m, hidden, p.planes, b.x_codes, b.x_sf, b.x_g, gu_cnt, p.gu_tiles, s);
+  QArgs a{};
+  a.wt = gate_up.tiled;
+  a.gs = gate_up.gs;
+  a.out = static_cast<uint16_t*>(b.h);
+  a.m = (int)m;
+  a.n_out = (int)inter;
+  a.ldo = (int)inter;
+  a.kc = p.gu_kc;
+  a.ntiles = p.gu_tiles;
+  a.planes = p.planes;
+  a.sfb = static_cast<const uint8_t*>(b.x_sf);
+  a.g = b.x_g;
+  a.partials = static_cast<float*>(b.partials);
+  a.counters = gu_cnt;
+  if (e == cudaSuccess && lv.rank > 0 && lv.a_gu) {
+    e = launch_lora_xa(x, m, hidden, lv.a_gu, 2 * lv.rank, b.xa_gu, s);
+    a.lora.xa = static_cast<const uint16_t*>(b.xa_gu);
+    a.lora.xa_ld = 2 * lv.rank;
+    a.lora.b0 = lv.b_g;
+    a.lora.b1 = lv.b_u;
+    a.lora.off1 = lv.rank;
+    a.lora.r = lv.rank;
+  }
+  if (e == cudaSuccess) {
+    ProfScope prof(s, "tc_planes_gate_up_silu");
+    e = launch_planes_nt<true>(p.nt, p.planes, xm, a, p.gu_grid, s);
+  }
+  if (e == cudaSuccess)
+    e = launch_quantize_planes(b.h, m, inter, p.planes, b.h_codes, b.h_sf, b.h_g, dn_cnt, p.dn_tiles, s);
+  QArgs d{};
+  d.wt = down.tiled;
+  d.gs = down.gs;
+  d.out = static_cast<uint16_t*>(out);
+  d.m = (int)m;
+  d.n_out = (int)hidden;
+  d.ldo = (int)hidden;
+  d.kc = p.dn_kc;
+  d.ntiles = p.dn_tiles;
+  d.planes = p.planes;
+  d.sfb = static_cast<const uint8_t*>(b.h_sf);
+  d.g = b.h_g;
+  d.partials = static_cast<float*>(b.partials);
+  d.counters = dn_cnt;
+  if (e == cudaSuccess && lv.rank > 0 && lv.a_d) {
+    e = launch_lora_xa(b.h, m, inter, lv.a_d, lv.rank, b.xa_d, s);
+    d.lora.xa = static_cast<const uint16_t*>(b.xa_d);
+    d.lora.xa_ld = lv.rank;
+    d.lora.b0 = lv.b_d;
+    d.lora.r = lv.rank;
+  }
+  if (e != cudaSuccess) return e;
+  ProfScope prof(s, "tc_planes_down");
+  return launch_planes_nt<false>(p.nt, p.planes, hm, d, p.dn_grid, s);
+}
 
 PersistPlan plan_persist(int64_t m, int64_t hidden, int64_t inter, int num_sms) {
   PersistPlan p;

@@ -39,7 +39,7 @@ class ProjectionPlan(ctypes.Structure):
 
 
 KERNEL_FAMILIES = {0: "none", 1: "tc_w4a16", 2: "tc_w4a4", 3: "gemv_w4a16", 4: "gemv_w4a4",
-                   5: "tc_w4a16_persistent"}
+                   5: "tc_w4a16_persistent", 6: "tc_planes"}
 ROLES = {"linear": 0, "gate_up": 1, "down": 2}
 
 

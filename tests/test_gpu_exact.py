@@ -52,9 +52,9 @@ def exact_weight(rng, n, k, scale_bytes=POW2_SCALES, zero_block_p=0.02):
     return codes, scales
 
 
-def make_handle(native, codes, scales):
+def make_handle(native, codes, scales, formats="all"):
     return native.ffn_nvfp4_weight_create(torch.from_numpy(codes).cuda(), torch.from_numpy(scales).cuda(),
-                                          torch.ones(1, dtype=torch.float32, device="cuda"))
+                                          torch.ones(1, dtype=torch.float32, device="cuda"), formats=formats)
 
 
 W4A16_CASES = [
@@ -163,20 +163,23 @@ def exact_ffn_inputs(rng, m, H, I, down_nonzeros=4):
 
 
 FFN_EXACT_CASES = [
-    # (m, hidden, inter): few-row persistent kernels for m <= 64 (tile widths
-    # 16/32/64; down K ranges that cut tiles, inter % 64 == 32), per-tile
-    # kernels with split-K and the SiLU*mul reduction for wider m
-    (1, 512, 1536), (5, 1024, 4096), (16, 512, 800), (33, 512, 1536), (64, 1024, 2048),
-    (100, 512, 1536), (300, 512, 800),
+    # (m, hidden, inter, handle formats): m <= 8 with both layouts runs the
+    # block-scaled FP4 kernels with activation planes (m = 1: 16 planes; 2..8:
+    # 8), bf16-only handles the per-tile kernels at the same m; tile widths
+    # 16/32/64 per-tile, down K ranges that cut tiles, inter % 64 == 32, and
+    # split-K with the SiLU*mul reduction for wider m
+    (1, 512, 1536, "all"), (2, 512, 800, "all"), (5, 1024, 4096, "all"), (8, 512, 1536, "all"),
+    (1, 512, 1536, "bf16"), (5, 1024, 4096, "bf16"), (16, 512, 800, "all"), (33, 512, 1536, "all"),
+    (64, 1024, 2048, "all"), (100, 512, 1536, "all"), (300, 512, 800, "all"),
 ]
 
 
-@pytest.mark.parametrize("m,H,I", FFN_EXACT_CASES)
-def test_ffn_exact_inputs_bit_exact(native, m, H, I):
+@pytest.mark.parametrize("m,H,I,formats", FFN_EXACT_CASES)
+def test_ffn_exact_inputs_bit_exact(native, m, H, I, formats):
     rng = np.random.default_rng(3000 + m + H + I)
     x, qg, qu, qd = exact_ffn_inputs(rng, m, H, I)
     ref = O.ffn_w4a16(x.astype(np.float64), qg, qu, qd)
-    hs = [make_handle(native, q[0], q[1]) for q in (qg, qu, qd)]
+    hs = [make_handle(native, q[0], q[1], formats) for q in (qg, qu, qd)]
     gate_up = native.ffn_nvfp4_weight_create_gate_up(hs[0], hs[1])
     out = native.ffn_nvfp4_forward(torch.from_numpy(x).cuda().to(torch.bfloat16), gate_up, hs[2], "bf16")
     torch.cuda.synchronize()
@@ -197,8 +200,8 @@ def test_persistent_path_bit_exact_in_subprocess(native):
         "import sys; sys.path.insert(0, 'tests'); sys.path.insert(0, '.');"
         "import test_gpu_exact as T; from nvfp4_quantized_dense_w4a16_b200 import native as N;"
         "assert N.ffn_nvfp4_projection_plan(5, 1024, 4096, role='down')['family'] == 'tc_w4a16_persistent';"
-        "[T.test_ffn_exact_inputs_bit_exact(N, *c) for c in [(1, 512, 1536), (5, 1024, 4096), (16, 512, 800),"
-        " (33, 512, 1536), (64, 1024, 2048)]]; print('persistent-ok')")
+        "[T.test_ffn_exact_inputs_bit_exact(N, *c, 'all') for c in [(1, 512, 1536), (5, 1024, 4096),"
+        " (16, 512, 800), (33, 512, 1536), (64, 1024, 2048)]]; print('persistent-ok')")
     root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
     r = subprocess.run([sys.executable, "-c", code], cwd=root, capture_output=True, text=True, timeout=900,
                        env=dict(os.environ, FFN_NVFP4_W4A16_PATH="persistent"))
