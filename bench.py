@@ -382,7 +382,7 @@ def time_steps(N, wl, steps, flush, eager, barrier):
 
     Default: the steps are captured in one CUDA graph with a timing-event pair
     around each step, replayed once untimed and once timed; per-kernel
-    durations come from a second graph of the same steps with an event pair
+    durations come from launching the same steps directly with an event pair
     around every kernel (events between kernels also keep them from
     overlapping, which is why the timed graph has none).  With `eager` (for
     runs under a profiler) the steps are launched directly and timed with the
@@ -408,28 +408,28 @@ def time_steps(N, wl, steps, flush, eager, barrier):
     barrier()
     ms = sum(a.elapsed_time(b) for a, b in zip(starts, stops))
     del graph
-    pgraph, _, _ = capture_steps(N, wl, steps, flush, profile=True)
-    pgraph.replay()
-    barrier()
-    pgraph.replay()
+    # per-kernel durations: the same steps launched directly with an event
+    # pair around every kernel (recorded on the stream in front of and behind
+    # each launch, so each pair brackets that kernel's own execution)
+    N.ffn_nvfp4_profile_begin()
+    for i in range(steps):
+        if flush is not None:
+            flush.zero_()
+        wl.step(i)
     barrier()
     prof = N.ffn_nvfp4_profile_end()
-    del pgraph
     return ms, prof
 
 
-def capture_steps(N, wl, steps, flush, profile=False):
+def capture_steps(N, wl, steps, flush):
     """Capture `steps` forward steps (each after an optional L2 flush, between
     a pair of timing events) into one CUDA graph, so every timestamp is taken
-    on the device during replay and none includes host launch latency.  With
-    `profile`, the library's per-kernel events are captured too (the recording
-    stays open until ffn_nvfp4_profile_end).  Returns (graph, starts, stops)."""
+    on the device during replay and none includes host launch latency.
+    Returns (graph, starts, stops)."""
     import torch
     starts = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(steps)]
     stops = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(steps)]
     graph = torch.cuda.CUDAGraph()
-    if profile:
-        N.ffn_nvfp4_profile_begin()
     with torch.cuda.graph(graph, stream=torch.cuda.Stream()):
         for i in range(steps):
             if flush is not None:
@@ -577,7 +577,8 @@ def main():
                    "parallelism": f"replicas x{world}", "l2": res["l2"], "weight_layouts": res["layouts"],
                    "launch": ("eager launches" if args.eager else
                               "the K timed steps captured in one CUDA graph, replayed once; "
-                              "kernel durations from a second replay with an event pair per kernel")},
+                              "kernel durations from the same steps launched directly with an event "
+                              "pair per kernel")},
         "roofline": res["roofline"], "cpu_baseline": cpu, "e2e": res["e2e"],
         "gpu_launches": res["gpu_launches"], "kernels": res["kernels"], "clocks": res["clocks"],
     }

@@ -290,9 +290,9 @@ typedef enum ffn_kernel_family {
                                 (built for the fixed format too, e.g.
                                 FFN_FORMAT_ALL): the NVFP4 weights go to the
                                 block-scaled FP4 MMA as stored and each
-                                activation row as 8 or 16 NVFP4 residual planes
-                                (N = 8m or 16 columns, exact for bf16 rows of
-                                normal spread); equal K ranges per CTA, two
+                                activation row as 8 NVFP4 residual planes
+                                (N = 8m columns, at least 16; exact for bf16
+                                rows of normal spread); equal K ranges per CTA, two
                                 CTAs per SM, split-K sums added in-kernel.
                                 tile_rows reports the MMA's N.  Without the
                                 natural layout the layer takes FFN_KERNEL_TC_W4A16. */

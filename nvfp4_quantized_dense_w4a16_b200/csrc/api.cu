@@ -105,8 +105,9 @@ bool w4a16_persistent(int64_t m) { return w4a16_forced() == 3 && m <= ffn::kPers
 bool w4a16_planes(int64_t m, int64_t hidden, int64_t inter, const ffn_nvfp4_weight* gu,
                   const ffn_nvfp4_weight* dn) {
   const int f = w4a16_forced();
-  return (f == 0 || f == 4) && ffn::planes_for_rows(m) > 0 && hidden <= 24576 && inter <= 24576 &&
-         gu && dn && gu->tiled && dn->tiled;
+  (void)hidden;
+  (void)inter;
+  return (f == 0 || f == 4) && ffn::planes_for_rows(m) > 0 && gu && dn && gu->tiled && dn->tiled;
 }
 
 // Fixed format: the block-scaled FP4 tensor-core kernel, or the CUDA-core one
@@ -234,8 +235,7 @@ Carve carve_ffn(int64_t m, int64_t hidden, int64_t inter, ffn_act_format f, int6
 size_t ffn_workspace_bytes(int64_t m, int64_t hidden, int64_t inter, ffn_act_format f, int64_t lora_rank) {
   size_t b = carve_ffn(m, hidden, inter, f, lora_rank, false).total;
   const int forced = w4a16_forced();
-  if (f == FFN_ACT_BF16 && (forced == 0 || forced == 4) && ffn::planes_for_rows(m) > 0 && hidden <= 24576 &&
-      inter <= 24576) {
+  if (f == FFN_ACT_BF16 && (forced == 0 || forced == 4) && ffn::planes_for_rows(m) > 0) {
     const size_t bp = carve_ffn(m, hidden, inter, f, lora_rank, true).total;
     if (bp > b) b = bp;
   }
@@ -611,7 +611,7 @@ ffn_status ffn_nvfp4_projection_plan(int64_t m, int64_t n, int64_t k, ffn_act_fo
   const int ncols = (int)(gate_up ? n / 2 : n);
   const int forced = w4a16_forced();
   if (format == FFN_ACT_BF16 && role != FFN_ROLE_LINEAR && (forced == 0 || forced == 4) &&
-      ffn::planes_for_rows(m) > 0 && (gate_up ? k : n) <= 24576 && (gate_up ? n / 2 : k) <= 24576) {
+      ffn::planes_for_rows(m) > 0) {
     // (when both handles hold the natural tiled layout; else the tc_w4a16 row)
     const ffn::PlanesPlan p = gate_up ? ffn::plan_planes(m, k, n / 2, num_sms()) : ffn::plan_planes(m, n, k, num_sms());
     const int64_t W = gate_up ? (int64_t)p.gu_tiles * p.gu_kc : (int64_t)p.dn_tiles * p.dn_kc;

@@ -1625,7 +1625,7 @@ cudaError_t launch_planes_cfg(const CUtensorMap& map, const QArgs& a, int grid, 
 template <bool kGateUp>
 cudaError_t launch_planes_nt(int nt, int planes, const CUtensorMap& map, const QArgs& a, int grid,
                              cudaStream_t s) {
-  if (planes == 16) return launch_planes_cfg<16, 16, kGateUp>(map, a, grid, s);
+  (void)planes;  // 8 per row
   if (nt == 16) return launch_planes_cfg<16, 8, kGateUp>(map, a, grid, s);
   if (nt == 32) return launch_planes_cfg<32, 8, kGateUp>(map, a, grid, s);
   return launch_planes_cfg<64, 8, kGateUp>(map, a, grid, s);
