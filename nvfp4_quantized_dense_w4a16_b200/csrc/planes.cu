@@ -29,7 +29,8 @@
 namespace ffn {
 namespace {
 
-constexpr int kPlaneThreads = 256;  // one 16-element block per thread
+constexpr int kPlaneThreads = 128;  // four threads per 16-element block
+constexpr int kBlocksPerCta = kPlaneThreads / 4;
 constexpr int kPlanes = 8;
 
 __device__ __forceinline__ float block_reduce_max(float v, float* red) {
@@ -44,13 +45,18 @@ __device__ __forceinline__ float block_reduce_max(float v, float* red) {
   return m;
 }
 
-// grid (m, ceil(K / 16 / 256)): CTA (j, c) handles the 16-element blocks
-// 256c .. 256c + 255 of row j, after reading the whole row for its maximum
-// (every CTA of the row finds the same E).  Outputs: codes [m * P][K/2]
-// (row j * P + p), scale bytes in the blocked layout of the MMA's
-// scale-factor copy (rows j * P + p), g [m][P] (fp32).  After its
-// griddep_wait the kernel also zeroes the counters of the projection that
-// follows it, if given.
+// 2^k as fp32 (exact; built from the exponent bits in the normal range).
+__device__ __forceinline__ float exp2i(int k) {
+  return k >= -126 && k <= 127 ? __int_as_float((k + 127) << 23) : ldexpf(1.0f, k);
+}
+
+// grid (m, ceil(K / 16 / 32)): CTA (j, c) handles the 16-element blocks
+// 32c .. 32c + 31 of row j, four threads per block (four elements each),
+// after reading the whole row for its maximum (every CTA of the row finds the
+// same E).  Outputs: codes [m * P][K/2] (row j * P + p), scale bytes in the
+// blocked layout of the MMA's scale-factor copy (rows j * P + p), g [m][P]
+// (fp32).  After its griddep_wait the kernel also zeroes the counters of the
+// projection that follows it, if given.
 __global__ void __launch_bounds__(kPlaneThreads) quantize_planes_kernel(
     const uint16_t* __restrict__ x, int m, int K, uint8_t* __restrict__ codes,
     uint8_t* __restrict__ sf_blocks, float* __restrict__ g, int* zero_ptr, int zero_count) {
@@ -75,49 +81,46 @@ __global__ void __launch_bounds__(kPlaneThreads) quantize_planes_kernel(
   const float rowmax = block_reduce_max(local, red);
   const int E = rowmax > 0.0f ? ilogbf(rowmax) : 0;
   if (blockIdx.y == 0 && threadIdx.x < kPlanes)
-    g[j * kPlanes + threadIdx.x] = rowmax > 0.0f ? ldexpf(1.0f, E - 8 - (3 * (int)threadIdx.x) / 2) : 0.0f;
-  const int b = blockIdx.y * kPlaneThreads + threadIdx.x;
-  if (b >= nb) return;
-  float r[16];
-  {
-    const uint4* src = reinterpret_cast<const uint4*>(row + 16 * b);
-    const uint4 a = src[0], c = src[1];
-    const uint32_t w[8] = {a.x, a.y, a.z, a.w, c.x, c.y, c.z, c.w};
-#pragma unroll
-    for (int e = 0; e < 8; ++e) {
-      r[2 * e] = bf16_bits_to_float(w[e] & 0xffffu);
-      r[2 * e + 1] = bf16_bits_to_float(w[e] >> 16);
-    }
+    g[j * kPlanes + threadIdx.x] = rowmax > 0.0f ? exp2i(E - 8 - (3 * (int)threadIdx.x) / 2) : 0.0f;
+  const int b = blockIdx.y * kBlocksPerCta + (threadIdx.x >> 2);
+  const int part = threadIdx.x & 3;  // elements 4 part .. 4 part + 3 of the block
+  const bool valid = b < nb;         // whole groups of four lanes share validity
+  float r[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+  if (valid) {
+    const uint2 v = *reinterpret_cast<const uint2*>(row + 16 * b + 4 * part);
+    r[0] = bf16_bits_to_float(v.x & 0xffffu);
+    r[1] = bf16_bits_to_float(v.x >> 16);
+    r[2] = bf16_bits_to_float(v.y & 0xffffu);
+    r[3] = bf16_bits_to_float(v.y >> 16);
   }
 #pragma unroll 1
   for (int p = 0; p < kPlanes; ++p) {
-    const int rowp = j * kPlanes + p;
-    float amax = 0.0f;
-#pragma unroll
-    for (int e = 0; e < 16; ++e) amax = fmaxf(amax, fabsf(r[e]));
-    uint32_t s8 = 0, lo = 0, hi = 0;
+    float amax = fmaxf(fmaxf(fabsf(r[0]), fabsf(r[1])), fmaxf(fabsf(r[2]), fabsf(r[3])));
+    amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
+    amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
+    uint32_t s8 = 0, nib = 0;
     if (amax > 0.0f) {
       const int ge = E - 8 - (3 * p) / 2;  // log2 g_p
       // smallest power of two 2^e >= amax / 6 / g_p, clamped to E4M3's 2^-9..2^8
       int ex;
-      const float fr = frexpf(__fdiv_rn(ldexpf(amax, -ge), 6.0f), &ex);  // = fr * 2^ex, fr in [0.5, 1)
+      const float fr = frexpf(__fdiv_rn(amax * exp2i(-ge), 6.0f), &ex);  // = fr * 2^ex, fr in [0.5, 1)
       int e = fr == 0.5f ? ex - 1 : ex;
       e = e < -9 ? -9 : (e > 8 ? 8 : e);
       s8 = e >= -6 ? (uint32_t)(e + 7) << 3 : (1u << (e + 9));
       // r / (g_p * 2^e) and the represented values are exact power-of-two scalings
+      const float down = exp2i(-(ge + e)), up = exp2i(ge + e);
 #pragma unroll
-      for (int i = 0; i < 16; ++i) {
-        const uint32_t q = e2m1_encode(ldexpf(r[i], -(ge + e)));
-        const float v = (q & 8u ? -1.0f : 1.0f) * e2m1_mag(q & 7u);
-        r[i] -= ldexpf(v, ge + e);
-        if (i < 8)
-          lo |= q << (4 * i);
-        else
-          hi |= q << (4 * (i - 8));
+      for (int i = 0; i < 4; ++i) {
+        const uint32_t q = e2m1_encode(r[i] * down);
+        r[i] -= ((q & 8u) ? -e2m1_mag(q & 7u) : e2m1_mag(q & 7u)) * up;
+        nib |= q << (4 * i);
       }
     }
-    *reinterpret_cast<uint2*>(codes + (size_t)rowp * (K / 2) + 8 * b) = make_uint2(lo, hi);
-    sf_blocks[sf_blocked_offset(rowp, b, kc)] = (uint8_t)s8;
+    if (valid) {
+      const int rowp = j * kPlanes + p;
+      *reinterpret_cast<uint16_t*>(codes + (size_t)rowp * (K / 2) + 8 * b + 2 * part) = (uint16_t)nib;
+      if (part == 0) sf_blocks[sf_blocked_offset(rowp, b, kc)] = (uint8_t)s8;
+    }
   }
 }
 
@@ -130,7 +133,7 @@ cudaError_t launch_quantize_planes(const void* x, int64_t m, int64_t k, int plan
                                    float* g, int* zero_ptr, int zero_count, cudaStream_t s) {
   if (planes != kPlanes || k % 16) return cudaErrorInvalidValue;
   ProfScope prof(s, "quantize_planes");
-  const dim3 grid((unsigned)m, (unsigned)((k / 16 + kPlaneThreads - 1) / kPlaneThreads));
+  const dim3 grid((unsigned)m, (unsigned)((k / 16 + kBlocksPerCta - 1) / kBlocksPerCta));
   return launch_pdl(quantize_planes_kernel, grid, dim3(kPlaneThreads), 0, s, static_cast<const uint16_t*>(x),
                     (int)m, (int)k, static_cast<uint8_t*>(codes), static_cast<uint8_t*>(sf_blocks), g, zero_ptr,
                     zero_count);

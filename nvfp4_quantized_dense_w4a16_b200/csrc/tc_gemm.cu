@@ -258,7 +258,7 @@ __device__ __forceinline__ bool wait_drain(uint64_t* bar, uint32_t parity) {
 // codes = E2M1(h / s), the same arithmetic as the activation quantiser).
 // Stores are staged through shared memory (ebuf, 16 KB per warpgroup) so that
 // global writes are 16-byte and row-contiguous.
-template <int BN, int EPI, int NG, int NACC = 1>
+template <int BN, int EPI, int NG, int NACC = 1, bool LORA = false>
 __device__ __forceinline__ void epilogue_tile(const TcArgs& a, uint32_t tmem, int q, int lane,
                                               int g, uint8_t* ebuf, int xtile, int wtile,
                                               int nacc_used = 1, float gs_mul = 1.0f) {
@@ -298,7 +298,7 @@ __device__ __forceinline__ void epilogue_tile(const TcArgs& a, uint32_t tmem, in
       uint16_t* T = reinterpret_cast<uint16_t*>(ebuf);  // [32][128] bf16
       const float gs = a.gs[0] * gs_mul;
       const int64_t nrow = (int64_t)kTileRows * wtile + row;
-      const bool lv = a.lora.b0 != nullptr && nrow < a.n_out;
+      const bool lv = LORA && a.lora.b0 != nullptr && nrow < a.n_out;
 #pragma unroll
       for (int j = 0; j < 32; ++j) {
         float y = gs * __uint_as_float(v[j]);
@@ -321,7 +321,7 @@ __device__ __forceinline__ void epilogue_tile(const TcArgs& a, uint32_t tmem, in
       if (q >= 2) {
         const float gsu = a.gs[1] * gs_mul;
         const int64_t nu = 64 * (int64_t)wtile + row - 64;
-        const bool lv = a.lora.b1 != nullptr && nu < a.n_out;
+        const bool lv = LORA && a.lora.b1 != nullptr && nu < a.n_out;
 #pragma unroll
         for (int j = 0; j < 32; ++j) {
           float uv = bf16_round(gsu * __uint_as_float(v[j]));
@@ -333,7 +333,7 @@ __device__ __forceinline__ void epilogue_tile(const TcArgs& a, uint32_t tmem, in
       if (q < 2) {
         const float gsg = a.gs[0] * gs_mul;
         const int64_t ng = 64 * (int64_t)wtile + row;
-        const bool lv = a.lora.b0 != nullptr && ng < a.n_out;
+        const bool lv = LORA && a.lora.b0 != nullptr && ng < a.n_out;
 #pragma unroll
         for (int j = 0; j < 32; ++j) {
           float gv = bf16_round(gsg * __uint_as_float(v[j]));
@@ -374,7 +374,8 @@ __device__ __forceinline__ void epilogue_tile(const TcArgs& a, uint32_t tmem, in
   }
 }
 
-template <int BN, int SXS, int XC, int SWS, int SA, int DQG, int UA, int NI, bool DQX, int EPI>
+template <int BN, int SXS, int XC, int SWS, int SA, int DQG, int UA, int NI, bool DQX, int EPI,
+          bool LORA = false>
 __global__ void __launch_bounds__(TcCfg<BN, SXS, XC, SWS, SA, DQG, UA, NI, DQX>::kThreads,
                                   TcCfg<BN, SXS, XC, SWS, SA, DQG, UA, NI, DQX>::kMinBlocks)
 tc_w4a16_kernel(const __grid_constant__ CUtensorMap xmap, const TcArgs a) {
@@ -541,7 +542,7 @@ tc_w4a16_kernel(const __grid_constant__ CUtensorMap xmap, const TcArgs a) {
     tc_fence_after();
     griddep_wait();  // the previous kernel may still read the output buffer
     if (done && !*abort_flag)
-      epilogue_tile<BN, EPI, DQG, NI>(a, tmem, q, lane, g, epi + g * C::kEpiBytes, xtile, wtile,
+      epilogue_tile<BN, EPI, DQG, NI, LORA>(a, tmem, q, lane, g, epi + g * C::kEpiBytes, xtile, wtile,
                                       min(NI, nunits), kW4A16Unscale);
   }
   tc_fence_before();
@@ -1544,7 +1545,11 @@ bool make_x_map(CUtensorMap* map, const void* x, int64_t m, int64_t k, int box_r
 template <int BN, int SXS, int XC, int SWS, int SA, int DQG, int UA, int NI, bool DQX, int EPI>
 cudaError_t launch_cfg(const CUtensorMap& map, const TcArgs& a, dim3 grid, cudaStream_t s) {
   using C = TcCfg<BN, SXS, XC, SWS, SA, DQG, UA, NI, DQX>;
-  auto kern = tc_w4a16_kernel<BN, SXS, XC, SWS, SA, DQG, UA, NI, DQX, EPI>;
+  // the LoRA epilogue is a separate instantiation: its code must not weigh on
+  // the plain epilogue (registers, instruction cache)
+  const bool lora = EPI != kEpiPartial && (a.lora.b0 || a.lora.b1);
+  auto kern = lora ? tc_w4a16_kernel<BN, SXS, XC, SWS, SA, DQG, UA, NI, DQX, EPI, EPI != kEpiPartial>
+                   : tc_w4a16_kernel<BN, SXS, XC, SWS, SA, DQG, UA, NI, DQX, EPI, false>;
   // The attribute belongs to the current device's context, so it is set on
   // every launch (a host-side call): correct on any device and after a reset.
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemAlloc);
