@@ -39,8 +39,10 @@ constexpr int kXaKTile = 256;  // K elements staged per pass
 __global__ void __launch_bounds__(kXaRows * 32) lora_xa_kernel(const uint16_t* __restrict__ x, int m,
                                                                int64_t K, const uint16_t* __restrict__ A,
                                                                int R, uint16_t* __restrict__ xa) {
-  asm volatile("griddepcontrol.wait;" ::: "memory");  // x may come from the previous kernel
+  // the next kernel may launch now: it waits for this one before reading
+  // its results; x may come from the previous kernel
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  asm volatile("griddepcontrol.wait;" ::: "memory");
   __shared__ __align__(16) uint16_t As[kXaOuts][kXaKTile];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int j = blockIdx.x * kXaRows + warp;

@@ -29,8 +29,8 @@
 namespace ffn {
 namespace {
 
-constexpr int kPlaneThreads = 128;  // four threads per 16-element block
-constexpr int kBlocksPerCta = kPlaneThreads / 4;
+constexpr int kPlaneThreads = 128;  // eight threads per 16-element block
+constexpr int kBlocksPerCta = kPlaneThreads / 8;
 constexpr int kPlanes = 8;
 
 __device__ __forceinline__ float block_reduce_max(float v, float* red) {
@@ -50,18 +50,29 @@ __device__ __forceinline__ float exp2i(int k) {
   return k >= -126 && k <= 127 ? __int_as_float((k + 127) << 23) : ldexpf(1.0f, k);
 }
 
-// grid (m, ceil(K / 16 / 32)): CTA (j, c) handles the 16-element blocks
-// 32c .. 32c + 31 of row j, four threads per block (four elements each),
+// Smallest e with 6 * 2^e >= a, for a > 0 normal: with a in [2^k, 2^(k+1)),
+// e = k - 2 when a <= 1.5 * 2^k (6 * 2^(k-2) = 1.5 * 2^k), else k - 1
+// (3 * 2^k > a); e = k - 3 never suffices (0.75 * 2^k < a).  Integer work on
+// the bits of a, no division.
+__device__ __forceinline__ int ceil_log2_over_6(float a) {
+  const uint32_t bits = __float_as_uint(a);
+  const int k = (int)((bits >> 23) & 0xffu) - 127;
+  return (bits & 0x7fffffu) <= 0x400000u ? k - 2 : k - 1;
+}
+
+// grid (m, ceil(K / 16 / 16)): CTA (j, c) handles the 16-element blocks
+// 16c .. 16c + 15 of row j, eight threads per block (two elements each),
 // after reading the whole row for its maximum (every CTA of the row finds the
 // same E).  Outputs: codes [m * P][K/2] (row j * P + p), scale bytes in the
 // blocked layout of the MMA's scale-factor copy (rows j * P + p), g [m][P]
-// (fp32).  After its griddep_wait the kernel also zeroes the counters of the
-// projection that follows it, if given.
+// (fp32).  The next kernel may launch at once (it waits for this one before
+// reading the planes); after its own wait for the previous kernel this one
+// also zeroes the counters of the projection that follows it, if given.
 __global__ void __launch_bounds__(kPlaneThreads) quantize_planes_kernel(
     const uint16_t* __restrict__ x, int m, int K, uint8_t* __restrict__ codes,
     uint8_t* __restrict__ sf_blocks, float* __restrict__ g, int* zero_ptr, int zero_count) {
-  asm volatile("griddepcontrol.wait;" ::: "memory");  // x may come from the previous kernel
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  asm volatile("griddepcontrol.wait;" ::: "memory");  // x may come from the previous kernel
   __shared__ float red[kPlaneThreads / 32];
   const int cta = blockIdx.x * gridDim.y + blockIdx.y;
   for (int i = cta * kPlaneThreads + threadIdx.x; i < zero_count; i += gridDim.x * gridDim.y * kPlaneThreads)
@@ -82,43 +93,38 @@ __global__ void __launch_bounds__(kPlaneThreads) quantize_planes_kernel(
   const int E = rowmax > 0.0f ? ilogbf(rowmax) : 0;
   if (blockIdx.y == 0 && threadIdx.x < kPlanes)
     g[j * kPlanes + threadIdx.x] = rowmax > 0.0f ? exp2i(E - 8 - (3 * (int)threadIdx.x) / 2) : 0.0f;
-  const int b = blockIdx.y * kBlocksPerCta + (threadIdx.x >> 2);
-  const int part = threadIdx.x & 3;  // elements 4 part .. 4 part + 3 of the block
-  const bool valid = b < nb;         // whole groups of four lanes share validity
-  float r[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+  const int b = blockIdx.y * kBlocksPerCta + (threadIdx.x >> 3);
+  const int part = threadIdx.x & 7;  // elements 2 part, 2 part + 1 of the block
+  const bool valid = b < nb;         // whole groups of eight lanes share validity
+  float r0 = 0.0f, r1 = 0.0f;
   if (valid) {
-    const uint2 v = *reinterpret_cast<const uint2*>(row + 16 * b + 4 * part);
-    r[0] = bf16_bits_to_float(v.x & 0xffffu);
-    r[1] = bf16_bits_to_float(v.x >> 16);
-    r[2] = bf16_bits_to_float(v.y & 0xffffu);
-    r[3] = bf16_bits_to_float(v.y >> 16);
+    const uint32_t v = *reinterpret_cast<const uint32_t*>(row + 16 * b + 2 * part);
+    r0 = bf16_bits_to_float(v & 0xffffu);
+    r1 = bf16_bits_to_float(v >> 16);
   }
 #pragma unroll 1
   for (int p = 0; p < kPlanes; ++p) {
-    float amax = fmaxf(fmaxf(fabsf(r[0]), fabsf(r[1])), fmaxf(fabsf(r[2]), fabsf(r[3])));
+    float amax = fmaxf(fabsf(r0), fabsf(r1));
     amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
     amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
-    uint32_t s8 = 0, nib = 0;
+    amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 4));
+    uint32_t s8 = 0, byte = 0;
     if (amax > 0.0f) {
       const int ge = E - 8 - (3 * p) / 2;  // log2 g_p
       // smallest power of two 2^e >= amax / 6 / g_p, clamped to E4M3's 2^-9..2^8
-      int ex;
-      const float fr = frexpf(__fdiv_rn(amax * exp2i(-ge), 6.0f), &ex);  // = fr * 2^ex, fr in [0.5, 1)
-      int e = fr == 0.5f ? ex - 1 : ex;
+      int e = ceil_log2_over_6(amax * exp2i(-ge));
       e = e < -9 ? -9 : (e > 8 ? 8 : e);
       s8 = e >= -6 ? (uint32_t)(e + 7) << 3 : (1u << (e + 9));
       // r / (g_p * 2^e) and the represented values are exact power-of-two scalings
       const float down = exp2i(-(ge + e)), up = exp2i(ge + e);
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const uint32_t q = e2m1_encode(r[i] * down);
-        r[i] -= ((q & 8u) ? -e2m1_mag(q & 7u) : e2m1_mag(q & 7u)) * up;
-        nib |= q << (4 * i);
-      }
+      const uint32_t q0 = e2m1_encode(r0 * down), q1 = e2m1_encode(r1 * down);
+      r0 -= ((q0 & 8u) ? -e2m1_mag(q0 & 7u) : e2m1_mag(q0 & 7u)) * up;
+      r1 -= ((q1 & 8u) ? -e2m1_mag(q1 & 7u) : e2m1_mag(q1 & 7u)) * up;
+      byte = q0 | (q1 << 4);
     }
     if (valid) {
       const int rowp = j * kPlanes + p;
-      *reinterpret_cast<uint16_t*>(codes + (size_t)rowp * (K / 2) + 8 * b + 2 * part) = (uint16_t)nib;
+      codes[(size_t)rowp * (K / 2) + 8 * b + part] = (uint8_t)byte;
       if (part == 0) sf_blocks[sf_blocked_offset(rowp, b, kc)] = (uint8_t)s8;
     }
   }

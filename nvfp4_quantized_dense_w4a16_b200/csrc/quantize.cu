@@ -107,8 +107,10 @@ __global__ void quantize_act_blocked_kernel(const uint16_t* __restrict__ x, int6
                                             uint8_t* __restrict__ codes,
                                             uint8_t* __restrict__ sf_blocks) {
   // x comes from the previous kernel (with programmatic dependent launch)
-  asm volatile("griddepcontrol.wait;" ::: "memory");
+  // the next kernel may launch now: it waits for this one before reading
+  // its results
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  asm volatile("griddepcontrol.wait;" ::: "memory");
   const int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;
   if (i >= nblocks) return;
   Block16 b;

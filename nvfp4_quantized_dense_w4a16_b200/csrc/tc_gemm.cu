@@ -1242,31 +1242,45 @@ tc_planes_kernel(const __grid_constant__ CUtensorMap xmap, const QArgs a) {
   if (warp == 0) {
     // -------------------------- producer: weights, plane codes, plane scales
     if (lane == 0) {
-      Seg sg;
-      int st_i = 0;
-      bool ok = true;
-      bool waited = false;
-      for (int j = 0; ok && range_segment(a.ntiles, a.kc, j, sg); ++j) {
-        for (int c = 0; c < sg.nk; c += kQChunks, ++st_i) {
-          const int s = st_i % S, nch = min(kQChunks, sg.nk - c);
-          if (st_i >= S && !mbar_wait(&empty[s], ((st_i / S) - 1) & 1, abort_flag, err, 1)) {
-            ok = false;
-            break;
+      // The weights of the first ring of stages do not depend on the previous
+      // kernel: they are requested before waiting for it (the planes are
+      // its output), so this kernel's CTAs stream weights while that kernel
+      // finishes.  Pass 0 issues those weights, pass 1 everything else.
+      int pre = 0;
+      for (int pass = 0; pass < 2; ++pass) {
+        if (pass == 1) griddep_wait();
+        Seg sg;
+        int st_i = 0;
+        bool ok = true;
+        for (int j = 0; ok && range_segment(a.ntiles, a.kc, j, sg); ++j) {
+          for (int c = 0; c < sg.nk; c += kQChunks, ++st_i) {
+            if (pass == 0 && st_i >= S) {
+              ok = false;
+              break;
+            }
+            const int s = st_i % S, nch = min(kQChunks, sg.nk - c);
+            uint8_t* st = smem + s * C::kStageBytes;
+            const int kchunk = sg.c0 + c;
+            if (pass == 0 || st_i >= pre) {
+              if (st_i >= S && !mbar_wait(&empty[s], ((st_i / S) - 1) & 1, abort_flag, err, 1)) {
+                ok = false;
+                break;
+              }
+              mbar_arrive_expect_tx(&full[s], nch * (kChunkBytes + 512) + NT * 128);
+              bulk_load(st, a.wt + ((size_t)sg.tile * a.kc + kchunk) * kChunkBytes, nch * kChunkBytes, &full[s]);
+              if (pass == 0) {
+                ++pre;
+                continue;
+              }
+            }
+            tma_load_2d(st + kW4Chunks * kChunkBytes, &xmap, 32 * kchunk, 0, &full[s]);
+            bulk_load(st + kW4Chunks * kChunkBytes + C::kXBytes, a.sfb + (size_t)kchunk * 512, nch * 512,
+                      &full[s]);
           }
-          uint8_t* st = smem + s * C::kStageBytes;
-          const int kchunk = sg.c0 + c;
-          mbar_arrive_expect_tx(&full[s], nch * (kChunkBytes + 512) + NT * 128);
-          bulk_load(st, a.wt + ((size_t)sg.tile * a.kc + kchunk) * kChunkBytes, nch * kChunkBytes, &full[s]);
-          if (!waited) {  // the planes come from the previous kernel
-            griddep_wait();
-            waited = true;
-          }
-          tma_load_2d(st + kW4Chunks * kChunkBytes, &xmap, 32 * kchunk, 0, &full[s]);
-          bulk_load(st + kW4Chunks * kChunkBytes + C::kXBytes, a.sfb + (size_t)kchunk * 512, nch * 512,
-                    &full[s]);
         }
+        if (pass == 1)
+          for (int i = max(0, st_i - S); i < st_i; ++i) wait_drain(&full[i % S], (i / S) & 1);
       }
-      for (int i = max(0, st_i - S); i < st_i; ++i) wait_drain(&full[i % S], (i / S) & 1);
     }
   } else if (warp == 1) {
     // ------------------------------------------------------ MMA issuer
