@@ -80,16 +80,29 @@ __global__ void __launch_bounds__(kPlaneThreads) quantize_planes_kernel(
   const int j = blockIdx.x;
   const int nb = K / 16, kc = (K + 63) / 64;
   const uint16_t* row = x + (size_t)j * K;
-  // the row's maximum |x| (eight bf16 per 16-byte load)
-  float local = 0.0f;
-  for (int i = threadIdx.x; i < K / 8; i += kPlaneThreads) {
-    const uint4 v = reinterpret_cast<const uint4*>(row)[i];
-    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+  // the row's maximum |x|: eight bf16 per 16-byte load, eight independent
+  // loads in flight per thread (|bf16| bits order like the values)
+  uint32_t mx[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+  const uint4* r16 = reinterpret_cast<const uint4*>(row);
+  const int n16 = K / 8;
+  for (int i0 = threadIdx.x; i0 < n16; i0 += 8 * kPlaneThreads) {
+    uint4 v[8];
 #pragma unroll
-    for (int e = 0; e < 4; ++e)
-      local = fmaxf(local, fmaxf(fabsf(bf16_bits_to_float(w[e] & 0xffffu)), fabsf(bf16_bits_to_float(w[e] >> 16))));
+    for (int u = 0; u < 8; ++u) {
+      const int i = i0 + u * kPlaneThreads;
+      v[u] = i < n16 ? r16[i] : make_uint4(0, 0, 0, 0);
+    }
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const uint32_t w[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) mx[u] = max(mx[u], max(w[e] & 0x7fffu, (w[e] >> 16) & 0x7fffu));
+    }
   }
-  const float rowmax = block_reduce_max(local, red);
+  uint32_t mbits = 0;
+#pragma unroll
+  for (int u = 0; u < 8; ++u) mbits = max(mbits, mx[u]);
+  const float rowmax = block_reduce_max(bf16_bits_to_float(mbits), red);
   const int E = rowmax > 0.0f ? ilogbf(rowmax) : 0;
   if (blockIdx.y == 0 && threadIdx.x < kPlanes)
     g[j * kPlanes + threadIdx.x] = rowmax > 0.0f ? exp2i(E - 8 - (3 * (int)threadIdx.x) / 2) : 0.0f;
