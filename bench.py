@@ -263,6 +263,10 @@ class Workload:
         m, H, I = self.m, self.H, self.I
         if "quantize_activations" in kname:
             return "hbm", None
+        if "planes_prologue" in kname:  # reads x (its planes are a few KB)
+            return "hbm", m * H * 2
+        if "planes_layer" in kname:  # both projections in one persistent kernel
+            return "hbm", self.weight_bytes + m * H * 2 * 2 + m * I * 2 * 2
         if "gate_up" in kname:
             flops, byts = 2.0 * m * 2 * I * H, nvfp4_bytes(2 * I, H) + m * H * 2 + m * I * 2
         else:

@@ -149,8 +149,8 @@ bool serves(const ffn_nvfp4_weight* w, ffn_act_format f) {
 // 256-byte aligned): [h bf16 m*inter] [xq codes m*hidden/2] [xq scales
 // m*hidden/16] [hq codes m*inter/2] [hq scales m*inter/16].
 struct Carve {
-  size_t h = 0, xq_c = 0, xq_s = 0, hq_c = 0, hq_s = 0, part = 0, cnt = 0, xa_gu = 0, xa_d = 0, total = 0;
-  size_t xg = 0, hg = 0;  // plane factors
+  size_t h = 0, xq_c = 0, xq_s = 0, hq_c = 0, hq_s = 0, part = 0, part2 = 0, cnt = 0, xa_gu = 0, xa_d = 0,
+         total = 0;
   ffn::TcPlan gate_up, down;
   ffn::PersistPlan persist;
   ffn::PlanesPlan planes;
@@ -191,18 +191,17 @@ Carve carve_ffn(int64_t m, int64_t hidden, int64_t inter, ffn_act_format f, int6
     off += round_up((size_t)m * lora_rank * 2, 256);
   }
   if (f == FFN_ACT_BF16 && m > 0 && planes) {
-    // plane codes [m*P, k/2], scale blocks [kc][512], factors [m][P], split-K
-    // partials and tile counters
+    // x's and h's planes (codes, scale bytes), split-K partials of both
+    // projections, the zeroed words (tile counters, ready flags) and the
+    // row and chunk exponents
     c.planes = ffn::plan_planes(m, hidden, inter, num_sms());
-    const size_t rows = (size_t)m * c.planes.planes;
-    c.xq_c = off; off += round_up(rows * hidden / 2, 256);
-    c.xq_s = off; off += round_up((size_t)((hidden + 63) / 64) * 512, 256);
-    c.hq_c = off; off += round_up(rows * inter / 2, 256);
-    c.hq_s = off; off += round_up((size_t)((inter + 63) / 64) * 512, 256);
-    c.xg = off; off += round_up(rows * sizeof(float), 256);
-    c.hg = off; off += round_up(rows * sizeof(float), 256);
-    c.part = off; off += round_up(c.planes.partial_bytes, 256);
-    c.cnt = off; off += round_up((size_t)c.planes.counter_count * sizeof(int), 256);
+    c.xq_c = off; off += round_up(c.planes.x_code_bytes, 256);
+    c.xq_s = off; off += round_up(c.planes.x_sf_bytes, 256);
+    c.hq_c = off; off += round_up(c.planes.h_code_bytes, 256);
+    c.hq_s = off; off += round_up(c.planes.h_sf_bytes, 256);
+    c.part = off; off += round_up(c.planes.gu_partial_bytes, 256);
+    c.part2 = off; off += round_up(c.planes.dn_partial_bytes, 256);
+    c.cnt = off; off += round_up((size_t)(c.planes.zero_ints + c.planes.other_ints) * sizeof(int), 256);
   } else if (f == FFN_ACT_BF16 && m > 0 && w4a16_persistent(m)) {
     c.persist = ffn::plan_persist(m, hidden, inter, num_sms());
     c.part = off;
@@ -235,7 +234,7 @@ Carve carve_ffn(int64_t m, int64_t hidden, int64_t inter, ffn_act_format f, int6
 size_t ffn_workspace_bytes(int64_t m, int64_t hidden, int64_t inter, ffn_act_format f, int64_t lora_rank) {
   size_t b = carve_ffn(m, hidden, inter, f, lora_rank, false).total;
   const int forced = w4a16_forced();
-  if (f == FFN_ACT_BF16 && (forced == 0 || forced == 4) && ffn::planes_for_rows(m) > 0) {
+  if (f == FFN_ACT_BF16 && lora_rank == 0 && (forced == 0 || forced == 4) && ffn::planes_for_rows(m) > 0) {
     const size_t bp = carve_ffn(m, hidden, inter, f, lora_rank, true).total;
     if (bp > b) b = bp;
   }
@@ -524,7 +523,7 @@ ffn_status ffn_nvfp4_forward_lora(const void* x, int64_t m, int64_t hidden, int6
     }
     if (dev != lv.device) return FFN_ERR_INVALID_ARG;
   }
-  const bool planes = format == FFN_ACT_BF16 && w4a16_planes(m, hidden, inter, gate_up, down);
+  const bool planes = format == FFN_ACT_BF16 && lv.rank == 0 && w4a16_planes(m, hidden, inter, gate_up, down);
   const Carve c = carve_ffn(m, hidden, inter, format, lv.rank, planes);
   if (!workspace || workspace_bytes < c.total) return FFN_ERR_WORKSPACE;
   if (!aligned16(x) || !aligned16(out) || !aligned16(workspace)) return FFN_ERR_ALIGNMENT;
@@ -535,18 +534,14 @@ ffn_status ffn_nvfp4_forward_lora(const void* x, int64_t m, int64_t hidden, int6
   cudaError_t e;
   if (planes) {
     ffn::PlanesBuffers b;
-    b.h = h;
-    b.x_codes = ws + c.xq_c;
-    b.x_sf = ws + c.xq_s;
-    b.h_codes = ws + c.hq_c;
-    b.h_sf = ws + c.hq_s;
-    b.x_g = reinterpret_cast<float*>(ws + c.xg);
-    b.h_g = reinterpret_cast<float*>(ws + c.hg);
-    b.partials = ws + c.part;
-    b.counters = reinterpret_cast<int*>(ws + c.cnt);
-    b.xa_gu = ws + c.xa_gu;
-    b.xa_d = ws + c.xa_d;
-    e = ffn::launch_planes_ffn(x, m, gate_up->tc(), down->tc(), c.planes, b, out, s, lv);
+    b.xq = ws + c.xq_c;
+    b.xs = ws + c.xq_s;
+    b.hq = ws + c.hq_c;
+    b.hs = ws + c.hq_s;
+    b.part_gu = ws + c.part;
+    b.part_dn = ws + c.part2;
+    b.ints = reinterpret_cast<int*>(ws + c.cnt);
+    e = ffn::launch_planes_ffn(x, m, gate_up->tc(), down->tc(), c.planes, b, out, s);
   } else if (format == FFN_ACT_BF16 && w4a16_persistent(m)) {
     e = ffn::launch_persist_ffn(x, m, gate_up->tc(), down->tc(), c.persist, h, ws + c.part,
                                 reinterpret_cast<int*>(ws + c.cnt), out, s, lv, ws + c.xa_gu, ws + c.xa_d);
@@ -614,9 +609,14 @@ ffn_status ffn_nvfp4_projection_plan(int64_t m, int64_t n, int64_t k, ffn_act_fo
       ffn::planes_for_rows(m) > 0) {
     // (when both handles hold the natural tiled layout; else the tc_w4a16 row)
     const ffn::PlanesPlan p = gate_up ? ffn::plan_planes(m, k, n / 2, num_sms()) : ffn::plan_planes(m, n, k, num_sms());
-    const int64_t W = gate_up ? (int64_t)p.gu_tiles * p.gu_kc : (int64_t)p.dn_tiles * p.dn_kc;
-    const int grid = gate_up ? p.gu_grid : p.dn_grid, kc = gate_up ? p.gu_kc : p.dn_kc;
-    *out = ffn_projection_plan{FFN_KERNEL_TC_PLANES, p.nt, (int)(((int64_t)kc * grid + W - 1) / W + 1), grid};
+    // (without a LoRA adapter) one persistent kernel runs both projections;
+    // K ranges per output tile: at most ceil(kc / (tiles * kc / parts)) + 1
+    const int tiles = gate_up ? p.gu_tiles : p.dn_tiles, kc = gate_up ? p.gu_kc : p.dn_kc;
+    const int parts = gate_up ? p.gu_parts : p.grid;
+    const int64_t W = (int64_t)tiles * kc;
+    const int splits = parts <= tiles ? (tiles % parts ? 2 : 1) : (int)(((int64_t)kc * parts + W - 1) / W + 1);
+    *out = ffn_projection_plan{FFN_KERNEL_TC_PLANES, p.nt, gate_up && p.gu_parts == p.gu_tiles ? 1 : splits,
+                               p.grid};
   } else if (format == FFN_ACT_BF16 && role != FFN_ROLE_LINEAR && w4a16_persistent(m)) {
     // gate+up: n = 2 * inter, k = hidden; down: n = hidden, k = inter
     const ffn::PersistPlan p = gate_up ? ffn::plan_persist(m, k, n / 2, num_sms())

@@ -83,25 +83,25 @@ cudaError_t launch_persist_ffn(const void* x, int64_t m, const TcWeight& gate_up
                                cudaStream_t s, const LoraView& lv = LoraView(), void* xa_gu = nullptr,
                                void* xa_d = nullptr);
 // Few-row W4A16 layer on the block-scaled FP4 tensor core (natural tiled
-// weights as the MMA's A operand, activations as NVFP4 planes; planes.cu).
+// weights as the MMA's A operand, activations as NVFP4 planes built in the
+// GEMM kernel's shared memory).
 int planes_for_rows(int64_t m);  // planes per activation row, 0 when the path does not apply
-cudaError_t launch_quantize_planes(const void* x, int64_t m, int64_t k, int planes, void* codes, void* sf_blocks,
-                                   float* g, int* zero_ptr, int zero_count, cudaStream_t s);
 struct PlanesPlan {
-  int planes = 0, nt = 0;
-  int gu_tiles = 0, gu_kc = 0, gu_grid = 0, dn_tiles = 0, dn_kc = 0, dn_grid = 0;
-  size_t partial_bytes = 0;
-  int counter_count = 0;
+  int planes = 0, nt = 0, rows = 0, grid = 0;
+  int gu_tiles = 0, gu_kc = 0, gu_parts = 0, dn_tiles = 0, dn_kc = 0;
+  size_t gu_partial_bytes = 0, dn_partial_bytes = 0, x_code_bytes = 0, x_sf_bytes = 0, h_code_bytes = 0,
+         h_sf_bytes = 0;
+  int zero_ints = 0;   // ints the prologue zeroes
+  int other_ints = 0;  // ints after them (row and chunk exponents)
 };
 struct PlanesBuffers {  // workspace regions of the few-row block-scaled layer
-  void *h, *x_codes, *x_sf, *h_codes, *h_sf, *partials, *xa_gu, *xa_d;
-  float *x_g, *h_g;
-  int* counters;
+  void *xq, *xs, *hq, *hs, *part_gu, *part_dn;
+  int* ints;
 };
 PlanesPlan plan_planes(int64_t m, int64_t hidden, int64_t inter, int num_sms);
+// Requires hidden and inter multiples of 32, and no LoRA adapter.
 cudaError_t launch_planes_ffn(const void* x, int64_t m, const TcWeight& gate_up, const TcWeight& down,
-                              const PlanesPlan& p, const PlanesBuffers& b, void* out, cudaStream_t s,
-                              const LoraView& lv);
+                              const PlanesPlan& p, const PlanesBuffers& b, void* out, cudaStream_t s);
 // Fixed-format (W4A4) projection on the block-scaled FP4 tensor core.  The
 // plan depends on (n, k) only (plus the number of 128-row activation tiles).
 TcPlan plan_w4a4(int64_t m, int64_t n, int64_t k, bool gate_up, int num_sms);

@@ -998,7 +998,7 @@ struct W4Cfg {
   static_assert(kSfbCol + XT * 4 * kW4Chunks * kStages <= kTmemCols, "TMEM budget");
   static_assert(kStageBytes % 1024 == 0, "stage alignment");
   static_assert(kSmemAlloc <= 232448, "shared memory budget");
-  static_assert(kSmemEpi >= 16384, "the epilogue buffer aliases the rings");
+  static_assert(kSmemEpi >= 2 * 16384, "the two epilogue buffers alias the rings");
 };
 
 struct W4Args {
@@ -1097,31 +1097,45 @@ tc_w4a4_kernel(const __grid_constant__ CUtensorMap xmap, const W4Args w4) {
         if (!mbar_wait(&full[s], (i / S) & 1, abort_flag, err, 2)) break;
         tc_fence_after();
         const uint8_t* st = smem + s * C::kStageBytes;
+        // the stage's scale copies first, then its MMAs (each MMA then finds
+        // its scales in TMEM without waiting for a copy issued just before)
         for (int c = 0; c < nch; ++c) {
           const uint32_t slot = 4 * (s * kW4Chunks + c);
           const uint8_t* wc = st + c * kChunkBytes;
           tmem_cp_32x128b_x4(tmem + C::kSfaCol + slot, smem_desc_interleave(smem_u32(wc + 4096), 16, 128));
-          const uint64_t a_desc = smem_desc_interleave(smem_u32(wc), 2048, 128);
           for (int t = 0; t < nxt; ++t) {
             const uint8_t* xt = st + C::kWBytes + t * (C::kXBytes + C::kSfbBytes);
-            const uint32_t sfb = tmem + C::kSfbCol + t * 4 * kW4Chunks * S + slot;
-            tmem_cp_32x128b_x4(sfb, smem_desc_interleave(smem_u32(xt + C::kXBytes + 512 * c), 16, 128));
+            tmem_cp_32x128b_x4(tmem + C::kSfbCol + t * 4 * kW4Chunks * S + slot,
+                               smem_desc_interleave(smem_u32(xt + C::kXBytes + 512 * c), 16, 128));
+          }
+        }
+        for (int c = 0; c < nch; ++c) {
+          const uint32_t slot = 4 * (s * kW4Chunks + c);
+          const uint64_t a_desc = smem_desc_interleave(smem_u32(st + c * kChunkBytes), 2048, 128);
+          for (int t = 0; t < nxt; ++t) {
+            const uint8_t* xt = st + C::kWBytes + t * (C::kXBytes + C::kSfbBytes);
             mma_mxf4nvf4(tmem + t * kW4BN, a_desc, smem_desc_sw128(smem_u32(xt)) + 2 * c, idesc,
-                         tmem + C::kSfaCol + slot, sfb, (i | c) != 0 ? 1u : 0u);
+                         tmem + C::kSfaCol + slot, tmem + C::kSfbCol + t * 4 * kW4Chunks * S + slot,
+                         (i | c) != 0 ? 1u : 0u);
           }
         }
         mma_commit(&empty[s]);
       }
       mma_commit(accum);
     }
-  } else if (warp >= 4) {
-    const int q = warp & 3;
+  }
+  // epilogue on all eight warps once the last MMA is done: warpgroup g takes
+  // every other 32-row chunk of each activation tile (warp w reads TMEM
+  // lanes 32 (w % 4) ..), each with its own 16 KB buffer
+  __syncwarp();
+  {
+    const int q = warp & 3, g = warp < 4 ? 1 : 0;
     const bool done = __all_sync(0xffffffffu, wait_drain(accum, 0));
     tc_fence_after();
     griddep_wait();  // the previous kernel may still read this kernel's outputs
     if (done && !*abort_flag)
       for (int t = 0; t < nxt; ++t)
-        epilogue_tile<kW4BN, EPI, 1>(a, tmem + t * kW4BN, q, lane, 0, epi, xt0 + t, wtile);
+        epilogue_tile<kW4BN, EPI, 2>(a, tmem + t * kW4BN, q, lane, g, epi + g * 16384, xt0 + t, wtile);
   }
   tc_fence_before();
   __syncthreads();
@@ -1132,93 +1146,282 @@ tc_w4a4_kernel(const __grid_constant__ CUtensorMap xmap, const W4Args w4) {
 }
 
 // ---------------------------------------------------------------------------
-// Few-row W4A16 projection on the block-scaled FP4 tensor core.  The weights
-// go to kind::mxf4nvf4 as stored (natural tiled chunks: codes are the A
-// operand, the chunk's 512-byte scale block is SFA) -- no software
-// dequantisation; the activation rows arrive as P NVFP4 planes per row (see
-// planes.cu), N = m * P columns, with their scale blocks as SFB.  The
-// epilogue folds the planes back, y[j, n] = sum_p g[j, p] * D[n, j*P + p].
-// Work: the (weight tile, 64-element chunk) space cut into one contiguous,
-// equal range per CTA (two CTAs per SM), each range a list of segments (one
-// per tile it touches); stages of up to 4 chunks never cross a segment.  Each
-// segment's fp32 partial sums go to the workspace, slot (CTA + tile); the CTA
-// that completes a tile's count (atomic, zeroed by the plane quantiser that
-// runs before) adds the tile's partials in K order and writes the output:
-// SiLU*mul into h for the fused gate+up weight, or bf16(gs * y) for down,
-// with LoRA deltas when given.  Two accumulators alternate between segments
-// so that a segment's epilogue overlaps the next segment's MMAs.
+// Few-row W4A16 layer on the block-scaled FP4 tensor core.
+//
+// The NVFP4 weights go to tcgen05 kind::mxf4nvf4 as stored (natural tiled
+// chunks: the codes are the A operand, the chunk's 512-byte scale block is
+// SFA) -- no software dequantisation.  Each bf16 activation row becomes the B
+// operand as P = 8 NVFP4 "planes", x = sum_p g_p * (s_p,b * q_p,k) + r_P,
+// each plane one MMA column (N = 8m, at least 16):
+//  * g_p = 2^(E - 8 - floor(3p / 2)), E = floor(log2 max|x|) of the row (a
+//    per-row power-of-two factor that keeps every block scale of the plane
+//    within E4M3's powers of two 2^-9..2^8; applied in the epilogue);
+//  * per 16-block a power-of-two scale s = 2^ceil(log2(amax / 6 / g_p)) of
+//    the residual r left by planes 0..p-1 (exact in E4M3, and r then scales
+//    exactly), codes q = E2M1(r / (g_p * s)), and r -= g_p * s * q (exact:
+//    the represented value has at most two significant bits and lies within a
+//    factor two of r).
+// Each plane removes at least a factor 3 from every block's residual while
+// g_p's range drops by 2^1.5 per plane, so no block outgrows its plane; a
+// plane takes the next two to three bits near each block's maximum, and 8
+// planes represent seeded bf16 rows (normal, outlier-channel, cubed-normal)
+// exactly or to ~1e-9 of the row maximum; small integers need the first
+// plane only.  The epilogue folds the planes back, y[j] = sum_p g_p * D_j,p,
+// so the result is the fp32-accumulated product of the exact bf16 rows.
+//
+// One layer is two launches.  A small prologue kernel builds x's planes
+// with one exponent per row (codes [m P][H/2], scale bytes [H/64][m P][4],
+// E[m]) and zeroes the layer's counters.  Then one persistent kernel, two
+// CTAs per SM, all resident, runs both projections:
+//  * gate+up: whole tiles (gate rows 64t.., then the matching up rows), one
+//    per CTA, when there are no more tiles than CTAs, else equal ranges of
+//    the (tile, 64-element chunk) space with split-K partial sums that the
+//    CTA completing a tile's count adds in K order.  The CTA that finishes
+//    tile t computes h = bf16(silu(bf16 g) * bf16 u) for its 64 columns and
+//    at once the planes of that 64-column chunk of h, with the chunk's own
+//    exponent per row, then raises the chunk's ready flag;
+//  * down: equal ranges of its (tile, chunk) space; a stage of chunks is
+//    copied in once their flags are up (no grid-wide barrier), each chunk
+//    goes to its own accumulator, and the epilogue folds every stage with
+//    the chunks' exponents; split-K partial sums as above.
+// Each CTA's weight stream runs through both projections without a break,
+// and once its gate+up loads are issued it prefetches its down weights into
+// L2.  Every wait is bounded and raises a device error bit when it expires.
 // ---------------------------------------------------------------------------
-constexpr int kQChunks = 4;  // 64-element chunks per stage
+constexpr int kQChunks = 4;   // 64-element chunks per stage
+constexpr int kQPlanes = 8;   // activation planes per row
+constexpr int kSegZero = -1000;      // the row is all zero
+constexpr int kSegNonFinite = 1000;  // the row holds an Inf or NaN
 
-template <int NT>
+// Fixed configuration: up to two activation rows (N = 16 plane columns).
 struct QCfg {
-  static constexpr int kXBytes = NT * 128;               // NT plane rows x 256 elements
-  static constexpr int kStageBytes = kW4Chunks * kChunkBytes + kXBytes + kQChunks * 512;
-  static constexpr int kStages = NT <= 32 ? 4 : 3;
-  static constexpr int kSmemBar = kStages * kStageBytes;
+  static constexpr int kNT = 16;                          // MMA N
+  static constexpr int kMR = kNT / kQPlanes;              // activation rows
+  static constexpr int kXBytes = kNT * 128;               // 16 plane rows x 256 elements (128-byte swizzle)
+  static constexpr int kStageBytes = kQChunks * kChunkBytes + kXBytes + kQChunks * 512;
+  static constexpr int kStages = 4;
+  static constexpr int kSmemMisc = kStages * kStageBytes;
+  // misc: 16 words, Y [kMR][128] fp32 (a tile's sums)
+  static constexpr int kSmemY = kSmemMisc + 64;
+  static constexpr int kSmemBar = kSmemY + kMR * 128 * 4;
   static constexpr int kNumBars = 2 * kStages + 4;       // full, empty, accfull[2], accfree[2]
   static constexpr int kSmemAlloc = kSmemBar + kNumBars * 8 + 32 + 1024;
-  static constexpr int kAccCols = 2 * NT;
-  static constexpr int kSfaCol = kAccCols;
+  // TMEM: two accumulator buffers, then the scale-factor columns
+  static constexpr int kAccBuf = kNT;
+  static constexpr int kSfaCol = 2 * kAccBuf;
   static constexpr int kSfbCol = kSfaCol + 4 * kQChunks * kStages;
-  static constexpr int kTmemNeed = kSfbCol + 4 * kQChunks * kStages;
-  static constexpr int kTmemCols = kTmemNeed <= 256 ? 256 : 512;
+  static constexpr int kTmemCols = 256;
+  static_assert(kSfbCol + 4 * kQChunks * kStages <= kTmemCols, "TMEM budget");
   static_assert(kStageBytes % 1024 == 0, "stage alignment (128-byte swizzle)");
   static_assert(2 * (kSmemAlloc + 1024) <= 233472, "two CTAs per SM");
-  static_assert(kTmemCols == 256, "two CTAs per SM share the 512 TMEM columns");
-  static_assert(NT % 16 == 0 && NT >= 16 && NT <= 64, "MMA N");
 };
 
-struct QArgs {
-  const uint8_t* wt;     // natural tiled weight [ntiles][kc][4608]
-  const float* gs;       // tensor scale(s)
-  uint16_t* out;         // bf16 [m, ldo]: h (gate+up) or out (down)
-  int m, n_out, ldo, kc, ntiles, planes;
-  const uint8_t* sfb;    // plane scale blocks [kc][512]
-  const float* g;        // plane factors [m][planes]
-  float* partials;       // [gridDim.x + ntiles][m][128]
-  int* counters;         // [ntiles], zero on entry
-  LoraArgs lora;
+// 2^k as fp32 (exact; built from the exponent bits in the normal range).
+__device__ __forceinline__ float exp2i(int k) {
+  return k >= -126 && k <= 127 ? __int_as_float((k + 127) << 23) : ldexpf(1.0f, k);
+}
+
+// Smallest e with 6 * 2^e >= a, for a > 0 normal: with a in [2^k, 2^(k+1)),
+// e = k - 2 when a <= 1.5 * 2^k (6 * 2^(k-2) = 1.5 * 2^k), else k - 1
+// (3 * 2^k > a); e = k - 3 never suffices (0.75 * 2^k < a).  Integer work on
+// the bits of a, no division.
+__device__ __forceinline__ int ceil_log2_over_6(float a) {
+  const uint32_t bits = __float_as_uint(a);
+  const int k = (int)((bits >> 23) & 0xffu) - 127;
+  return (bits & 0x7fffffu) <= 0x400000u ? k - 2 : k - 1;
+}
+
+// Row exponent from the largest |bf16| bit pattern of the row.
+__device__ __forceinline__ int row_exponent(uint32_t max_bits) {
+  return max_bits == 0 ? kSegZero : max_bits >= 0x7f80u ? kSegNonFinite : ilogbf(bf16_bits_to_float(max_bits));
+}
+
+// The P planes of one 16-element block, by the eight lanes part = 0..7 of an
+// aligned group of eight (two elements each; every lane of the warp calls).
+// Writes byte 8 b + part of plane row j P + p (rows of row_bytes) and, from
+// part 0, the block's scale byte at [b / 4][rows][4] + b % 4.
+__device__ __forceinline__ void block_planes(float r0, float r1, int E, bool valid, int part, int j, int b,
+                                             uint8_t* codes, size_t row_bytes, uint8_t* sf, int rows) {
+#pragma unroll 1
+  for (int p = 0; p < kQPlanes; ++p) {
+    float amax = fmaxf(fabsf(r0), fabsf(r1));
+    amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
+    amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
+    amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 4));
+    uint32_t s8 = 0, byte = 0;
+    if (amax > 0.0f) {
+      const int ge = E - 8 - (3 * p) / 2;  // log2 g_p
+      // smallest power of two 2^e >= amax / 6 / g_p, clamped to E4M3's 2^-9..2^8
+      int e = ceil_log2_over_6(amax * exp2i(-ge));
+      e = e < -9 ? -9 : (e > 8 ? 8 : e);
+      s8 = e >= -6 ? (uint32_t)(e + 7) << 3 : (1u << (e + 9));
+      // r / (g_p 2^e) and the represented values are exact power-of-two scalings
+      const float down = exp2i(-(ge + e)), up = exp2i(ge + e);
+      const uint32_t q0 = e2m1_encode(r0 * down), q1 = e2m1_encode(r1 * down);
+      r0 -= ((q0 & 8u) ? -e2m1_mag(q0 & 7u) : e2m1_mag(q0 & 7u)) * up;
+      r1 -= ((q1 & 8u) ? -e2m1_mag(q1 & 7u) : e2m1_mag(q1 & 7u)) * up;
+      byte = q0 | (q1 << 4);
+    }
+    if (valid) {
+      const int rowp = j * kQPlanes + p;
+      codes[(size_t)rowp * row_bytes + 8 * b + part] = (uint8_t)byte;
+      if (part == 0) sf[((size_t)(b >> 2) * rows + rowp) * 4 + (b & 3)] = (uint8_t)s8;
+    }
+  }
+}
+
+// Prologue: grid (m, ceil(K / 16 / 16)), 128 threads; CTA (j, c) builds the
+// planes of blocks 16c .. 16c + 15 of row j after finding the row's maximum
+// (every CTA of the row finds the same E), CTA (j, 0) writes E[j], and the
+// CTAs zero the next kernel's counters.  It lets the next kernel launch at
+// once (that one waits for this one before reading anything it writes).
+constexpr int kPlaneThreads = 128;
+__global__ void __launch_bounds__(kPlaneThreads) planes_prologue_kernel(const uint16_t* __restrict__ x, int m, int K,
+                                                                        uint8_t* __restrict__ codes,
+                                                                        uint8_t* __restrict__ sf, int* __restrict__ E_out,
+                                                                        int* zero_ptr, int zero_count) {
+  griddep_launch_dependents();
+  griddep_wait();  // x comes from the previous kernel, which may also still use the counters
+  __shared__ uint32_t red[kPlaneThreads / 32];
+  const int cta = blockIdx.x * gridDim.y + blockIdx.y;
+  for (int i = cta * kPlaneThreads + threadIdx.x; i < zero_count; i += gridDim.x * gridDim.y * kPlaneThreads)
+    zero_ptr[i] = 0;
+  const int j = blockIdx.x;
+  const uint16_t* row = x + (size_t)j * K;
+  // the row's maximum |x|: eight bf16 per 16-byte load, eight independent
+  // loads in flight per thread (|bf16| bit patterns order like the values)
+  uint32_t mx = 0;
+  const uint4* r16 = reinterpret_cast<const uint4*>(row);
+  const int n16 = K / 8;
+  for (int i0 = threadIdx.x; i0 < n16; i0 += 8 * kPlaneThreads) {
+    uint4 v[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const int i = i0 + u * kPlaneThreads;
+      v[u] = i < n16 ? r16[i] : make_uint4(0, 0, 0, 0);
+    }
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const uint32_t w[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) mx = max(mx, max(w[e] & 0x7fffu, (w[e] >> 16) & 0x7fffu));
+    }
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) mx = max(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = mx;
+  __syncthreads();
+  mx = max(max(red[0], red[1]), max(red[2], red[3]));
+  const int E = row_exponent(mx);
+  if (blockIdx.y == 0 && threadIdx.x == 0) E_out[j] = E;
+  const int nb = K / 16;
+  const int b = blockIdx.y * (kPlaneThreads / 8) + (threadIdx.x >> 3);
+  const int part = threadIdx.x & 7;  // elements 2 part, 2 part + 1 of the block
+  const bool valid = b < nb;         // whole groups of eight lanes share validity
+  float r0 = 0.0f, r1 = 0.0f;
+  if (valid && E != kSegNonFinite) {
+    const uint32_t v = *reinterpret_cast<const uint32_t*>(row + 16 * b + 2 * part);
+    r0 = bf16_bits_to_float(v & 0xffffu);
+    r1 = bf16_bits_to_float(v >> 16);
+  }
+  block_planes(r0, r1, E, valid, part, j, b, codes, (size_t)K / 2, sf, m * kQPlanes);
+}
+
+struct LArgs {
+  const uint8_t* wt_gu;  // natural tiled gate+up weight [gu_tiles][gu_kc][4608] (gate/up interleaved by 64)
+  const uint8_t* wt_dn;  // natural tiled down weight [dn_tiles][dn_kc][4608]
+  const float* gs_gu;    // gate and up tensor scales
+  const float* gs_dn;
+  const uint8_t* xq;     // x planes (prologue): codes [m P][H/2], scales [H/64][m P][4], E [m]
+  const uint8_t* xs;
+  const int* xe;
+  uint8_t* hq;           // h planes: codes [m P][I/2], scales [I/64][m P][4], E [I/64][m]
+  uint8_t* hs;
+  int* he;
+  uint16_t* out;         // bf16 [m, H]
+  float* part_gu;        // split-K partial sums [gu_parts + gu_tiles][m][128]
+  float* part_dn;        // [gridDim.x + dn_tiles][m][128]
+  int* cnt_gu;           // [gu_tiles] chunks done, zero on entry
+  int* cnt_dn;           // [dn_tiles]
+  int* ready;            // [gu_tiles] h chunk's planes written, zero on entry
+  int m, hidden, inter, gu_tiles, gu_kc, gu_parts, dn_tiles, dn_kc;
 };
 
-// Segment j of this CTA's equal range of the (tile, chunk) space.
-__device__ __forceinline__ bool range_segment(int ntiles, int kc, int j, Seg& s) {
-  const int G = gridDim.x, g = blockIdx.x;
-  const int64_t W = (int64_t)ntiles * kc;
-  const int64_t lo = W * g / G, hi = W * (g + 1) / G;
-  const int t = (int)(lo / kc) + j;
-  const int64_t b = lo > (int64_t)t * kc ? lo : (int64_t)t * kc;
-  const int64_t e = hi < (int64_t)(t + 1) * kc ? hi : (int64_t)(t + 1) * kc;
+// Segment j of part g's equal share of the (tile, chunk) space split into
+// `parts` shares (parts * tiles * kc < 2^32, checked by the host).
+__device__ __forceinline__ bool range_segment(int ntiles, int kc, int parts, int g, int j, Seg& s) {
+  if (g >= parts) return false;
+  const uint32_t W = (uint32_t)ntiles * kc;
+  const uint32_t lo = W * (uint32_t)g / parts, hi = W * (uint32_t)(g + 1) / parts;
+  const uint32_t t = lo / kc + j;
+  const uint32_t b = max(lo, t * kc), e = min(hi, (t + 1) * kc);
   if (b >= e) return false;
-  s.tile = t;
-  s.c0 = (int)(b - (int64_t)t * kc);
+  s.tile = (int)t;
+  s.c0 = (int)(b - t * kc);
   s.nk = (int)(e - b);
   return true;
 }
 
-template <int NT, int P, bool kGateUp>
-__global__ void __launch_bounds__(256, 2)
-tc_planes_kernel(const __grid_constant__ CUtensorMap xmap, const QArgs a) {
-  static_assert(NT % P == 0, "whole rows of planes per MMA");
-  constexpr int MR = NT / P;  // activation rows (m <= MR)
-  using C = QCfg<NT>;
-  constexpr int S = C::kStages;
+__device__ __forceinline__ bool q_segment(const LArgs& a, int ph, int j, Seg& s) {
+  return ph ? range_segment(a.dn_tiles, a.dn_kc, gridDim.x, blockIdx.x, j, s)
+            : range_segment(a.gu_tiles, a.gu_kc, a.gu_parts, blockIdx.x, j, s);
+}
+
+__device__ __forceinline__ int ld_acquire(const int* p) {
+  int v;
+  asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+
+// Bounded wait for a chunk's ready flag.
+__device__ __forceinline__ bool wait_ready(const int* flag, volatile int* abort, int* err) {
+  if (ld_acquire(flag)) return true;
+  const long long t0 = clock64();
+  for (;;) {
+    if (ld_acquire(flag)) return true;
+    if (*abort) return false;
+    if (clock64() - t0 > kWaitLimitCycles) {
+      *abort = 1;
+      atomicOr(err, 32);
+      return false;
+    }
+  }
+}
+
+// Sum of the split-K partial slots of tile t (CTAs g0..g1 of `parts` that
+// own a non-empty share of it), in K order.
+__device__ __forceinline__ float sum_partials(const float* part, int m, int jr, int rr, int t, uint32_t W, int parts,
+                                              int g0, int g1) {
+  float sum = 0.0f;
+  for (int gg = g0; gg <= g1; ++gg)
+    if (W * (uint32_t)gg / parts != W * (uint32_t)(gg + 1) / parts)
+      sum += __ldcg(part + ((size_t)(gg + t) * m + jr) * kTileRows + rr);
+  return sum;
+}
+
+__global__ void __launch_bounds__(256, 2) tc_planes_layer_kernel(const LArgs a) {
+  using C = QCfg;
+  constexpr int S = C::kStages, P = kQPlanes, MR = C::kMR, NT = C::kNT;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
+  int* misc = reinterpret_cast<int*>(smem + C::kSmemMisc);
+  volatile int* sh_fail = misc;            // [2] epilogue stop flags by segment parity
+  volatile int* last_flag = misc + 2;
+  float* Y = reinterpret_cast<float*>(smem + C::kSmemY);  // [MR][128] a finished tile's sums
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::kSmemBar);
   uint64_t* empty = full + S;
   uint64_t* accfull = empty + S;   // [2]
   uint64_t* accfree = accfull + 2; // [2]
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(accfree + 2);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
-  volatile int* last_flag = reinterpret_cast<volatile int*>(tmem_slot + 2);
   int* err = &g_ffn_device_error;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int rows = a.m * P;  // plane rows in use
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < S; ++s) {
-      mbar_init(&full[s], 1);
+      mbar_init(&full[s], 2);  // the weights' expect_tx arrival + the stage's operand warp
       mbar_init(&empty[s], 1);
     }
     for (int b = 0; b < 2; ++b) {
@@ -1226,13 +1429,13 @@ tc_planes_kernel(const __grid_constant__ CUtensorMap xmap, const QArgs a) {
       mbar_init(&accfree[b], 4);
     }
     *abort_flag = 0;
+    sh_fail[0] = sh_fail[1] = 0;
     fence_mbar_init();
   }
   if (warp == 2) {
     tmem_alloc(tmem_slot, C::kTmemCols);
     tmem_relinquish();
   }
-  if (warp == 0 && lane == 0) tma_prefetch_desc(&xmap);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -1240,168 +1443,358 @@ tc_planes_kernel(const __grid_constant__ CUtensorMap xmap, const QArgs a) {
   griddep_launch_dependents();
 
   if (warp == 0) {
-    // -------------------------- producer: weights, plane codes, plane scales
+    // ------------------------------------------------- weight producer
+    // (weights never depend on the previous kernel: no wait; gate+up then
+    // down without a break)
     if (lane == 0) {
-      // The weights of the first ring of stages do not depend on the previous
-      // kernel: they are requested before waiting for it (the planes are
-      // its output), so this kernel's CTAs stream weights while that kernel
-      // finishes.  Pass 0 issues those weights, pass 1 everything else.
-      int pre = 0;
-      for (int pass = 0; pass < 2; ++pass) {
-        if (pass == 1) griddep_wait();
+      int st_i = 0;
+      bool ok = true;
+      for (int ph = 0; ph < 2 && ok; ++ph) {
+        const uint8_t* wt = ph ? a.wt_dn : a.wt_gu;
+        const int kc = ph ? a.dn_kc : a.gu_kc;
+        if (ph == 1) {
+          // this CTA's down weights beyond the ring's first fill, into L2
+          // while the gate+up phase drains
+          Seg sg;
+          int skip = S;
+          for (int j = 0; q_segment(a, 1, j, sg); ++j) {
+            for (int c = 0; c < sg.nk; c += kQChunks) {
+              if (skip > 0) {
+                --skip;
+                continue;
+              }
+              const int nch = min(kQChunks, sg.nk - c);
+              asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(
+                               wt + ((size_t)sg.tile * kc + sg.c0 + c) * kChunkBytes),
+                           "r"(nch * kChunkBytes)
+                           : "memory");
+            }
+          }
+        }
         Seg sg;
-        int st_i = 0;
-        bool ok = true;
-        for (int j = 0; ok && range_segment(a.ntiles, a.kc, j, sg); ++j) {
+        for (int j = 0; ok && q_segment(a, ph, j, sg); ++j) {
           for (int c = 0; c < sg.nk; c += kQChunks, ++st_i) {
-            if (pass == 0 && st_i >= S) {
+            const int s = st_i % S, nch = min(kQChunks, sg.nk - c);
+            if (st_i >= S && !mbar_wait(&empty[s], ((st_i / S) - 1) & 1, abort_flag, err, 1)) {
               ok = false;
               break;
             }
-            const int s = st_i % S, nch = min(kQChunks, sg.nk - c);
-            uint8_t* st = smem + s * C::kStageBytes;
-            const int kchunk = sg.c0 + c;
-            if (pass == 0 || st_i >= pre) {
-              if (st_i >= S && !mbar_wait(&empty[s], ((st_i / S) - 1) & 1, abort_flag, err, 1)) {
-                ok = false;
-                break;
-              }
-              mbar_arrive_expect_tx(&full[s], nch * (kChunkBytes + 512) + NT * 128);
-              bulk_load(st, a.wt + ((size_t)sg.tile * a.kc + kchunk) * kChunkBytes, nch * kChunkBytes, &full[s]);
-              if (pass == 0) {
-                ++pre;
-                continue;
-              }
-            }
-            tma_load_2d(st + kW4Chunks * kChunkBytes, &xmap, 32 * kchunk, 0, &full[s]);
-            bulk_load(st + kW4Chunks * kChunkBytes + C::kXBytes, a.sfb + (size_t)kchunk * 512, nch * 512,
-                      &full[s]);
+            mbar_arrive_expect_tx(&full[s], nch * kChunkBytes);
+            bulk_load(smem + s * C::kStageBytes, wt + ((size_t)sg.tile * kc + sg.c0 + c) * kChunkBytes,
+                      nch * kChunkBytes, &full[s]);
           }
         }
-        if (pass == 1)
-          for (int i = max(0, st_i - S); i < st_i; ++i) wait_drain(&full[i % S], (i / S) & 1);
       }
+      for (int i = max(0, st_i - S); i < st_i; ++i) wait_drain(&full[i % S], (i / S) & 1);
     }
   } else if (warp == 1) {
     // ------------------------------------------------------ MMA issuer
+    // accumulator use u: one per segment
     if (lane == 0) {
       const uint32_t idesc = idesc_mxf4nvf4(kTileRows, NT);
-      Seg sg;
-      int st_i = 0;
+      int st_i = 0, u = 0;
       bool ok = true;
-      for (int j = 0; ok && range_segment(a.ntiles, a.kc, j, sg); ++j) {
-        const int buf = j & 1;
-        if (j >= 2 && !mbar_wait(&accfree[buf], ((j >> 1) - 1) & 1, abort_flag, err, 2)) break;
-        tc_fence_after();
+      for (int ph = 0; ph < 2 && ok; ++ph) {
+        Seg sg;
+        for (int j = 0; ok && q_segment(a, ph, j, sg); ++j) {
+          for (int c = 0; c < sg.nk; c += kQChunks, ++st_i) {
+            const int s = st_i % S, nch = min(kQChunks, sg.nk - c);
+            const bool new_acc = c == 0;
+            const int buf = u & 1;
+            if (new_acc && u >= 2 && !mbar_wait(&accfree[buf], ((u >> 1) - 1) & 1, abort_flag, err, 2)) {
+              ok = false;
+              break;
+            }
+            if (!mbar_wait(&full[s], (st_i / S) & 1, abort_flag, err, 2)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            const uint8_t* st = smem + s * C::kStageBytes;
+            const uint8_t* xs = st + kQChunks * kChunkBytes;
+            const uint64_t b_base = smem_desc_sw128(smem_u32(xs));
+            for (int cc = 0; cc < nch; ++cc) {  // the stage's scale copies, then its MMAs
+              const uint32_t slot = 4 * (s * kQChunks + cc);
+              tmem_cp_32x128b_x4(tmem + C::kSfaCol + slot,
+                                 smem_desc_interleave(smem_u32(st + cc * kChunkBytes + 4096), 16, 128));
+              tmem_cp_32x128b_x4(tmem + C::kSfbCol + slot,
+                                 smem_desc_interleave(smem_u32(xs + C::kXBytes + 512 * cc), 16, 128));
+            }
+            for (int cc = 0; cc < nch; ++cc) {
+              const uint32_t slot = 4 * (s * kQChunks + cc);
+              mma_mxf4nvf4(tmem + buf * C::kAccBuf, smem_desc_interleave(smem_u32(st + cc * kChunkBytes), 2048, 128),
+                           b_base + 2 * cc, idesc, tmem + C::kSfaCol + slot, tmem + C::kSfbCol + slot,
+                           (c | cc) != 0 ? 1u : 0u);
+            }
+            mma_commit(&empty[s]);
+            if (c + kQChunks >= sg.nk) {
+              mma_commit(&accfull[buf]);
+              ++u;
+            }
+          }
+        }
+      }
+    }
+  } else if (warp < 4) {
+    // ------- warps 2-3: each stage's B operand (plane codes, 128-byte
+    // swizzle) and SFB, copied from the planes in global memory; warp 2
+    // fills the even stages, warp 3 the odd ones, each with all of a
+    // stage's loads in flight at once.  Down: once every h chunk of this
+    // CTA's range is final, each chunk's scale bytes are re-based from its
+    // own exponent E_c to the segment's E = max E_c (2^-(E - E_c) times,
+    // exact while the scale stays >= 2^-9; a smaller one is flushed to 0)
+    constexpr int kMaxU = NT * 8 / 32;         // 16-byte code units per lane
+    constexpr int kMaxW = NT * kQChunks / 32;  // scale words per lane
+    const int pt = threadIdx.x - 64;
+    const int mine = warp - 2;
+    // plane rows >= m P stay zero (their MMA columns are never read)
+    for (int s = 0; s < S; ++s)
+      for (int i = pt; i < (C::kXBytes + kQChunks * 512) / 16; i += 64)
+        reinterpret_cast<uint4*>(smem + s * C::kStageBytes + kQChunks * kChunkBytes)[i] = make_uint4(0, 0, 0, 0);
+    named_bar_sync(2, 64);  // both warps zeroed before either fills
+    griddep_wait();         // x's planes come from the prologue
+    int st_i = 0;
+    bool ok = true;
+    for (int ph = 0; ph < 2 && ok; ++ph) {
+      const uint8_t* q = ph ? a.hq : a.xq;
+      const uint8_t* qs = ph ? a.hs : a.xs;
+      const int K = ph ? a.inter : a.hidden;
+      Seg sg;
+      if (ph == 1) {  // every h chunk this CTA's down range reads is final
+        bool okr = true;
+        for (int j = 0; okr && q_segment(a, 1, j, sg); ++j)
+          for (int i = lane; okr && i < sg.nk; i += 32) okr = wait_ready(a.ready + sg.c0 + i, abort_flag, err);
+        if (!__all_sync(0xffffffffu, okr)) break;
+      }
+      for (int j = 0; ok && q_segment(a, ph, j, sg); ++j) {
+        int eseg[MR];  // down: the segment's exponent per row
+#pragma unroll
+        for (int jr = 0; jr < MR; ++jr) {
+          int e = kSegZero;
+          if (ph == 1 && jr < a.m)
+            for (int i = lane; i < sg.nk; i += 32) e = max(e, __ldcg(a.he + (size_t)(sg.c0 + i) * a.m + jr));
+#pragma unroll
+          for (int o = 16; o > 0; o >>= 1) e = max(e, __shfl_xor_sync(0xffffffffu, e, o));
+          eseg[jr] = e;
+        }
         for (int c = 0; c < sg.nk; c += kQChunks, ++st_i) {
+          if ((st_i & 1) != mine) continue;
           const int s = st_i % S, nch = min(kQChunks, sg.nk - c);
-          if (!mbar_wait(&full[s], (st_i / S) & 1, abort_flag, err, 2)) {
+          const int cg = sg.c0 + c;  // first chunk of the stage
+          if (st_i >= S &&
+              !__all_sync(0xffffffffu, mbar_wait(&empty[s], ((st_i / S) - 1) & 1, abort_flag, err, 4))) {
             ok = false;
             break;
           }
-          tc_fence_after();
-          const uint8_t* st = smem + s * C::kStageBytes;
-          const uint64_t b_base = smem_desc_sw128(smem_u32(st + kW4Chunks * kChunkBytes));
-          for (int cc = 0; cc < nch; ++cc) {
-            const uint32_t slot = 4 * (s * kQChunks + cc);
-            const uint8_t* wc = st + cc * kChunkBytes;
-            tmem_cp_32x128b_x4(tmem + C::kSfaCol + slot, smem_desc_interleave(smem_u32(wc + 4096), 16, 128));
-            tmem_cp_32x128b_x4(tmem + C::kSfbCol + slot,
-                               smem_desc_interleave(smem_u32(st + kW4Chunks * kChunkBytes + C::kXBytes + 512 * cc),
-                                                    16, 128));
-            mma_mxf4nvf4(tmem + buf * NT, smem_desc_interleave(smem_u32(wc), 2048, 128), b_base + 2 * cc, idesc,
-                         tmem + C::kSfaCol + slot, tmem + C::kSfbCol + slot, (c | cc) != 0 ? 1u : 0u);
+          uint8_t* xs = smem + s * C::kStageBytes + kQChunks * kChunkBytes;
+          uint8_t* sfb = xs + C::kXBytes;
+          // codes: 16-byte units (row, u) of the stage's 128-byte rows
+          uint4 v[kMaxU];
+#pragma unroll
+          for (int k = 0; k < kMaxU; ++k) {
+            const int i = lane + 32 * k, r = i >> 3, u = i & 7;
+            const int byte = cg * 32 + 16 * u;
+            v[k] = make_uint4(0, 0, 0, 0);
+            if (r < rows && u < 2 * nch && byte < K / 2)
+              v[k] = __ldcg(reinterpret_cast<const uint4*>(q + (size_t)r * (K / 2) + byte));
           }
-          mma_commit(&empty[s]);
+          // scale bytes: four per (chunk, row), masked past K; down: with the
+          // chunk's exponent
+          uint32_t w[kMaxW];
+          int ec[kMaxW];
+#pragma unroll
+          for (int k = 0; k < kMaxW; ++k) {
+            const int i = lane + 32 * k, cc = i / rows, r = i - cc * rows;
+            w[k] = 0;
+            ec[k] = kSegZero;
+            if (cc < nch) {
+              const int kleft = K - 64 * (cg + cc);  // > 0
+              w[k] = __ldcg(reinterpret_cast<const uint32_t*>(qs + ((size_t)(cg + cc) * rows + r) * 4));
+              if (kleft < 64) w[k] &= (1u << (8 * (kleft / 16))) - 1u;
+              if (ph == 1) ec[k] = __ldcg(a.he + (size_t)(cg + cc) * a.m + r / P);
+            }
+          }
+#pragma unroll
+          for (int k = 0; k < kMaxU; ++k) {
+            const int i = lane + 32 * k, r = i >> 3, u = i & 7;
+            if (r < rows && u < 2 * nch) *reinterpret_cast<uint4*>(xs + r * 128 + ((u ^ (r & 7)) << 4)) = v[k];
+          }
+#pragma unroll
+          for (int k = 0; k < kMaxW; ++k) {
+            const int i = lane + 32 * k, cc = i / rows, r = i - cc * rows;
+            if (cc < nch) {
+              uint32_t wv = w[k];
+              if (ph == 1 && wv != 0) {
+                const int jr = r / P;
+                const int es = jr == 0 ? eseg[0] : eseg[MR - 1];
+                const int delta = es - ec[k];  // >= 0 (E = max E_c)
+                if (delta != 0 && es != kSegNonFinite) {
+                  uint32_t o = 0;
+#pragma unroll
+                  for (int bi = 0; bi < 4; ++bi) {
+                    const uint32_t b8 = (wv >> (8 * bi)) & 0xffu;
+                    if (b8 == 0) continue;
+                    // power-of-two E4M3: normal (e + 7) << 3, subnormal 1 << (e + 9)
+                    const int e = b8 >= 8 ? (int)(b8 >> 3) - 7 : (b8 == 1 ? -9 : b8 == 2 ? -8 : -7);
+                    const int e2 = e - delta;
+                    const uint32_t n8 = e2 >= -6 ? (uint32_t)(e2 + 7) << 3 : e2 >= -9 ? 1u << (e2 + 9) : 0u;
+                    o |= n8 << (8 * bi);
+                  }
+                  wv = o;
+                }
+              }
+              *reinterpret_cast<uint32_t*>(sfb + 512 * cc + 16 * (r & 31) + 4 * (r >> 5)) = wv;
+            }
+          }
+          asm volatile("fence.proxy.async.shared::cta;" ::: "memory");  // generic writes -> MMA reads
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&full[s]);
         }
-        if (ok) mma_commit(&accfull[buf]);
       }
     }
-  } else if (warp >= 4) {
-    // ----------------------- segment epilogues and the split-K finalisation
+  } else {
+    // ------------- epilogues: gate+up segments (h and its chunk planes),
+    // down stages (fold per chunk), split-K finalisation
     const int q = warp & 3;
     const int row = 32 * q + lane;
     const int tid = threadIdx.x - 128;
     const uint32_t lane_addr = (uint32_t)(32 * q) << 16;
-    bool waited = false;
-    Seg sg;
-    for (int j = 0; range_segment(a.ntiles, a.kc, j, sg); ++j) {
-      const int buf = j & 1;
-      const bool ok = __all_sync(0xffffffffu, wait_drain(&accfull[buf], (j >> 1) & 1));
-      tc_fence_after();
-      if (!waited) {
-        griddep_wait();  // the previous kernel may still read this kernel's outputs
-        waited = true;
-      }
-      if (!ok || *abort_flag) break;
-      uint32_t d[NT];
+    griddep_wait();  // the prologue (and so every earlier kernel) is complete
+    int xe[MR];
 #pragma unroll
-      for (int c = 0; c < NT / 16; ++c) {
-        uint32_t v[16];
-        tmem_ld16(tmem + lane_addr + buf * NT + 16 * c, v);
+    for (int jr = 0; jr < MR; ++jr) xe[jr] = jr < a.m ? __ldcg(a.xe + jr) : kSegZero;
+    int u = 0, segs = 0;
+    bool dead = false;  // a wait of this warp expired: skip the remaining waits
+    bool fail = false;
+    for (int ph = 0; ph < 2 && !fail; ++ph) {
+      const int nt = ph ? a.dn_tiles : a.gu_tiles, kc = ph ? a.dn_kc : a.gu_kc;
+      const int parts = ph ? (int)gridDim.x : a.gu_parts;
+      const uint32_t W = (uint32_t)nt * kc;
+      Seg sg;
+      for (int j = 0; q_segment(a, ph, j, sg); ++j, ++segs) {
+        float y[MR];
 #pragma unroll
-        for (int i = 0; i < 16; ++i) d[16 * c + i] = v[i];
-      }
-      tmem_ld_wait();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&accfree[buf]);  // the MMAs may reuse the accumulator
-      // fold the planes (p ascending): partial[slot][jr][row] = sum_p g[jr, p] * D[row, jr * P + p]
-      float* Pp = a.partials + (size_t)(blockIdx.x + sg.tile) * a.m * kTileRows;
+        for (int jr = 0; jr < MR; ++jr) y[jr] = 0.0f;
+        // the segment's accumulator, after its last stage
+        {
+          const int buf = u & 1;
+          if (!dead) dead = !__all_sync(0xffffffffu, mbar_wait(&accfull[buf], (u >> 1) & 1, abort_flag, err, 16));
+          tc_fence_after();
+          uint32_t d[NT];
+          tmem_ld16(tmem + lane_addr + buf * C::kAccBuf, d);
+          // down: the segment's exponent per row, E = max E_c over its chunks
+          // (the chunks are final: their planes fed these MMAs)
+          int E[MR];
 #pragma unroll
-      for (int jr = 0; jr < MR; ++jr) {
-        if (jr < a.m) {
-          float y = 0.0f;
+          for (int jr = 0; jr < MR; ++jr) {
+            int e = kSegZero;
+            if (ph == 1 && jr < a.m)
+              for (int i = lane; i < sg.nk; i += 32) e = max(e, __ldcg(a.he + (size_t)(sg.c0 + i) * a.m + jr));
 #pragma unroll
-          for (int p = 0; p < P; ++p) y = fmaf(__ldg(a.g + jr * P + p), __uint_as_float(d[jr * P + p]), y);
-          Pp[(size_t)jr * kTileRows + row] = y;
-        }
-      }
-      __threadfence();
-      named_bar_sync(1, 128);
-      if (tid == 0) {
-        const int64_t W = (int64_t)a.ntiles * a.kc;
-        const int G = gridDim.x;
-        const int g0 = range_owner((int64_t)sg.tile * a.kc, W, G);
-        const int g1 = range_owner((int64_t)sg.tile * a.kc + a.kc - 1, W, G);
-        *last_flag = atomicAdd(&a.counters[sg.tile], 1) == g1 - g0 ? 1 : 0;
-      }
-      named_bar_sync(1, 128);
-      if (*last_flag) {
-        __threadfence();
-        const int64_t W = (int64_t)a.ntiles * a.kc;
-        const int G = gridDim.x;
-        const int g0 = range_owner((int64_t)sg.tile * a.kc, W, G);
-        const int g1 = range_owner((int64_t)sg.tile * a.kc + a.kc - 1, W, G);
-        if (kGateUp) {
-          // h[jr, 64t + r] from gate row r and up row r + 64 of the tile
-          for (int idx = tid; idx < a.m * 64; idx += 128) {
-            const int jr = idx / 64, rr = idx % 64;
-            const int n = 64 * sg.tile + rr;
-            if (n >= a.n_out) continue;
-            float gsum = 0.0f, usum = 0.0f;
-            for (int gg = g0; gg <= g1; ++gg) {
-              const float* Pt = a.partials + ((size_t)(gg + sg.tile) * a.m + jr) * kTileRows;
-              gsum += __ldcg(Pt + rr);
-              usum += __ldcg(Pt + rr + 64);
-            }
-            const float gv = lora_add(bf16_round(a.gs[0] * gsum), a.lora.b0, a.lora.off0, a.lora, jr, n);
-            const float uv = lora_add(bf16_round(a.gs[1] * usum), a.lora.b1, a.lora.off1, a.lora, jr, n);
-            a.out[(size_t)jr * a.ldo + n] = f32_to_bf16_bits(silu_fast(gv) * uv);
+            for (int o = 16; o > 0; o >>= 1) e = max(e, __shfl_xor_sync(0xffffffffu, e, o));
+            E[jr] = ph ? e : xe[jr];
           }
+          tmem_ld_wait();
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&accfree[buf]);  // the MMAs may reuse the accumulator
+          ++u;
+          // fold the planes (p ascending): y[jr] = sum_p g_p * D[row, jr P + p]
+#pragma unroll
+          for (int jr = 0; jr < MR; ++jr) {
+            if (jr < a.m) {
+              if (E[jr] == kSegNonFinite) {
+                y[jr] = __int_as_float(0x7fc00000);  // a non-finite activation
+              } else if (E[jr] != kSegZero) {
+#pragma unroll
+                for (int p = 0; p < P; ++p) y[jr] = fmaf(exp2i(E[jr] - 8 - (3 * p) / 2), __uint_as_float(d[jr * P + p]), y[jr]);
+              }
+            }
+          }
+        }
+        // the segment's sums are in y: stop together if a wait expired
+        if (lane == 0 && (dead || *abort_flag)) sh_fail[segs & 1] = 1;
+        named_bar_sync(1, 128);
+        if (sh_fail[segs & 1]) {
+          fail = true;
+          break;
+        }
+        const int g0 = (int)((((uint64_t)sg.tile * kc + 1) * parts - 1) / W);  // owner of the tile's first chunk
+        const int g1 = (int)((((uint64_t)sg.tile * kc + kc) * parts - 1) / W);  // and of its last
+        bool have = sg.nk == kc;  // a whole tile: its sums are final here
+        float* part = ph ? a.part_dn : a.part_gu;
+        if (!have) {
+          float* Pp = part + (size_t)(blockIdx.x + sg.tile) * a.m * kTileRows;
+#pragma unroll
+          for (int jr = 0; jr < MR; ++jr)
+            if (jr < a.m) Pp[(size_t)jr * kTileRows + row] = y[jr];
+          __threadfence();
+          named_bar_sync(1, 128);
+          // the tile is complete when its counter reaches kc chunks
+          if (tid == 0) *last_flag = atomicAdd((ph ? a.cnt_dn : a.cnt_gu) + sg.tile, sg.nk) + sg.nk == kc ? 1 : 0;
+          named_bar_sync(1, 128);
+          have = *last_flag != 0;
+          if (have) __threadfence();
+        }
+        if (!have) continue;
+        if (ph == 1) {
+          // out[jr, 128 t + r]
+          if (sg.nk == kc) {
+            const int n = kTileRows * sg.tile + row;
+#pragma unroll
+            for (int jr = 0; jr < MR; ++jr)
+              if (jr < a.m && n < a.hidden) a.out[(size_t)jr * a.hidden + n] = f32_to_bf16_bits(a.gs_dn[0] * y[jr]);
+          } else {
+            for (int idx = tid; idx < a.m * kTileRows; idx += 128) {
+              const int jr = idx / kTileRows, rr = idx % kTileRows;
+              const int n = kTileRows * sg.tile + rr;
+              if (n < a.hidden)
+                a.out[(size_t)jr * a.hidden + n] =
+                    f32_to_bf16_bits(a.gs_dn[0] * sum_partials(part, a.m, jr, rr, sg.tile, W, parts, g0, g1));
+            }
+          }
+          continue;
+        }
+        // gate+up tile t final: Y[jr][r] = its sums (gate r, up r + 64)
+        if (sg.nk == kc) {
+#pragma unroll
+          for (int jr = 0; jr < MR; ++jr)
+            if (jr < a.m) Y[jr * kTileRows + row] = y[jr];
         } else {
           for (int idx = tid; idx < a.m * kTileRows; idx += 128) {
             const int jr = idx / kTileRows, rr = idx % kTileRows;
-            const int n = kTileRows * sg.tile + rr;
-            if (n >= a.n_out) continue;
-            float sum = 0.0f;
-            for (int gg = g0; gg <= g1; ++gg)
-              sum += __ldcg(a.partials + ((size_t)(gg + sg.tile) * a.m + jr) * kTileRows + rr);
-            float y = a.gs[0] * sum;
-            if (a.lora.b0) y = lora_add(bf16_round(y), a.lora.b0, a.lora.off0, a.lora, jr, n);
-            a.out[(size_t)jr * a.ldo + n] = f32_to_bf16_bits(y);
+            Y[jr * kTileRows + rr] = sum_partials(part, a.m, jr, rr, sg.tile, W, parts, g0, g1);
           }
         }
+        named_bar_sync(1, 128);
+        // warp q = activation row jr: lanes take h columns 64 t + 2 lane, +1,
+        // find the chunk's exponent and write its planes (eight lanes per
+        // 16-block)
+        if (q < a.m) {
+          const int jr = q;
+          float hv[2];
+#pragma unroll
+          for (int e = 0; e < 2; ++e) {
+            const int r = 2 * lane + e, n = 64 * sg.tile + r;
+            hv[e] = 0.0f;
+            if (n < a.inter) {
+              const float gv = bf16_round(a.gs_gu[0] * Y[jr * kTileRows + r]);
+              const float uv = bf16_round(a.gs_gu[1] * Y[jr * kTileRows + 64 + r]);
+              hv[e] = bf16_round(silu_fast(gv) * uv);
+            }
+          }
+          uint32_t mx = max(f32_to_bf16_bits(hv[0]) & 0x7fffu, f32_to_bf16_bits(hv[1]) & 0x7fffu);
+#pragma unroll
+          for (int o = 16; o > 0; o >>= 1) mx = max(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+          const int E = row_exponent(mx);
+          if (E == kSegNonFinite) hv[0] = hv[1] = 0.0f;
+          const int b = 4 * sg.tile + (lane >> 3);
+          block_planes(hv[0], hv[1], E, b < a.inter / 16, lane & 7, jr, b, a.hq, (size_t)a.inter / 2, a.hs, rows);
+          if (lane == 0) a.he[(size_t)sg.tile * a.m + jr] = E;
+        }
+        __threadfence();
+        named_bar_sync(1, 128);
+        if (tid == 0) asm volatile("st.release.gpu.global.b32 [%0], %1;" ::"l"(a.ready + sg.tile), "r"(1) : "memory");
       }
     }
   }
@@ -1632,126 +2025,104 @@ cudaError_t launch_persist_bn(int bn, const CUtensorMap& map, const PArgs& a, in
   }
 }
 
-template <int NT, int P, bool kGateUp>
-cudaError_t launch_planes_cfg(const CUtensorMap& map, const QArgs& a, int grid, cudaStream_t s) {
-  using C = QCfg<NT>;
-  auto kern = tc_planes_kernel<NT, P, kGateUp>;
+// The down phase waits for chunks that other CTAs finish, so every CTA must
+// be resident at once: the grid is the occupancy (two CTAs per SM, with the
+// shared-memory carveout at its maximum) times the SMs, at most `max_grid`
+// (what the workspace was sized for).
+cudaError_t launch_layer(LArgs a, int max_grid, int num_sms, cudaStream_t s) {
+  using C = QCfg;
+  auto kern = tc_planes_layer_kernel;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemAlloc);
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout, cudaSharedmemCarveoutMaxShared);
+  int dev = 0, smem_sm = 0;
+  if (e == cudaSuccess) e = cudaGetDevice(&dev);
+  if (e == cudaSuccess) e = cudaDeviceGetAttribute(&smem_sm, cudaDevAttrMaxSharedMemoryPerMultiprocessor, dev);
   if (e != cudaSuccess) return e;
-  return launch_pdl(kern, dim3(grid), dim3(256), C::kSmemAlloc, s, map, a);
-}
-
-template <bool kGateUp>
-cudaError_t launch_planes_nt(int nt, int planes, const CUtensorMap& map, const QArgs& a, int grid,
-                             cudaStream_t s) {
-  (void)planes;  // 8 per row
-  if (nt == 16) return launch_planes_cfg<16, 8, kGateUp>(map, a, grid, s);
-  if (nt == 32) return launch_planes_cfg<32, 8, kGateUp>(map, a, grid, s);
-  return launch_planes_cfg<64, 8, kGateUp>(map, a, grid, s);
-}
-
-// 2-D map over plane codes [rows, k/2] bytes with a 128-byte x nt-row box and
-// the 128-byte swizzle (the MMA's B operand layout).
-bool make_planes_map(CUtensorMap* map, const void* codes, int64_t rows, int64_t k, int nt) {
-  auto enc = get_encode();
-  if (!enc) return false;
-  cuuint64_t dims[2] = {(cuuint64_t)(k / 2), (cuuint64_t)rows};
-  cuuint64_t strides[1] = {(cuuint64_t)(k / 2)};
-  cuuint32_t box[2] = {128, (cuuint32_t)nt};
-  cuuint32_t estr[2] = {1, 1};
-  return enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(codes), dims, strides, box, estr,
-             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+  // registers: __launch_bounds__(256, 2) keeps two CTAs within the register
+  // file; threads: 512 of 2048; shared memory (1 KB per CTA reserved):
+  const int occupancy = 2 * (C::kSmemAlloc + 1024) <= smem_sm ? 2 : 1;
+  const int grid = min(max_grid, occupancy * num_sms);
+  if (grid < 1) return cudaErrorInvalidConfiguration;
+  a.gu_parts = min(a.gu_parts, grid);
+  return launch_pdl(kern, dim3(grid), dim3(256), C::kSmemAlloc, s, a);
 }
 
 }  // namespace
 
 int tc_tile_bytes_per_row_chunk() { return kChunkBytes; }
 
+int planes_for_rows(int64_t m) { return m <= QCfg::kMR ? kQPlanes : 0; }
+
 PlanesPlan plan_planes(int64_t m, int64_t hidden, int64_t inter, int num_sms) {
   PlanesPlan p;
   p.planes = planes_for_rows(m);
   if (!p.planes) return p;
-  const int64_t cols = m * p.planes;
-  p.nt = cols <= 16 ? 16 : cols <= 32 ? 32 : 64;
+  p.nt = QCfg::kNT;
+  p.rows = (int)(m * p.planes);
   p.gu_tiles = (int)((inter + 63) / 64);
   p.gu_kc = (int)((hidden + kChunkK - 1) / kChunkK);
   p.dn_tiles = (int)((hidden + kTileRows - 1) / kTileRows);
   p.dn_kc = (int)((inter + kChunkK - 1) / kChunkK);
-  const int64_t slots = 2LL * num_sms, Wg = (int64_t)p.gu_tiles * p.gu_kc, Wd = (int64_t)p.dn_tiles * p.dn_kc;
-  p.gu_grid = (int)(Wg < slots ? Wg : slots);
-  p.dn_grid = (int)(Wd < slots ? Wd : slots);
-  const size_t pg = (size_t)(p.gu_grid + p.gu_tiles) * m * kTileRows * sizeof(float);
-  const size_t pd = (size_t)(p.dn_grid + p.dn_tiles) * m * kTileRows * sizeof(float);
-  p.partial_bytes = pg > pd ? pg : pd;
-  p.counter_count = p.gu_tiles + p.dn_tiles;
+  p.grid = 2 * num_sms;  // at most two CTAs per SM, all resident
+  // gate+up: whole tiles when they do not outnumber the CTAs
+  p.gu_parts = p.gu_tiles <= p.grid ? p.gu_tiles : p.grid;
+  p.gu_partial_bytes = (size_t)(p.gu_parts + p.gu_tiles) * m * kTileRows * sizeof(float);
+  p.dn_partial_bytes = (size_t)(p.grid + p.dn_tiles) * m * kTileRows * sizeof(float);
+  p.x_code_bytes = (size_t)p.rows * (size_t)(hidden / 2);
+  p.x_sf_bytes = (size_t)p.gu_kc * p.rows * 4;
+  p.h_code_bytes = (size_t)p.rows * (size_t)(inter / 2);
+  p.h_sf_bytes = (size_t)p.dn_kc * p.rows * 4;
+  p.zero_ints = p.gu_tiles + p.dn_tiles + p.gu_tiles;  // tile counters, h chunk ready flags
+  p.other_ints = (int)m + p.gu_tiles * (int)m;          // x's row exponents, h's chunk exponents
   return p;
 }
 
 cudaError_t launch_planes_ffn(const void* x, int64_t m, const TcWeight& gate_up, const TcWeight& down,
-                              const PlanesPlan& p, const PlanesBuffers& b, void* out, cudaStream_t s,
-                              const LoraView& lv) {
+                              const PlanesPlan& p, const PlanesBuffers& b, void* out, cudaStream_t s) {
   const int64_t hidden = down.n, inter = gate_up.n / 2;
-  const int rows = (int)(m * p.planes);
-  CUtensorMap xm, hm;
-  if (!make_planes_map(&xm, b.x_codes, rows, hidden, p.nt) || !make_planes_map(&hm, b.h_codes, rows, inter, p.nt))
+  if (hidden % 32 || inter % 32) return cudaErrorInvalidValue;
+  // 32-bit range arithmetic in the kernel
+  if ((uint64_t)p.gu_tiles * p.gu_kc * p.grid >= (1ull << 32) || (uint64_t)p.dn_tiles * p.dn_kc * p.grid >= (1ull << 32))
     return cudaErrorInvalidValue;
-  int* gu_cnt = b.counters;
-  int* dn_cnt = b.counters + p.gu_tiles;
-  cudaError_t e = launch_quantize_planes(x, m, hidden, p.planes, b.x_codes, b.x_sf, b.x_g, gu_cnt, p.gu_tiles, s);
-  QArgs a{};
-  a.wt = gate_up.tiled;
-  a.gs = gate_up.gs;
-  a.out = static_cast<uint16_t*>(b.h);
-  a.m = (int)m;
-  a.n_out = (int)inter;
-  a.ldo = (int)inter;
-  a.kc = p.gu_kc;
-  a.ntiles = p.gu_tiles;
-  a.planes = p.planes;
-  a.sfb = static_cast<const uint8_t*>(b.x_sf);
-  a.g = b.x_g;
-  a.partials = static_cast<float*>(b.partials);
-  a.counters = gu_cnt;
-  if (e == cudaSuccess && lv.rank > 0 && lv.a_gu) {
-    e = launch_lora_xa(x, m, hidden, lv.a_gu, 2 * lv.rank, b.xa_gu, s);
-    a.lora.xa = static_cast<const uint16_t*>(b.xa_gu);
-    a.lora.xa_ld = 2 * lv.rank;
-    a.lora.b0 = lv.b_g;
-    a.lora.b1 = lv.b_u;
-    a.lora.off1 = lv.rank;
-    a.lora.r = lv.rank;
-  }
-  if (e == cudaSuccess) {
-    ProfScope prof(s, "tc_planes_gate_up_silu");
-    e = launch_planes_nt<true>(p.nt, p.planes, xm, a, p.gu_grid, s);
-  }
-  if (e == cudaSuccess)
-    e = launch_quantize_planes(b.h, m, inter, p.planes, b.h_codes, b.h_sf, b.h_g, dn_cnt, p.dn_tiles, s);
-  QArgs d{};
-  d.wt = down.tiled;
-  d.gs = down.gs;
-  d.out = static_cast<uint16_t*>(out);
-  d.m = (int)m;
-  d.n_out = (int)hidden;
-  d.ldo = (int)hidden;
-  d.kc = p.dn_kc;
-  d.ntiles = p.dn_tiles;
-  d.planes = p.planes;
-  d.sfb = static_cast<const uint8_t*>(b.h_sf);
-  d.g = b.h_g;
-  d.partials = static_cast<float*>(b.partials);
-  d.counters = dn_cnt;
-  if (e == cudaSuccess && lv.rank > 0 && lv.a_d) {
-    e = launch_lora_xa(b.h, m, inter, lv.a_d, lv.rank, b.xa_d, s);
-    d.lora.xa = static_cast<const uint16_t*>(b.xa_d);
-    d.lora.xa_ld = lv.rank;
-    d.lora.b0 = lv.b_d;
-    d.lora.r = lv.rank;
+  int* zero = b.ints;  // [cnt_gu][cnt_dn][ready] zeroed, then x's E [m], h's E [gu_tiles][m]
+  int* xe = zero + p.zero_ints;
+  cudaError_t e;
+  {
+    ProfScope prof(s, "planes_prologue");
+    const dim3 grid((unsigned)m, (unsigned)((hidden / 16 + kPlaneThreads / 8 - 1) / (kPlaneThreads / 8)));
+    e = launch_pdl(planes_prologue_kernel, grid, dim3(kPlaneThreads), 0, s, static_cast<const uint16_t*>(x),
+                   (int)m, (int)hidden, static_cast<uint8_t*>(b.xq), static_cast<uint8_t*>(b.xs), xe, zero,
+                   p.zero_ints);
   }
   if (e != cudaSuccess) return e;
-  ProfScope prof(s, "tc_planes_down");
-  return launch_planes_nt<false>(p.nt, p.planes, hm, d, p.dn_grid, s);
+  LArgs a{};
+  a.wt_gu = gate_up.tiled;
+  a.wt_dn = down.tiled;
+  a.gs_gu = gate_up.gs;
+  a.gs_dn = down.gs;
+  a.xq = static_cast<const uint8_t*>(b.xq);
+  a.xs = static_cast<const uint8_t*>(b.xs);
+  a.xe = xe;
+  a.hq = static_cast<uint8_t*>(b.hq);
+  a.hs = static_cast<uint8_t*>(b.hs);
+  a.he = xe + m;
+  a.out = static_cast<uint16_t*>(out);
+  a.part_gu = static_cast<float*>(b.part_gu);
+  a.part_dn = static_cast<float*>(b.part_dn);
+  a.cnt_gu = zero;
+  a.cnt_dn = zero + p.gu_tiles;
+  a.ready = a.cnt_dn + p.dn_tiles;
+  a.m = (int)m;
+  a.hidden = (int)hidden;
+  a.inter = (int)inter;
+  a.gu_tiles = p.gu_tiles;
+  a.gu_kc = p.gu_kc;
+  a.gu_parts = p.gu_parts;
+  a.dn_tiles = p.dn_tiles;
+  a.dn_kc = p.dn_kc;
+  ProfScope prof(s, "tc_planes_layer");
+  return launch_layer(a, p.grid, p.grid / 2, s);
 }
 
 PersistPlan plan_persist(int64_t m, int64_t hidden, int64_t inter, int num_sms) {

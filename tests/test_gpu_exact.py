@@ -164,8 +164,8 @@ def exact_ffn_inputs(rng, m, H, I, down_nonzeros=4):
 
 FFN_EXACT_CASES = [
     # (m, hidden, inter, handle formats): m <= 8 with both layouts runs the
-    # block-scaled FP4 kernels with activation planes (m = 1: 16 planes; 2..8:
-    # 8), bf16-only handles the per-tile kernels at the same m; tile widths
+    # block-scaled FP4 layer kernel with 8 activation planes per row,
+    # bf16-only handles the per-tile kernels at the same m; tile widths
     # 16/32/64 per-tile, down K ranges that cut tiles, inter % 64 == 32, and
     # split-K with the SiLU*mul reduction for wider m
     (1, 512, 1536, "all"), (2, 512, 800, "all"), (5, 1024, 4096, "all"), (8, 512, 1536, "all"),
@@ -186,8 +186,11 @@ def test_ffn_exact_inputs_bit_exact(native, m, H, I, formats):
     got = bf16_to_f64(out)
     bad = np.argwhere(got != ref)
     plan = native.ffn_nvfp4_projection_plan(m, H, I, "bf16", role="down")
-    assert bad.size == 0, f"{plan}: {len(bad)} mismatches, first at {bad[:3].tolist()}"
-    assert native.ffn_nvfp4_device_error(clear=False) == 0
+    err = native.ffn_nvfp4_device_error(clear=False)
+    assert bad.size == 0, (f"{plan}: {len(bad)} mismatches, first at {bad[:3].tolist()}: got "
+                           f"{[got[tuple(b)] for b in bad[:3]]}, want {[ref[tuple(b)] for b in bad[:3]]}; "
+                           f"device error bits {err}")
+    assert err == 0
 
 
 def test_persistent_path_bit_exact_in_subprocess(native):
