@@ -1179,14 +1179,14 @@ tc_w4a4_kernel(const __grid_constant__ CUtensorMap xmap, const W4Args w4) {
 //    CTA completing a tile's count adds in K order.  The CTA that finishes
 //    tile t computes h = bf16(silu(bf16 g) * bf16 u) for its 64 columns and
 //    at once the planes of that 64-column chunk of h, with the chunk's own
-//    exponent per row, then raises the chunk's ready flag;
-//  * down: equal ranges of its (tile, chunk) space; a stage of chunks is
-//    copied in once their flags are up (no grid-wide barrier), each chunk
-//    goes to its own accumulator, and the epilogue folds every stage with
-//    the chunks' exponents; split-K partial sums as above.
-// Each CTA's weight stream runs through both projections without a break,
-// and once its gate+up loads are issued it prefetches its down weights into
-// L2.  Every wait is bounded and raises a device error bit when it expires.
+//    exponent per row, then counts the tile as done;
+//  * down: equal ranges of its (tile, chunk) space, started once every
+//    gate+up tile is counted (one word, polled by one thread per CTA with a
+//    back-off; no grid-wide barrier otherwise).  The copy warps re-base each
+//    chunk's power-of-two scale bytes onto the segment's largest exponent,
+//    so a segment keeps one accumulator; split-K partial sums as above.
+// Each CTA's weight stream runs through both projections without a break.
+// Every wait is bounded and raises a device error bit when it expires.
 // ---------------------------------------------------------------------------
 constexpr int kQChunks = 4;   // 64-element chunks per stage
 constexpr int kQPlanes = 8;   // activation planes per row
@@ -1206,8 +1206,10 @@ struct QCfg {
   static constexpr int kSmemBar = kSmemY + kMR * 128 * 4;
   static constexpr int kNumBars = 2 * kStages + 4;       // full, empty, accfull[2], accfree[2]
   static constexpr int kSmemAlloc = kSmemBar + kNumBars * 8 + 32 + 1024;
-  // TMEM: two accumulator buffers, then the scale-factor columns
-  static constexpr int kAccBuf = kNT;
+  // TMEM: two accumulator buffers (one accumulator per MMA-issuing warp in
+  // each), then the scale-factor columns
+  static constexpr int kIssuers = 2;
+  static constexpr int kAccBuf = kIssuers * kNT;
   static constexpr int kSfaCol = 2 * kAccBuf;
   static constexpr int kSfbCol = kSfaCol + 4 * kQChunks * kStages;
   static constexpr int kTmemCols = 256;
@@ -1343,7 +1345,7 @@ struct LArgs {
   float* part_dn;        // [gridDim.x + dn_tiles][m][128]
   int* cnt_gu;           // [gu_tiles] chunks done, zero on entry
   int* cnt_dn;           // [dn_tiles]
-  int* ready;            // [gu_tiles] h chunk's planes written, zero on entry
+  uint32_t* gu_done;     // gate+up tiles whose h planes are written, zero on entry
   int m, hidden, inter, gu_tiles, gu_kc, gu_parts, dn_tiles, dn_kc;
 };
 
@@ -1373,18 +1375,19 @@ __device__ __forceinline__ int ld_acquire(const int* p) {
   return v;
 }
 
-// Bounded wait for a chunk's ready flag.
-__device__ __forceinline__ bool wait_ready(const int* flag, volatile int* abort, int* err) {
-  if (ld_acquire(flag)) return true;
+// Bounded wait until *ctr reaches `target`, polling with a back-off (one
+// thread per CTA polls one word).
+__device__ __forceinline__ bool wait_count(const uint32_t* ctr, uint32_t target, volatile int* abort, int* err) {
   const long long t0 = clock64();
   for (;;) {
-    if (ld_acquire(flag)) return true;
+    if ((uint32_t)ld_acquire(reinterpret_cast<const int*>(ctr)) >= target) return true;
     if (*abort) return false;
     if (clock64() - t0 > kWaitLimitCycles) {
       *abort = 1;
       atomicOr(err, 32);
       return false;
     }
+    __nanosleep(256);
   }
 }
 
@@ -1399,7 +1402,8 @@ __device__ __forceinline__ float sum_partials(const float* part, int m, int jr, 
   return sum;
 }
 
-__global__ void __launch_bounds__(256, 2) tc_planes_layer_kernel(const LArgs a) {
+constexpr int kLayerThreads = 288;  // 9 warps
+__global__ void __launch_bounds__(kLayerThreads, 2) tc_planes_layer_kernel(const LArgs a) {
   using C = QCfg;
   constexpr int S = C::kStages, P = kQPlanes, MR = C::kMR, NT = C::kNT;
   extern __shared__ uint8_t smem_raw[];
@@ -1408,6 +1412,7 @@ __global__ void __launch_bounds__(256, 2) tc_planes_layer_kernel(const LArgs a) 
   int* misc = reinterpret_cast<int*>(smem + C::kSmemMisc);
   volatile int* sh_fail = misc;            // [2] epilogue stop flags by segment parity
   volatile int* last_flag = misc + 2;
+  volatile int* sh_ready = misc + 3;      // the down phase's inputs are final
   float* Y = reinterpret_cast<float*>(smem + C::kSmemY);  // [MR][128] a finished tile's sums
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::kSmemBar);
   uint64_t* empty = full + S;
@@ -1425,7 +1430,7 @@ __global__ void __launch_bounds__(256, 2) tc_planes_layer_kernel(const LArgs a) 
       mbar_init(&empty[s], 1);
     }
     for (int b = 0; b < 2; ++b) {
-      mbar_init(&accfull[b], 1);
+      mbar_init(&accfull[b], C::kIssuers);
       mbar_init(&accfree[b], 4);
     }
     *abort_flag = 0;
@@ -1452,25 +1457,6 @@ __global__ void __launch_bounds__(256, 2) tc_planes_layer_kernel(const LArgs a) 
       for (int ph = 0; ph < 2 && ok; ++ph) {
         const uint8_t* wt = ph ? a.wt_dn : a.wt_gu;
         const int kc = ph ? a.dn_kc : a.gu_kc;
-        if (ph == 1) {
-          // this CTA's down weights beyond the ring's first fill, into L2
-          // while the gate+up phase drains
-          Seg sg;
-          int skip = S;
-          for (int j = 0; q_segment(a, 1, j, sg); ++j) {
-            for (int c = 0; c < sg.nk; c += kQChunks) {
-              if (skip > 0) {
-                --skip;
-                continue;
-              }
-              const int nch = min(kQChunks, sg.nk - c);
-              asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(
-                               wt + ((size_t)sg.tile * kc + sg.c0 + c) * kChunkBytes),
-                           "r"(nch * kChunkBytes)
-                           : "memory");
-            }
-          }
-        }
         Seg sg;
         for (int j = 0; ok && q_segment(a, ph, j, sg); ++j) {
           for (int c = 0; c < sg.nk; c += kQChunks, ++st_i) {
@@ -1487,24 +1473,31 @@ __global__ void __launch_bounds__(256, 2) tc_planes_layer_kernel(const LArgs a) 
       }
       for (int i = max(0, st_i - S); i < st_i; ++i) wait_drain(&full[i % S], (i / S) & 1);
     }
-  } else if (warp == 1) {
-    // ------------------------------------------------------ MMA issuer
+  } else if (warp == 1 || warp == 8) {
+    // ---------------------- MMA issuers: warp 1 the even stages, warp 8 the
+    // odd ones, each into its own accumulator of the segment's buffer (two
+    // instruction streams: one thread's tcgen05 issue rate is the limit)
     // accumulator use u: one per segment
     if (lane == 0) {
+      const int mi = warp == 1 ? 0 : 1;
       const uint32_t idesc = idesc_mxf4nvf4(kTileRows, NT);
       int st_i = 0, u = 0;
       bool ok = true;
       for (int ph = 0; ph < 2 && ok; ++ph) {
         Seg sg;
-        for (int j = 0; ok && q_segment(a, ph, j, sg); ++j) {
+        for (int j = 0; ok && q_segment(a, ph, j, sg); ++j, ++u) {
+          const int buf = u & 1;
+          // every issuer waits for every segment's buffer (parity waits must
+          // not skip a phase)
+          if (u >= 2 && !mbar_wait(&accfree[buf], ((u >> 1) - 1) & 1, abort_flag, err, 2)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          bool first = true;
           for (int c = 0; c < sg.nk; c += kQChunks, ++st_i) {
+            if ((st_i & 1) != mi) continue;
             const int s = st_i % S, nch = min(kQChunks, sg.nk - c);
-            const bool new_acc = c == 0;
-            const int buf = u & 1;
-            if (new_acc && u >= 2 && !mbar_wait(&accfree[buf], ((u >> 1) - 1) & 1, abort_flag, err, 2)) {
-              ok = false;
-              break;
-            }
             if (!mbar_wait(&full[s], (st_i / S) & 1, abort_flag, err, 2)) {
               ok = false;
               break;
@@ -1522,16 +1515,14 @@ __global__ void __launch_bounds__(256, 2) tc_planes_layer_kernel(const LArgs a) 
             }
             for (int cc = 0; cc < nch; ++cc) {
               const uint32_t slot = 4 * (s * kQChunks + cc);
-              mma_mxf4nvf4(tmem + buf * C::kAccBuf, smem_desc_interleave(smem_u32(st + cc * kChunkBytes), 2048, 128),
-                           b_base + 2 * cc, idesc, tmem + C::kSfaCol + slot, tmem + C::kSfbCol + slot,
-                           (c | cc) != 0 ? 1u : 0u);
+              mma_mxf4nvf4(tmem + buf * C::kAccBuf + mi * NT,
+                           smem_desc_interleave(smem_u32(st + cc * kChunkBytes), 2048, 128), b_base + 2 * cc, idesc,
+                           tmem + C::kSfaCol + slot, tmem + C::kSfbCol + slot, (!first || cc != 0) ? 1u : 0u);
             }
+            first = false;
             mma_commit(&empty[s]);
-            if (c + kQChunks >= sg.nk) {
-              mma_commit(&accfull[buf]);
-              ++u;
-            }
           }
+          if (ok) mma_commit(&accfull[buf]);  // (also when this issuer had no stage in the segment)
         }
       }
     }
@@ -1555,16 +1546,20 @@ __global__ void __launch_bounds__(256, 2) tc_planes_layer_kernel(const LArgs a) 
     griddep_wait();         // x's planes come from the prologue
     int st_i = 0;
     bool ok = true;
-    for (int ph = 0; ph < 2 && ok; ++ph) {
+    for (int ph = 0; ph < 2; ++ph) {
       const uint8_t* q = ph ? a.hq : a.xq;
       const uint8_t* qs = ph ? a.hs : a.xs;
       const int K = ph ? a.inter : a.hidden;
       Seg sg;
-      if (ph == 1) {  // every h chunk this CTA's down range reads is final
-        bool okr = true;
-        for (int j = 0; okr && q_segment(a, 1, j, sg); ++j)
-          for (int i = lane; okr && i < sg.nk; i += 32) okr = wait_ready(a.ready + sg.c0 + i, abort_flag, err);
-        if (!__all_sync(0xffffffffu, okr)) break;
+      if (ph == 1) {
+        // every h chunk is final once all gate+up tiles are counted: warp 2
+        // polls, warp 3 waits at the barrier (both always reach it)
+        if (mine == 0 && lane == 0) {
+          const bool has_down = q_segment(a, 1, 0, sg);
+          *sh_ready = ok && (!has_down || wait_count(a.gu_done, a.gu_tiles, abort_flag, err)) ? 1 : 0;
+        }
+        named_bar_sync(2, 64);
+        if (!*sh_ready) ok = false;
       }
       for (int j = 0; ok && q_segment(a, ph, j, sg); ++j) {
         int eseg[MR];  // down: the segment's exponent per row
@@ -1663,7 +1658,7 @@ __global__ void __launch_bounds__(256, 2) tc_planes_layer_kernel(const LArgs a) 
     int xe[MR];
 #pragma unroll
     for (int jr = 0; jr < MR; ++jr) xe[jr] = jr < a.m ? __ldcg(a.xe + jr) : kSegZero;
-    int u = 0, segs = 0;
+    int u = 0, segs = 0, st_i = 0;
     bool dead = false;  // a wait of this warp expired: skip the remaining waits
     bool fail = false;
     for (int ph = 0; ph < 2 && !fail; ++ph) {
@@ -1675,13 +1670,18 @@ __global__ void __launch_bounds__(256, 2) tc_planes_layer_kernel(const LArgs a) 
         float y[MR];
 #pragma unroll
         for (int jr = 0; jr < MR; ++jr) y[jr] = 0.0f;
-        // the segment's accumulator, after its last stage
+        // the segment's accumulators, after its last stage: issuer mi wrote
+        // one iff the segment has a stage of its parity
+        const int ns = (sg.nk + kQChunks - 1) / kQChunks;
+        const bool had[2] = {ns >= 2 || (st_i & 1) == 0, ns >= 2 || (st_i & 1) == 1};
+        st_i += ns;
         {
           const int buf = u & 1;
           if (!dead) dead = !__all_sync(0xffffffffu, mbar_wait(&accfull[buf], (u >> 1) & 1, abort_flag, err, 16));
           tc_fence_after();
-          uint32_t d[NT];
-          tmem_ld16(tmem + lane_addr + buf * C::kAccBuf, d);
+          uint32_t d0[NT], d1[NT];
+          tmem_ld16(tmem + lane_addr + buf * C::kAccBuf, d0);
+          tmem_ld16(tmem + lane_addr + buf * C::kAccBuf + NT, d1);
           // down: the segment's exponent per row, E = max E_c over its chunks
           // (the chunks are final: their planes fed these MMAs)
           int E[MR];
@@ -1697,9 +1697,10 @@ __global__ void __launch_bounds__(256, 2) tc_planes_layer_kernel(const LArgs a) 
           tmem_ld_wait();
           tc_fence_before();
           __syncwarp();
-          if (lane == 0) mbar_arrive(&accfree[buf]);  // the MMAs may reuse the accumulator
+          if (lane == 0) mbar_arrive(&accfree[buf]);  // the MMAs may reuse the accumulators
           ++u;
-          // fold the planes (p ascending): y[jr] = sum_p g_p * D[row, jr P + p]
+          // fold the planes (p ascending): y[jr] = sum_p g_p * D[row, jr P + p],
+          // D the sum of the two issuers' accumulators
 #pragma unroll
           for (int jr = 0; jr < MR; ++jr) {
             if (jr < a.m) {
@@ -1707,7 +1708,11 @@ __global__ void __launch_bounds__(256, 2) tc_planes_layer_kernel(const LArgs a) 
                 y[jr] = __int_as_float(0x7fc00000);  // a non-finite activation
               } else if (E[jr] != kSegZero) {
 #pragma unroll
-                for (int p = 0; p < P; ++p) y[jr] = fmaf(exp2i(E[jr] - 8 - (3 * p) / 2), __uint_as_float(d[jr * P + p]), y[jr]);
+                for (int p = 0; p < P; ++p) {
+                  const float dv = (had[0] ? __uint_as_float(d0[jr * P + p]) : 0.0f) +
+                                   (had[1] ? __uint_as_float(d1[jr * P + p]) : 0.0f);
+                  y[jr] = fmaf(exp2i(E[jr] - 8 - (3 * p) / 2), dv, y[jr]);
+                }
               }
             }
           }
@@ -1794,7 +1799,7 @@ __global__ void __launch_bounds__(256, 2) tc_planes_layer_kernel(const LArgs a) 
         }
         __threadfence();
         named_bar_sync(1, 128);
-        if (tid == 0) asm volatile("st.release.gpu.global.b32 [%0], %1;" ::"l"(a.ready + sg.tile), "r"(1) : "memory");
+        if (tid == 0) asm volatile("red.release.gpu.global.add.u32 [%0], 1;" ::"l"(a.gu_done) : "memory");
       }
     }
   }
@@ -2045,7 +2050,7 @@ cudaError_t launch_layer(LArgs a, int max_grid, int num_sms, cudaStream_t s) {
   const int grid = min(max_grid, occupancy * num_sms);
   if (grid < 1) return cudaErrorInvalidConfiguration;
   a.gu_parts = min(a.gu_parts, grid);
-  return launch_pdl(kern, dim3(grid), dim3(256), C::kSmemAlloc, s, a);
+  return launch_pdl(kern, dim3(grid), dim3(kLayerThreads), C::kSmemAlloc, s, a);
 }
 
 }  // namespace
@@ -2073,7 +2078,7 @@ PlanesPlan plan_planes(int64_t m, int64_t hidden, int64_t inter, int num_sms) {
   p.x_sf_bytes = (size_t)p.gu_kc * p.rows * 4;
   p.h_code_bytes = (size_t)p.rows * (size_t)(inter / 2);
   p.h_sf_bytes = (size_t)p.dn_kc * p.rows * 4;
-  p.zero_ints = p.gu_tiles + p.dn_tiles + p.gu_tiles;  // tile counters, h chunk ready flags
+  p.zero_ints = p.gu_tiles + p.dn_tiles + 1;  // tile counters, finished gate+up tiles
   p.other_ints = (int)m + p.gu_tiles * (int)m;          // x's row exponents, h's chunk exponents
   return p;
 }
@@ -2085,11 +2090,16 @@ cudaError_t launch_planes_ffn(const void* x, int64_t m, const TcWeight& gate_up,
   // 32-bit range arithmetic in the kernel
   if ((uint64_t)p.gu_tiles * p.gu_kc * p.grid >= (1ull << 32) || (uint64_t)p.dn_tiles * p.dn_kc * p.grid >= (1ull << 32))
     return cudaErrorInvalidValue;
-  int* zero = b.ints;  // [cnt_gu][cnt_dn][ready] zeroed, then x's E [m], h's E [gu_tiles][m]
+  int* zero = b.ints;  // [cnt_gu][cnt_dn][gu_done] zeroed, then x's E [m], h's E [gu_tiles][m]
   int* xe = zero + p.zero_ints;
   cudaError_t e;
   {
     ProfScope prof(s, "planes_prologue");
+    // the same shared-memory carveout as the layer kernel, so that SMs need
+    // no reconfiguration between the two
+    e = cudaFuncSetAttribute(planes_prologue_kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
+                             cudaSharedmemCarveoutMaxShared);
+    if (e != cudaSuccess) return e;
     const dim3 grid((unsigned)m, (unsigned)((hidden / 16 + kPlaneThreads / 8 - 1) / (kPlaneThreads / 8)));
     e = launch_pdl(planes_prologue_kernel, grid, dim3(kPlaneThreads), 0, s, static_cast<const uint16_t*>(x),
                    (int)m, (int)hidden, static_cast<uint8_t*>(b.xq), static_cast<uint8_t*>(b.xs), xe, zero,
@@ -2112,7 +2122,7 @@ cudaError_t launch_planes_ffn(const void* x, int64_t m, const TcWeight& gate_up,
   a.part_dn = static_cast<float*>(b.part_dn);
   a.cnt_gu = zero;
   a.cnt_dn = zero + p.gu_tiles;
-  a.ready = a.cnt_dn + p.dn_tiles;
+  a.gu_done = reinterpret_cast<uint32_t*>(a.cnt_dn + p.dn_tiles);
   a.m = (int)m;
   a.hidden = (int)hidden;
   a.inter = (int)inter;
