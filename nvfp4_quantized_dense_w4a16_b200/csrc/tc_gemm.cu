@@ -36,6 +36,9 @@
 #include <mutex>
 #include <utility>
 
+#include <cuda_fp4.h>
+#include <cuda_fp16.h>
+
 #include "common.cuh"
 #include "internal.h"
 #include "launch.cuh"
@@ -992,10 +995,13 @@ struct W4Cfg {
   static constexpr int kSmemBar = kSmemEpi + (kSmemEpi >= 16384 ? 0 : 16384);
   static constexpr int kSmemBytes = kSmemBar + (2 * kStages + 1) * 8 + 16;
   static constexpr int kSmemAlloc = kSmemBytes + 1024;
-  static constexpr int kSfaCol = XT * kW4BN;                             // TMEM columns
-  static constexpr int kSfbCol = kSfaCol + 4 * kW4Chunks * kStages;     // + 4 * kW4Chunks * kStages per tile
+  // TMEM columns: XT accumulators, then per activation tile (one MMA-issuing
+  // warp each) its own copy of the weight scales, then its activation scales
+  static constexpr int kSlotCols = 4 * kW4Chunks * kStages;
+  static constexpr int kSfaCol = XT * kW4BN;
+  static constexpr int kSfbCol = kSfaCol + XT * kSlotCols;
   static constexpr int kTmemCols = 512;
-  static_assert(kSfbCol + XT * 4 * kW4Chunks * kStages <= kTmemCols, "TMEM budget");
+  static_assert(kSfbCol + XT * kSlotCols <= kTmemCols, "TMEM budget");
   static_assert(kStageBytes % 1024 == 0, "stage alignment");
   static_assert(kSmemAlloc <= 232448, "shared memory budget");
   static_assert(kSmemEpi >= 2 * 16384, "the two epilogue buffers alias the rings");
@@ -1034,9 +1040,9 @@ tc_w4a4_kernel(const __grid_constant__ CUtensorMap xmap, const W4Args w4) {
   if (threadIdx.x == 0) {
     for (int s = 0; s < S; ++s) {
       mbar_init(&full[s], 1);
-      mbar_init(&empty[s], 1);
+      mbar_init(&empty[s], nxt);  // one commit per MMA-issuing warp
     }
-    mbar_init(accum, 1);
+    mbar_init(accum, nxt);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -1088,41 +1094,34 @@ tc_w4a4_kernel(const __grid_constant__ CUtensorMap xmap, const W4Args w4) {
       }
       for (int i = max(0, issued - S); i < issued; ++i) wait_drain(&full[i % S], (i / S) & 1);
     }
-  } else if (warp == 1) {
-    if (lane == 0) {
-      const uint32_t idesc = idesc_mxf4nvf4(kTileRows, kW4BN);
-      for (int i = 0; i < nstage; ++i) {
-        const int s = i % S;
-        const int nch = min(kW4Chunks, nk - kW4Chunks * i);
-        if (!mbar_wait(&full[s], (i / S) & 1, abort_flag, err, 2)) break;
-        tc_fence_after();
-        const uint8_t* st = smem + s * C::kStageBytes;
-        // the stage's scale copies first, then its MMAs (each MMA then finds
-        // its scales in TMEM without waiting for a copy issued just before)
-        for (int c = 0; c < nch; ++c) {
-          const uint32_t slot = 4 * (s * kW4Chunks + c);
-          const uint8_t* wc = st + c * kChunkBytes;
-          tmem_cp_32x128b_x4(tmem + C::kSfaCol + slot, smem_desc_interleave(smem_u32(wc + 4096), 16, 128));
-          for (int t = 0; t < nxt; ++t) {
-            const uint8_t* xt = st + C::kWBytes + t * (C::kXBytes + C::kSfbBytes);
-            tmem_cp_32x128b_x4(tmem + C::kSfbCol + t * 4 * kW4Chunks * S + slot,
-                               smem_desc_interleave(smem_u32(xt + C::kXBytes + 512 * c), 16, 128));
-          }
-        }
-        for (int c = 0; c < nch; ++c) {
-          const uint32_t slot = 4 * (s * kW4Chunks + c);
-          const uint64_t a_desc = smem_desc_interleave(smem_u32(st + c * kChunkBytes), 2048, 128);
-          for (int t = 0; t < nxt; ++t) {
-            const uint8_t* xt = st + C::kWBytes + t * (C::kXBytes + C::kSfbBytes);
-            mma_mxf4nvf4(tmem + t * kW4BN, a_desc, smem_desc_sw128(smem_u32(xt)) + 2 * c, idesc,
-                         tmem + C::kSfaCol + slot, tmem + C::kSfbCol + t * 4 * kW4Chunks * S + slot,
-                         (i | c) != 0 ? 1u : 0u);
-          }
-        }
-        mma_commit(&empty[s]);
+  } else if ((warp == 1 || warp == 3) && lane == 0 && (warp == 1 ? 0 : 1) < nxt) {
+    // MMA issuers: warp 1 for activation tile 0, warp 3 for tile 1 (two
+    // tcgen05 instruction streams; one thread's issue rate is the limit),
+    // each with its own copy of the weight scales
+    const int t = warp == 1 ? 0 : 1;
+    const uint32_t idesc = idesc_mxf4nvf4(kTileRows, kW4BN);
+    const uint32_t sfa0 = tmem + C::kSfaCol + t * C::kSlotCols, sfb0 = tmem + C::kSfbCol + t * C::kSlotCols;
+    for (int i = 0; i < nstage; ++i) {
+      const int s = i % S;
+      const int nch = min(kW4Chunks, nk - kW4Chunks * i);
+      if (!mbar_wait(&full[s], (i / S) & 1, abort_flag, err, 2)) break;
+      tc_fence_after();
+      const uint8_t* st = smem + s * C::kStageBytes;
+      const uint8_t* xt = st + C::kWBytes + t * (C::kXBytes + C::kSfbBytes);
+      // the stage's scale copies first, then its MMAs
+      for (int c = 0; c < nch; ++c) {
+        const uint32_t slot = 4 * (s * kW4Chunks + c);
+        tmem_cp_32x128b_x4(sfa0 + slot, smem_desc_interleave(smem_u32(st + c * kChunkBytes + 4096), 16, 128));
+        tmem_cp_32x128b_x4(sfb0 + slot, smem_desc_interleave(smem_u32(xt + C::kXBytes + 512 * c), 16, 128));
       }
-      mma_commit(accum);
+      for (int c = 0; c < nch; ++c) {
+        const uint32_t slot = 4 * (s * kW4Chunks + c);
+        mma_mxf4nvf4(tmem + t * kW4BN, smem_desc_interleave(smem_u32(st + c * kChunkBytes), 2048, 128),
+                     smem_desc_sw128(smem_u32(xt)) + 2 * c, idesc, sfa0 + slot, sfb0 + slot, (i | c) != 0 ? 1u : 0u);
+      }
+      mma_commit(&empty[s]);
     }
+    mma_commit(accum);
   }
   // epilogue on all eight warps once the last MMA is done: warpgroup g takes
   // every other 32-row chunk of each activation tile (warp w reads TMEM
@@ -1183,8 +1182,9 @@ tc_w4a4_kernel(const __grid_constant__ CUtensorMap xmap, const W4Args w4) {
 //  * down: equal ranges of its (tile, chunk) space, started once every
 //    gate+up tile is counted (one word, polled by one thread per CTA with a
 //    back-off; no grid-wide barrier otherwise).  The copy warps re-base each
-//    chunk's power-of-two scale bytes onto the segment's largest exponent,
-//    so a segment keeps one accumulator; split-K partial sums as above.
+//    chunk's power-of-two scale bytes onto the row's largest chunk exponent
+//    (kept with an atomic maximum), so a segment keeps one accumulator;
+//    split-K partial sums as above.
 // Each CTA's weight stream runs through both projections without a break.
 // Every wait is bounded and raises a device error bit when it expires.
 // ---------------------------------------------------------------------------
@@ -1241,33 +1241,58 @@ __device__ __forceinline__ int row_exponent(uint32_t max_bits) {
 // The P planes of one 16-element block, by the eight lanes part = 0..7 of an
 // aligned group of eight (two elements each; every lane of the warp calls).
 // Writes byte 8 b + part of plane row j P + p (rows of row_bytes) and, from
-// part 0, the block's scale byte at [b / 4][rows][4] + b % 4.
+// part 0, the block's scale byte at [b / 4][rows][4] + b % 4.  The planes
+// are a sequential chain, so the chain is kept short: the block maximum of
+// |r| is taken on the fp32 bit patterns (they order like the values), and
+// the scale exponent e = ceil(log2(amax / 6)) - log2 g_p comes from the bits
+// of amax (the same e as scaling amax by 1 / g_p first, for normal amax).
 __device__ __forceinline__ void block_planes(float r0, float r1, int E, bool valid, int part, int j, int b,
                                              uint8_t* codes, size_t row_bytes, uint8_t* sf, int rows) {
-#pragma unroll 1
+  uint32_t bytes[kQPlanes], s8s[kQPlanes];
+#pragma unroll
   for (int p = 0; p < kQPlanes; ++p) {
-    float amax = fmaxf(fabsf(r0), fabsf(r1));
-    amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
-    amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
-    amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 4));
+    uint32_t am = max(__float_as_uint(r0) & 0x7fffffffu, __float_as_uint(r1) & 0x7fffffffu);
+    am = max(am, __shfl_xor_sync(0xffffffffu, am, 1));
+    am = max(am, __shfl_xor_sync(0xffffffffu, am, 2));
+    am = max(am, __shfl_xor_sync(0xffffffffu, am, 4));
     uint32_t s8 = 0, byte = 0;
-    if (amax > 0.0f) {
+    if (am != 0) {
       const int ge = E - 8 - (3 * p) / 2;  // log2 g_p
       // smallest power of two 2^e >= amax / 6 / g_p, clamped to E4M3's 2^-9..2^8
-      int e = ceil_log2_over_6(amax * exp2i(-ge));
+      int e;
+      if (am >= 0x00800000u) {  // normal: amax = 1.f * 2^k
+        const int k = (int)(am >> 23) - 127;
+        e = ((am & 0x7fffffu) <= 0x400000u ? k - 2 : k - 1) - ge;
+      } else {
+        e = ceil_log2_over_6(__uint_as_float(am) * exp2i(-ge));
+      }
       e = e < -9 ? -9 : (e > 8 ? 8 : e);
       s8 = e >= -6 ? (uint32_t)(e + 7) << 3 : (1u << (e + 9));
-      // r / (g_p 2^e) and the represented values are exact power-of-two scalings
-      const float down = exp2i(-(ge + e)), up = exp2i(ge + e);
-      const uint32_t q0 = e2m1_encode(r0 * down), q1 = e2m1_encode(r1 * down);
-      r0 -= ((q0 & 8u) ? -e2m1_mag(q0 & 7u) : e2m1_mag(q0 & 7u)) * up;
-      r1 -= ((q1 & 8u) ? -e2m1_mag(q1 & 7u) : e2m1_mag(q1 & 7u)) * up;
-      byte = q0 | (q1 << 4);
+      // r / (g_p 2^e) and the represented values are exact power-of-two
+      // scalings; the hardware conversion rounds to the nearest E2M1 value,
+      // ties to the even code, saturating at 6 (the same codes as
+      // e2m1_encode), and the code's value v gives the new residual
+      // (q - v) * g_p 2^e exactly (q and v are within a factor two)
+      const int sh = ge + e;
+      const float down = exp2i(-sh), up = exp2i(sh);
+      const float q0 = r0 * down, q1 = r1 * down;
+      byte = (uint32_t)__nv_cvt_float2_to_fp4x2(make_float2(q0, q1), __NV_E2M1, cudaRoundNearest);
+      const __half2_raw hv = __nv_cvt_fp4x2_to_halfraw2((__nv_fp4x2_storage_t)byte, __NV_E2M1);
+      __half_raw h0, h1;
+      h0.x = hv.x;
+      h1.x = hv.y;
+      r0 = (q0 - __half2float(__half(h0))) * up;
+      r1 = (q1 - __half2float(__half(h1))) * up;
     }
-    if (valid) {
+    bytes[p] = byte;
+    s8s[p] = s8;
+  }
+  if (valid) {
+#pragma unroll
+    for (int p = 0; p < kQPlanes; ++p) {
       const int rowp = j * kQPlanes + p;
-      codes[(size_t)rowp * row_bytes + 8 * b + part] = (uint8_t)byte;
-      if (part == 0) sf[((size_t)(b >> 2) * rows + rowp) * 4 + (b & 3)] = (uint8_t)s8;
+      codes[(size_t)rowp * row_bytes + 8 * b + part] = (uint8_t)bytes[p];
+      if (part == 0) sf[((size_t)(b >> 2) * rows + rowp) * 4 + (b & 3)] = (uint8_t)s8s[p];
     }
   }
 }
@@ -1346,6 +1371,7 @@ struct LArgs {
   int* cnt_gu;           // [gu_tiles] chunks done, zero on entry
   int* cnt_dn;           // [dn_tiles]
   uint32_t* gu_done;     // gate+up tiles whose h planes are written, zero on entry
+  int* he_max;           // [m] largest chunk exponent of h per row, + 1001 (0: none yet), zero on entry
   int m, hidden, inter, gu_tiles, gu_kc, gu_parts, dn_tiles, dn_kc;
 };
 
@@ -1389,6 +1415,12 @@ __device__ __forceinline__ bool wait_count(const uint32_t* ctr, uint32_t target,
     }
     __nanosleep(256);
   }
+}
+
+// Row exponent of h: the largest chunk exponent (stored + 1001; 0 = none).
+__device__ __forceinline__ int he_row(const int* he_max, int jr) {
+  const int v = __ldcg(he_max + jr);
+  return v == 0 ? kSegZero : v - 1001;
 }
 
 // Sum of the split-K partial slots of tile t (CTAs g0..g1 of `parts` that
@@ -1532,8 +1564,8 @@ __global__ void __launch_bounds__(kLayerThreads, 2) tc_planes_layer_kernel(const
     // fills the even stages, warp 3 the odd ones, each with all of a
     // stage's loads in flight at once.  Down: once every h chunk of this
     // CTA's range is final, each chunk's scale bytes are re-based from its
-    // own exponent E_c to the segment's E = max E_c (2^-(E - E_c) times,
-    // exact while the scale stays >= 2^-9; a smaller one is flushed to 0)
+    // own exponent E_c to the row's E = max E_c (2^-(E - E_c) times, exact
+    // while the scale stays >= 2^-9; a smaller one is flushed to 0)
     constexpr int kMaxU = NT * 8 / 32;         // 16-byte code units per lane
     constexpr int kMaxW = NT * kQChunks / 32;  // scale words per lane
     const int pt = threadIdx.x - 64;
@@ -1562,16 +1594,9 @@ __global__ void __launch_bounds__(kLayerThreads, 2) tc_planes_layer_kernel(const
         if (!*sh_ready) ok = false;
       }
       for (int j = 0; ok && q_segment(a, ph, j, sg); ++j) {
-        int eseg[MR];  // down: the segment's exponent per row
+        int eseg[MR];  // down: the row's exponent, E = max E_c over all chunks of h
 #pragma unroll
-        for (int jr = 0; jr < MR; ++jr) {
-          int e = kSegZero;
-          if (ph == 1 && jr < a.m)
-            for (int i = lane; i < sg.nk; i += 32) e = max(e, __ldcg(a.he + (size_t)(sg.c0 + i) * a.m + jr));
-#pragma unroll
-          for (int o = 16; o > 0; o >>= 1) e = max(e, __shfl_xor_sync(0xffffffffu, e, o));
-          eseg[jr] = e;
-        }
+        for (int jr = 0; jr < MR; ++jr) eseg[jr] = ph == 1 && jr < a.m ? he_row(a.he_max, jr) : kSegZero;
         for (int c = 0; c < sg.nk; c += kQChunks, ++st_i) {
           if ((st_i & 1) != mine) continue;
           const int s = st_i % S, nch = min(kQChunks, sg.nk - c);
@@ -1682,18 +1707,11 @@ __global__ void __launch_bounds__(kLayerThreads, 2) tc_planes_layer_kernel(const
           uint32_t d0[NT], d1[NT];
           tmem_ld16(tmem + lane_addr + buf * C::kAccBuf, d0);
           tmem_ld16(tmem + lane_addr + buf * C::kAccBuf + NT, d1);
-          // down: the segment's exponent per row, E = max E_c over its chunks
-          // (the chunks are final: their planes fed these MMAs)
+          // down: the row's exponent, E = max E_c over all chunks of h (final:
+          // their planes fed these MMAs)
           int E[MR];
 #pragma unroll
-          for (int jr = 0; jr < MR; ++jr) {
-            int e = kSegZero;
-            if (ph == 1 && jr < a.m)
-              for (int i = lane; i < sg.nk; i += 32) e = max(e, __ldcg(a.he + (size_t)(sg.c0 + i) * a.m + jr));
-#pragma unroll
-            for (int o = 16; o > 0; o >>= 1) e = max(e, __shfl_xor_sync(0xffffffffu, e, o));
-            E[jr] = ph ? e : xe[jr];
-          }
+          for (int jr = 0; jr < MR; ++jr) E[jr] = ph ? (jr < a.m ? he_row(a.he_max, jr) : kSegZero) : xe[jr];
           tmem_ld_wait();
           tc_fence_before();
           __syncwarp();
@@ -1795,7 +1813,10 @@ __global__ void __launch_bounds__(kLayerThreads, 2) tc_planes_layer_kernel(const
           if (E == kSegNonFinite) hv[0] = hv[1] = 0.0f;
           const int b = 4 * sg.tile + (lane >> 3);
           block_planes(hv[0], hv[1], E, b < a.inter / 16, lane & 7, jr, b, a.hq, (size_t)a.inter / 2, a.hs, rows);
-          if (lane == 0) a.he[(size_t)sg.tile * a.m + jr] = E;
+          if (lane == 0) {
+            a.he[(size_t)sg.tile * a.m + jr] = E;
+            atomicMax(a.he_max + jr, E + 1001);
+          }
         }
         __threadfence();
         named_bar_sync(1, 128);
@@ -2078,7 +2099,7 @@ PlanesPlan plan_planes(int64_t m, int64_t hidden, int64_t inter, int num_sms) {
   p.x_sf_bytes = (size_t)p.gu_kc * p.rows * 4;
   p.h_code_bytes = (size_t)p.rows * (size_t)(inter / 2);
   p.h_sf_bytes = (size_t)p.dn_kc * p.rows * 4;
-  p.zero_ints = p.gu_tiles + p.dn_tiles + 1;  // tile counters, finished gate+up tiles
+  p.zero_ints = p.gu_tiles + p.dn_tiles + 1 + (int)m;  // tile counters, finished gate+up tiles, h row exponents
   p.other_ints = (int)m + p.gu_tiles * (int)m;          // x's row exponents, h's chunk exponents
   return p;
 }
@@ -2090,7 +2111,7 @@ cudaError_t launch_planes_ffn(const void* x, int64_t m, const TcWeight& gate_up,
   // 32-bit range arithmetic in the kernel
   if ((uint64_t)p.gu_tiles * p.gu_kc * p.grid >= (1ull << 32) || (uint64_t)p.dn_tiles * p.dn_kc * p.grid >= (1ull << 32))
     return cudaErrorInvalidValue;
-  int* zero = b.ints;  // [cnt_gu][cnt_dn][gu_done] zeroed, then x's E [m], h's E [gu_tiles][m]
+  int* zero = b.ints;  // [cnt_gu][cnt_dn][gu_done][he_max m] zeroed, then x's E [m], h's E [gu_tiles][m]
   int* xe = zero + p.zero_ints;
   cudaError_t e;
   {
@@ -2123,6 +2144,7 @@ cudaError_t launch_planes_ffn(const void* x, int64_t m, const TcWeight& gate_up,
   a.cnt_gu = zero;
   a.cnt_dn = zero + p.gu_tiles;
   a.gu_done = reinterpret_cast<uint32_t*>(a.cnt_dn + p.dn_tiles);
+  a.he_max = a.cnt_dn + p.dn_tiles + 1;
   a.m = (int)m;
   a.hidden = (int)hidden;
   a.inter = (int)inter;
