@@ -285,17 +285,22 @@ typedef enum ffn_kernel_family {
                                 kernels, one CTA per SM, gate+up over whole tiles,
                                 down over equal K ranges reduced in-kernel
                                 (only with FFN_NVFP4_W4A16_PATH=persistent)     */
-  FFN_KERNEL_TC_PLANES = 6   /* FFN layer for m <= 8 with bf16 activations when
-                                both handles hold the natural tiled layout
-                                (built for the fixed format too, e.g.
-                                FFN_FORMAT_ALL): the NVFP4 weights go to the
-                                block-scaled FP4 MMA as stored and each
-                                activation row as 8 NVFP4 residual planes
-                                (N = 8m columns, at least 16; exact for bf16
-                                rows of normal spread); equal K ranges per CTA, two
-                                CTAs per SM, split-K sums added in-kernel.
-                                tile_rows reports the MMA's N.  Without the
-                                natural layout the layer takes FFN_KERNEL_TC_W4A16. */
+  FFN_KERNEL_TC_PLANES = 6   /* FFN layer for m <= 2 with bf16 activations and
+                                no LoRA adapter, when both handles hold the
+                                natural tiled layout (built for the fixed format
+                                too, e.g. FFN_FORMAT_ALL): the NVFP4 weights go
+                                to the block-scaled FP4 MMA as stored and each
+                                activation row as 8 NVFP4 residual planes (N = 16
+                                columns; exact for bf16 rows of normal spread).
+                                Two launches: a small prologue (x's planes,
+                                counters) and one persistent kernel, two CTAs
+                                per SM, all resident, for both projections
+                                (gate+up whole tiles, or equal K ranges when the
+                                tiles outnumber the CTAs; down equal K ranges;
+                                split-K sums added in-kernel in K order).
+                                tile_rows reports the MMA's N, grid the CTAs of
+                                the persistent kernel.  Without the natural
+                                layout the layer takes FFN_KERNEL_TC_W4A16.   */
 } ffn_kernel_family;
 
 typedef enum ffn_projection_role {
@@ -331,8 +336,10 @@ ffn_status ffn_nvfp4_tensor_peak(int kind, int issuers, int iters, double* tflop
 /* Device-side error bits.  Kernels that wait on asynchronous copies or on
  * tensor-core completion give up after about two seconds instead of hanging,
  * free their tensor memory, skip their stores and OR a bit into a device-wide
- * error word (1: producer, 2: MMA issuer, 4: dequant, 8: epilogue, 16: drain
- * timeout).  Synchronises the device, writes the word to *flags and, if
+ * error word (1: producer, 2: MMA issuer, 4: dequant or operand copy, 8:
+ * epilogue, 16: drain or accumulator wait, 32: a wait for work of other CTAs
+ * of the same launch, e.g. when they cannot all be resident because other
+ * work holds the SMs).  Synchronises the device, writes the word to *flags and, if
  * clear != 0, resets it to zero.  0 means every kernel completed normally. */
 ffn_status ffn_nvfp4_device_error(int* flags, int clear);
 

@@ -1424,13 +1424,23 @@ __device__ __forceinline__ int he_row(const int* he_max, int jr) {
 }
 
 // Sum of the split-K partial slots of tile t (CTAs g0..g1 of `parts` that
-// own a non-empty share of it), in K order.
+// own a non-empty share of it), in K order; the loads of eight slots at a
+// time are in flight together (one L2 round trip instead of eight).
 __device__ __forceinline__ float sum_partials(const float* part, int m, int jr, int rr, int t, uint32_t W, int parts,
                                               int g0, int g1) {
   float sum = 0.0f;
-  for (int gg = g0; gg <= g1; ++gg)
-    if (W * (uint32_t)gg / parts != W * (uint32_t)(gg + 1) / parts)
-      sum += __ldcg(part + ((size_t)(gg + t) * m + jr) * kTileRows + rr);
+  for (int g = g0; g <= g1; g += 8) {
+    float v[8];
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      const int gg = g + k;
+      v[k] = gg <= g1 && W * (uint32_t)gg / parts != W * (uint32_t)(gg + 1) / parts
+                 ? __ldcg(part + ((size_t)(gg + t) * m + jr) * kTileRows + rr)
+                 : 0.0f;
+    }
+#pragma unroll
+    for (int k = 0; k < 8; ++k) sum += v[k];  // (+0 for an empty share: the sum never is -0)
+  }
   return sum;
 }
 
@@ -1751,10 +1761,14 @@ __global__ void __launch_bounds__(kLayerThreads, 2) tc_planes_layer_kernel(const
 #pragma unroll
           for (int jr = 0; jr < MR; ++jr)
             if (jr < a.m) Pp[(size_t)jr * kTileRows + row] = y[jr];
-          __threadfence();
+          // the barrier orders the four warps' stores before thread 0's fence
+          // and count (cumulative at GPU scope)
           named_bar_sync(1, 128);
           // the tile is complete when its counter reaches kc chunks
-          if (tid == 0) *last_flag = atomicAdd((ph ? a.cnt_dn : a.cnt_gu) + sg.tile, sg.nk) + sg.nk == kc ? 1 : 0;
+          if (tid == 0) {
+            __threadfence();
+            *last_flag = atomicAdd((ph ? a.cnt_dn : a.cnt_gu) + sg.tile, sg.nk) + sg.nk == kc ? 1 : 0;
+          }
           named_bar_sync(1, 128);
           have = *last_flag != 0;
           if (have) __threadfence();
@@ -1818,9 +1832,11 @@ __global__ void __launch_bounds__(kLayerThreads, 2) tc_planes_layer_kernel(const
             atomicMax(a.he_max + jr, E + 1001);
           }
         }
-        __threadfence();
-        named_bar_sync(1, 128);
-        if (tid == 0) asm volatile("red.release.gpu.global.add.u32 [%0], 1;" ::"l"(a.gu_done) : "memory");
+        named_bar_sync(1, 128);  // the planes are written (ordered before the release below)
+        if (tid == 0) {
+          __threadfence();
+          asm volatile("red.release.gpu.global.add.u32 [%0], 1;" ::"l"(a.gu_done) : "memory");
+        }
       }
     }
   }
