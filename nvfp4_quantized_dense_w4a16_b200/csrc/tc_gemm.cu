@@ -1238,24 +1238,27 @@ __device__ __forceinline__ int row_exponent(uint32_t max_bits) {
   return max_bits == 0 ? kSegZero : max_bits >= 0x7f80u ? kSegNonFinite : ilogbf(bf16_bits_to_float(max_bits));
 }
 
-// The P planes of one 16-element block, by the eight lanes part = 0..7 of an
-// aligned group of eight (two elements each; every lane of the warp calls).
-// Writes byte 8 b + part of plane row j P + p (rows of row_bytes) and, from
-// part 0, the block's scale byte at [b / 4][rows][4] + b % 4.  The planes
-// are a sequential chain, so the chain is kept short: the block maximum of
-// |r| is taken on the fp32 bit patterns (they order like the values), and
-// the scale exponent e = ceil(log2(amax / 6)) - log2 g_p comes from the bits
-// of amax (the same e as scaling amax by 1 / g_p first, for normal amax).
-__device__ __forceinline__ void block_planes(float r0, float r1, int E, bool valid, int part, int j, int b,
+// The P planes of one 16-element block, by the four lanes part = 0..3 of an
+// aligned group of four (four elements each, v[0..3] = elements 4 part ..;
+// every lane of the warp calls).  Writes bytes 8 b + 2 part, +1 of plane row
+// j P + p (rows of row_bytes) and, from part 0, the block's scale byte at
+// [b / 4][rows][4] + b % 4.  The planes are a sequential chain, so the chain
+// is kept short: the block maximum of |r| is taken on the fp32 bit patterns
+// (they order like the values), the scale exponent e = ceil(log2(amax / 6))
+// - log2 g_p comes from the bits of amax (the same e as scaling amax by 1 /
+// g_p first, for normal amax), and the E2M1 codes are encoded and decoded by
+// the hardware conversions (round to nearest, ties to the even code,
+// saturating at 6: the codes of e2m1_encode).
+__device__ __forceinline__ void block_planes(float (&v)[4], int E, bool valid, int part, int j, int b,
                                              uint8_t* codes, size_t row_bytes, uint8_t* sf, int rows) {
-  uint32_t bytes[kQPlanes], s8s[kQPlanes];
+  uint32_t pairs[kQPlanes], s8s[kQPlanes];
 #pragma unroll
   for (int p = 0; p < kQPlanes; ++p) {
-    uint32_t am = max(__float_as_uint(r0) & 0x7fffffffu, __float_as_uint(r1) & 0x7fffffffu);
+    uint32_t am = max(max(__float_as_uint(v[0]) & 0x7fffffffu, __float_as_uint(v[1]) & 0x7fffffffu),
+                      max(__float_as_uint(v[2]) & 0x7fffffffu, __float_as_uint(v[3]) & 0x7fffffffu));
     am = max(am, __shfl_xor_sync(0xffffffffu, am, 1));
     am = max(am, __shfl_xor_sync(0xffffffffu, am, 2));
-    am = max(am, __shfl_xor_sync(0xffffffffu, am, 4));
-    uint32_t s8 = 0, byte = 0;
+    uint32_t s8 = 0, pair = 0;
     if (am != 0) {
       const int ge = E - 8 - (3 * p) / 2;  // log2 g_p
       // smallest power of two 2^e >= amax / 6 / g_p, clamped to E4M3's 2^-9..2^8
@@ -1269,40 +1272,44 @@ __device__ __forceinline__ void block_planes(float r0, float r1, int E, bool val
       e = e < -9 ? -9 : (e > 8 ? 8 : e);
       s8 = e >= -6 ? (uint32_t)(e + 7) << 3 : (1u << (e + 9));
       // r / (g_p 2^e) and the represented values are exact power-of-two
-      // scalings; the hardware conversion rounds to the nearest E2M1 value,
-      // ties to the even code, saturating at 6 (the same codes as
-      // e2m1_encode), and the code's value v gives the new residual
-      // (q - v) * g_p 2^e exactly (q and v are within a factor two)
+      // scalings, and the new residual (q - value) g_p 2^e is exact (q and
+      // the value of its code are within a factor two)
       const int sh = ge + e;
       const float down = exp2i(-sh), up = exp2i(sh);
-      const float q0 = r0 * down, q1 = r1 * down;
-      byte = (uint32_t)__nv_cvt_float2_to_fp4x2(make_float2(q0, q1), __NV_E2M1, cudaRoundNearest);
-      const __half2_raw hv = __nv_cvt_fp4x2_to_halfraw2((__nv_fp4x2_storage_t)byte, __NV_E2M1);
-      __half_raw h0, h1;
-      h0.x = hv.x;
-      h1.x = hv.y;
-      r0 = (q0 - __half2float(__half(h0))) * up;
-      r1 = (q1 - __half2float(__half(h1))) * up;
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const float q0 = v[2 * h] * down, q1 = v[2 * h + 1] * down;
+        const uint32_t byte = (uint32_t)__nv_cvt_float2_to_fp4x2(make_float2(q0, q1), __NV_E2M1, cudaRoundNearest);
+        const __half2_raw hv = __nv_cvt_fp4x2_to_halfraw2((__nv_fp4x2_storage_t)byte, __NV_E2M1);
+        __half_raw h0, h1;
+        h0.x = hv.x;
+        h1.x = hv.y;
+        v[2 * h] = (q0 - __half2float(__half(h0))) * up;
+        v[2 * h + 1] = (q1 - __half2float(__half(h1))) * up;
+        pair |= byte << (8 * h);
+      }
     }
-    bytes[p] = byte;
+    pairs[p] = pair;
     s8s[p] = s8;
   }
   if (valid) {
 #pragma unroll
     for (int p = 0; p < kQPlanes; ++p) {
       const int rowp = j * kQPlanes + p;
-      codes[(size_t)rowp * row_bytes + 8 * b + part] = (uint8_t)bytes[p];
+      *reinterpret_cast<uint16_t*>(codes + (size_t)rowp * row_bytes + 8 * b + 2 * part) = (uint16_t)pairs[p];
       if (part == 0) sf[((size_t)(b >> 2) * rows + rowp) * 4 + (b & 3)] = (uint8_t)s8s[p];
     }
   }
 }
 
-// Prologue: grid (m, ceil(K / 16 / 16)), 128 threads; CTA (j, c) builds the
-// planes of blocks 16c .. 16c + 15 of row j after finding the row's maximum
-// (every CTA of the row finds the same E), CTA (j, 0) writes E[j], and the
-// CTAs zero the next kernel's counters.  It lets the next kernel launch at
-// once (that one waits for this one before reading anything it writes).
+// Prologue: grid (m, ceil(K / 16 / 32)), 128 threads; CTA (j, c) builds the
+// planes of blocks 32c .. 32c + 31 of row j (four threads per block) after
+// finding the row's maximum (every CTA of the row finds the same E), CTA
+// (j, 0) writes E[j], and the CTAs zero the next kernel's counters.  It lets
+// the next kernel launch at once (that one waits for this one before reading
+// anything it writes).
 constexpr int kPlaneThreads = 128;
+constexpr int kPlaneBlocksPerCta = kPlaneThreads / 4;
 __global__ void __launch_bounds__(kPlaneThreads) planes_prologue_kernel(const uint16_t* __restrict__ x, int m, int K,
                                                                         uint8_t* __restrict__ codes,
                                                                         uint8_t* __restrict__ sf, int* __restrict__ E_out,
@@ -1342,16 +1349,18 @@ __global__ void __launch_bounds__(kPlaneThreads) planes_prologue_kernel(const ui
   const int E = row_exponent(mx);
   if (blockIdx.y == 0 && threadIdx.x == 0) E_out[j] = E;
   const int nb = K / 16;
-  const int b = blockIdx.y * (kPlaneThreads / 8) + (threadIdx.x >> 3);
-  const int part = threadIdx.x & 7;  // elements 2 part, 2 part + 1 of the block
-  const bool valid = b < nb;         // whole groups of eight lanes share validity
-  float r0 = 0.0f, r1 = 0.0f;
+  const int b = blockIdx.y * kPlaneBlocksPerCta + (threadIdx.x >> 2);
+  const int part = threadIdx.x & 3;  // elements 4 part .. 4 part + 3 of the block
+  const bool valid = b < nb;         // whole groups of four lanes share validity
+  float v[4] = {0.0f, 0.0f, 0.0f, 0.0f};
   if (valid && E != kSegNonFinite) {
-    const uint32_t v = *reinterpret_cast<const uint32_t*>(row + 16 * b + 2 * part);
-    r0 = bf16_bits_to_float(v & 0xffffu);
-    r1 = bf16_bits_to_float(v >> 16);
+    const uint2 w = *reinterpret_cast<const uint2*>(row + 16 * b + 4 * part);
+    v[0] = bf16_bits_to_float(w.x & 0xffffu);
+    v[1] = bf16_bits_to_float(w.x >> 16);
+    v[2] = bf16_bits_to_float(w.y & 0xffffu);
+    v[3] = bf16_bits_to_float(w.y >> 16);
   }
-  block_planes(r0, r1, E, valid, part, j, b, codes, (size_t)K / 2, sf, m * kQPlanes);
+  block_planes(v, E, valid, part, j, b, codes, (size_t)K / 2, sf, m * kQPlanes);
 }
 
 struct LArgs {
@@ -1804,29 +1813,29 @@ __global__ void __launch_bounds__(kLayerThreads, 2) tc_planes_layer_kernel(const
           }
         }
         named_bar_sync(1, 128);
-        // warp q = activation row jr: lanes take h columns 64 t + 2 lane, +1,
-        // find the chunk's exponent and write its planes (eight lanes per
-        // 16-block)
+        // warp q = activation row jr: lanes 0..15 take h columns 64 t + 4 lane
+        // .. + 3, find the chunk's exponent and write its planes (four lanes
+        // per 16-block)
         if (q < a.m) {
           const int jr = q;
-          float hv[2];
+          float hv[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+          uint32_t mx = 0;
 #pragma unroll
-          for (int e = 0; e < 2; ++e) {
-            const int r = 2 * lane + e, n = 64 * sg.tile + r;
-            hv[e] = 0.0f;
-            if (n < a.inter) {
+          for (int e = 0; e < 4; ++e) {
+            const int r = 4 * lane + e, n = 64 * sg.tile + r;
+            if (lane < 16 && n < a.inter) {
               const float gv = bf16_round(a.gs_gu[0] * Y[jr * kTileRows + r]);
               const float uv = bf16_round(a.gs_gu[1] * Y[jr * kTileRows + 64 + r]);
               hv[e] = bf16_round(silu_fast(gv) * uv);
+              mx = max(mx, (uint32_t)(f32_to_bf16_bits(hv[e]) & 0x7fffu));
             }
           }
-          uint32_t mx = max(f32_to_bf16_bits(hv[0]) & 0x7fffu, f32_to_bf16_bits(hv[1]) & 0x7fffu);
 #pragma unroll
           for (int o = 16; o > 0; o >>= 1) mx = max(mx, __shfl_xor_sync(0xffffffffu, mx, o));
           const int E = row_exponent(mx);
-          if (E == kSegNonFinite) hv[0] = hv[1] = 0.0f;
-          const int b = 4 * sg.tile + (lane >> 3);
-          block_planes(hv[0], hv[1], E, b < a.inter / 16, lane & 7, jr, b, a.hq, (size_t)a.inter / 2, a.hs, rows);
+          if (E == kSegNonFinite) hv[0] = hv[1] = hv[2] = hv[3] = 0.0f;
+          const int b = 4 * sg.tile + (lane >> 2);
+          block_planes(hv, E, lane < 16 && b < a.inter / 16, lane & 3, jr, b, a.hq, (size_t)a.inter / 2, a.hs, rows);
           if (lane == 0) {
             a.he[(size_t)sg.tile * a.m + jr] = E;
             atomicMax(a.he_max + jr, E + 1001);
@@ -2137,7 +2146,7 @@ cudaError_t launch_planes_ffn(const void* x, int64_t m, const TcWeight& gate_up,
     e = cudaFuncSetAttribute(planes_prologue_kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
                              cudaSharedmemCarveoutMaxShared);
     if (e != cudaSuccess) return e;
-    const dim3 grid((unsigned)m, (unsigned)((hidden / 16 + kPlaneThreads / 8 - 1) / (kPlaneThreads / 8)));
+    const dim3 grid((unsigned)m, (unsigned)((hidden / 16 + kPlaneBlocksPerCta - 1) / kPlaneBlocksPerCta));
     e = launch_pdl(planes_prologue_kernel, grid, dim3(kPlaneThreads), 0, s, static_cast<const uint16_t*>(x),
                    (int)m, (int)hidden, static_cast<uint8_t*>(b.xq), static_cast<uint8_t*>(b.xs), xe, zero,
                    p.zero_ints);
