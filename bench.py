@@ -116,9 +116,10 @@ def nvfp4_bytes(n, k):
 KERNEL_SOURCES = ("csrc/tc_gemm.cu", "csrc/sm100.cuh", "csrc/common.cuh", "csrc/internal.h")
 TRAFFIC = {
     ("tc_w4a16_gate_up_silu", "prefill"): {
-        "bytes": 146800896 + 128328960, "sources_sha1": "5976b4c07ea6be5b9cb88fe0ad51fe53f300e557"},
+        "bytes": 150174208 + 129634304, "sources_sha1": "767b750504cffff3284802b29f16c399e7ee659a"},
+    ("tc_planes_layer", "decode"): {
+        "bytes": 150531072 + 4223744, "sources_sha1": "767b750504cffff3284802b29f16c399e7ee659a"},
 }
-
 
 def normalised_source(text):
     """Source text without comments and whitespace (edits to either do not
@@ -283,8 +284,13 @@ def roofline(wl, prof, peaks, peak_src, workload):
     average launch duration, against the peak of the bound it is under."""
     if not prof:
         return None
-    kname, (launches, kms) = max(prof.items(), key=lambda kv: kv[1][1])
+    # the longest kernel whose algorithmic units are known
+    ranked = sorted(prof.items(), key=lambda kv: -kv[1][1])
+    known = [kv for kv in ranked if wl.kernel_units(kv[0], peaks)[1] is not None]
+    kname, (launches, kms) = (known or ranked)[0]
     bound, units = wl.kernel_units(kname, peaks)
+    if units is None:
+        return None
     avg_s = kms / launches * 1e-3
     if bound == "tensor":
         peak, what = tensor_peak(peaks, wl.fmt)
