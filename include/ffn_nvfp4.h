@@ -290,8 +290,11 @@ typedef enum ffn_kernel_family {
                                 natural tiled layout (built for the fixed format
                                 too, e.g. FFN_FORMAT_ALL): the NVFP4 weights go
                                 to the block-scaled FP4 MMA as stored and each
-                                activation row as 8 NVFP4 residual planes (N = 16
-                                columns; exact for bf16 rows of normal spread).
+                                activation row as 8 NVFP4 planes (N = 16 columns):
+                                2-bit digits of a 16-bit window below each
+                                16-block's top bit, exact when the block's
+                                elements lie within 2^8 of its largest (else
+                                truncated below 2^-15 of the block maximum).
                                 Two launches: a small prologue (x's planes,
                                 counters) and one persistent kernel, two CTAs
                                 per SM, all resident, for both projections

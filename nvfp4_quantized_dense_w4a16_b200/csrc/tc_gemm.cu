@@ -36,9 +36,6 @@
 #include <mutex>
 #include <utility>
 
-#include <cuda_fp4.h>
-#include <cuda_fp16.h>
-
 #include "common.cuh"
 #include "internal.h"
 #include "launch.cuh"
@@ -1150,23 +1147,21 @@ tc_w4a4_kernel(const __grid_constant__ CUtensorMap xmap, const W4Args w4) {
 // The NVFP4 weights go to tcgen05 kind::mxf4nvf4 as stored (natural tiled
 // chunks: the codes are the A operand, the chunk's 512-byte scale block is
 // SFA) -- no software dequantisation.  Each bf16 activation row becomes the B
-// operand as P = 8 NVFP4 "planes", x = sum_p g_p * (s_p,b * q_p,k) + r_P,
-// each plane one MMA column (N = 8m, at least 16):
-//  * g_p = 2^(E - 8 - floor(3p / 2)), E = floor(log2 max|x|) of the row (a
-//    per-row power-of-two factor that keeps every block scale of the plane
-//    within E4M3's powers of two 2^-9..2^8; applied in the epilogue);
-//  * per 16-block a power-of-two scale s = 2^ceil(log2(amax / 6 / g_p)) of
-//    the residual r left by planes 0..p-1 (exact in E4M3, and r then scales
-//    exactly), codes q = E2M1(r / (g_p * s)), and r -= g_p * s * q (exact:
-//    the represented value has at most two significant bits and lies within a
-//    factor two of r).
-// Each plane removes at least a factor 3 from every block's residual while
-// g_p's range drops by 2^1.5 per plane, so no block outgrows its plane; a
-// plane takes the next two to three bits near each block's maximum, and 8
-// planes represent seeded bf16 rows (normal, outlier-channel, cubed-normal)
-// exactly or to ~1e-9 of the row maximum; small integers need the first
-// plane only.  The epilogue folds the planes back, y[j] = sum_p g_p * D_j,p,
-// so the result is the fp32-accumulated product of the exact bf16 rows.
+// operand as P = 8 NVFP4 "planes", each one MMA column (N = 8m, at least 16):
+// a 16-bit window of every 16-block's values, starting at the block's top
+// bit, cut into 2-bit digits.  With E = floor(log2 max|x|) of the row and T
+// the largest exponent in the block, an element x = M * 2^(e - 7) (M its
+// 8-bit significand) is the integer A = M * 2^(e - T + 8) < 2^16 in units of
+// 2^(T - 15), and plane p holds its digit d_p = (A >> (14 - 2p)) & 3 with the
+// element's sign: E2M1 values 0, 1, 2, 3 (exact), block scale s = 2^(T - E +
+// 8) (a power of two within E4M3's 2^-9..2^8 for T >= E - 17; smaller blocks
+// are flushed), plane factor g_p = 2^(E - 2p - 9) applied in the epilogue,
+// so that d_p * s * g_p = d_p * 2^(T - 2p - 1) and sum_p = A * 2^(T - 15) = x.
+// Exact when every element of a block lies within 2^8 of the block's largest
+// (the window holds all 8 significant bits); a smaller element loses the
+// bits below 2^(T - 15) (truncation).  The digits of the 8 planes are
+// independent of each other: no chain of residuals.  The epilogue folds the
+// planes back, y[j] = sum_p g_p * D_j,p.
 //
 // One layer is two launches.  A small prologue kernel builds x's planes
 // with one exponent per row (codes [m P][H/2], scale bytes [H/64][m P][4],
@@ -1223,81 +1218,58 @@ __device__ __forceinline__ float exp2i(int k) {
   return k >= -126 && k <= 127 ? __int_as_float((k + 127) << 23) : ldexpf(1.0f, k);
 }
 
-// Smallest e with 6 * 2^e >= a, for a > 0 normal: with a in [2^k, 2^(k+1)),
-// e = k - 2 when a <= 1.5 * 2^k (6 * 2^(k-2) = 1.5 * 2^k), else k - 1
-// (3 * 2^k > a); e = k - 3 never suffices (0.75 * 2^k < a).  Integer work on
-// the bits of a, no division.
-__device__ __forceinline__ int ceil_log2_over_6(float a) {
-  const uint32_t bits = __float_as_uint(a);
-  const int k = (int)((bits >> 23) & 0xffu) - 127;
-  return (bits & 0x7fffffu) <= 0x400000u ? k - 2 : k - 1;
-}
-
 // Row exponent from the largest |bf16| bit pattern of the row.
 __device__ __forceinline__ int row_exponent(uint32_t max_bits) {
   return max_bits == 0 ? kSegZero : max_bits >= 0x7f80u ? kSegNonFinite : ilogbf(bf16_bits_to_float(max_bits));
 }
 
-// The P planes of one 16-element block, by the four lanes part = 0..3 of an
-// aligned group of four (four elements each, v[0..3] = elements 4 part ..;
-// every lane of the warp calls).  Writes bytes 8 b + 2 part, +1 of plane row
-// j P + p (rows of row_bytes) and, from part 0, the block's scale byte at
-// [b / 4][rows][4] + b % 4.  The planes are a sequential chain, so the chain
-// is kept short: the block maximum of |r| is taken on the fp32 bit patterns
-// (they order like the values), the scale exponent e = ceil(log2(amax / 6))
-// - log2 g_p comes from the bits of amax (the same e as scaling amax by 1 /
-// g_p first, for normal amax), and the E2M1 codes are encoded and decoded by
-// the hardware conversions (round to nearest, ties to the even code,
-// saturating at 6: the codes of e2m1_encode).
-__device__ __forceinline__ void block_planes(float (&v)[4], int E, bool valid, int part, int j, int b,
+// log2 of plane p's factor g_p for a row (or chunk) exponent E.
+__device__ __forceinline__ int plane_log2_factor(int E, int p) { return E - 2 * p - 9; }
+
+// The P planes of one 16-element block (the bit window described above), by
+// the four lanes part = 0..3 of an aligned group of four (four elements each,
+// v[0..3] = elements 4 part ..; exact bf16 values; every lane of the warp
+// calls).  Writes bytes 8 b + 2 part, +1 of plane row j P + p (rows of
+// row_bytes) and, from part 0, the block's scale byte at [b / 4][rows][4] +
+// b % 4 for every plane.
+__device__ __forceinline__ void block_planes(const float (&v)[4], int E, bool valid, int part, int j, int b,
                                              uint8_t* codes, size_t row_bytes, uint8_t* sf, int rows) {
-  uint32_t pairs[kQPlanes], s8s[kQPlanes];
+  // significand M and exponent e of each element (M = 0 for zero)
+  uint32_t M[4], sgn[4];
+  int ev[4], T = -1000;
 #pragma unroll
-  for (int p = 0; p < kQPlanes; ++p) {
-    uint32_t am = max(max(__float_as_uint(v[0]) & 0x7fffffffu, __float_as_uint(v[1]) & 0x7fffffffu),
-                      max(__float_as_uint(v[2]) & 0x7fffffffu, __float_as_uint(v[3]) & 0x7fffffffu));
-    am = max(am, __shfl_xor_sync(0xffffffffu, am, 1));
-    am = max(am, __shfl_xor_sync(0xffffffffu, am, 2));
-    uint32_t s8 = 0, pair = 0;
-    if (am != 0) {
-      const int ge = E - 8 - (3 * p) / 2;  // log2 g_p
-      // smallest power of two 2^e >= amax / 6 / g_p, clamped to E4M3's 2^-9..2^8
-      int e;
-      if (am >= 0x00800000u) {  // normal: amax = 1.f * 2^k
-        const int k = (int)(am >> 23) - 127;
-        e = ((am & 0x7fffffu) <= 0x400000u ? k - 2 : k - 1) - ge;
-      } else {
-        e = ceil_log2_over_6(__uint_as_float(am) * exp2i(-ge));
-      }
-      e = e < -9 ? -9 : (e > 8 ? 8 : e);
-      s8 = e >= -6 ? (uint32_t)(e + 7) << 3 : (1u << (e + 9));
-      // r / (g_p 2^e) and the represented values are exact power-of-two
-      // scalings, and the new residual (q - value) g_p 2^e is exact (q and
-      // the value of its code are within a factor two)
-      const int sh = ge + e;
-      const float down = exp2i(-sh), up = exp2i(sh);
+  for (int i = 0; i < 4; ++i) {
+    const uint32_t bits = __float_as_uint(v[i]);
+    const uint32_t fe = (bits >> 23) & 0xffu, mant = (bits >> 16) & 0x7fu;
+    sgn[i] = bits >> 31;
+    M[i] = fe ? (0x80u | mant) : mant;  // bf16 subnormals: 0.mant * 2^-126
+    ev[i] = fe ? (int)fe - 127 : -126;
+    if (M[i]) T = max(T, ev[i]);
+  }
+  T = max(T, __shfl_xor_sync(0xffffffffu, T, 1));
+  T = max(T, __shfl_xor_sync(0xffffffffu, T, 2));
+  const int es = T - E + 8;  // block scale 2^es
+  const bool keep = T > -1000 && es >= -9;
+  const uint32_t s8 = !keep ? 0u : es >= -6 ? (uint32_t)(es + 7) << 3 : (1u << (es + 9));
+  uint32_t A[4];
 #pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        const float q0 = v[2 * h] * down, q1 = v[2 * h + 1] * down;
-        const uint32_t byte = (uint32_t)__nv_cvt_float2_to_fp4x2(make_float2(q0, q1), __NV_E2M1, cudaRoundNearest);
-        const __half2_raw hv = __nv_cvt_fp4x2_to_halfraw2((__nv_fp4x2_storage_t)byte, __NV_E2M1);
-        __half_raw h0, h1;
-        h0.x = hv.x;
-        h1.x = hv.y;
-        v[2 * h] = (q0 - __half2float(__half(h0))) * up;
-        v[2 * h + 1] = (q1 - __half2float(__half(h1))) * up;
-        pair |= byte << (8 * h);
-      }
-    }
-    pairs[p] = pair;
-    s8s[p] = s8;
+  for (int i = 0; i < 4; ++i) {
+    const int sh = ev[i] - T + 8;  // <= 8
+    A[i] = !keep || M[i] == 0 ? 0u : sh >= 0 ? M[i] << sh : (sh > -16 ? M[i] >> -sh : 0u);
   }
   if (valid) {
 #pragma unroll
     for (int p = 0; p < kQPlanes; ++p) {
+      uint32_t pair = 0;
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const uint32_t d = (A[i] >> (14 - 2 * p)) & 3u;  // E2M1 code of d: 0, 2 (1.0), 4 (2.0), 5 (3.0)
+        const uint32_t c = d ? ((0x5420u >> (4 * d)) & 0xfu) | (sgn[i] << 3) : 0u;
+        pair |= c << (4 * i);
+      }
       const int rowp = j * kQPlanes + p;
-      *reinterpret_cast<uint16_t*>(codes + (size_t)rowp * row_bytes + 8 * b + 2 * part) = (uint16_t)pairs[p];
-      if (part == 0) sf[((size_t)(b >> 2) * rows + rowp) * 4 + (b & 3)] = (uint8_t)s8s[p];
+      *reinterpret_cast<uint16_t*>(codes + (size_t)rowp * row_bytes + 8 * b + 2 * part) = (uint16_t)pair;
+      if (part == 0) sf[((size_t)(b >> 2) * rows + rowp) * 4 + (b & 3)] = (uint8_t)s8;
     }
   }
 }
@@ -1748,7 +1720,7 @@ __global__ void __launch_bounds__(kLayerThreads, 2) tc_planes_layer_kernel(const
                 for (int p = 0; p < P; ++p) {
                   const float dv = (had[0] ? __uint_as_float(d0[jr * P + p]) : 0.0f) +
                                    (had[1] ? __uint_as_float(d1[jr * P + p]) : 0.0f);
-                  y[jr] = fmaf(exp2i(E[jr] - 8 - (3 * p) / 2), dv, y[jr]);
+                  y[jr] = fmaf(exp2i(plane_log2_factor(E[jr], p)), dv, y[jr]);
                 }
               }
             }
