@@ -87,7 +87,9 @@ const char* ffn_status_string(ffn_status s);
 /* FFN_NVFP4_ABI_VERSION of the built library. */
 int ffn_nvfp4_abi_version(void);
 
-/* Quantise a bf16 weight W[n, k] to NVFP4.
+/* Quantise a bf16 weight W[n, k] to NVFP4.  (The pages name NVFP4 weights
+ * but print no quantiser; the format is the public NVFP4 one, readings
+ * R1-R4 of the design notes.)
  *   w_bf16        [n, k] bf16 (input)
  *   codes         uint8 [n, k/2]  (output)
  *   block_scales  uint8 [n, k/16] (output, E4M3)
@@ -105,7 +107,8 @@ ffn_status ffn_nvfp4_quantize_weights(const void* w_bf16, int64_t n, int64_t k,
                                       float* global_scale, void* stream);
 
 /* Quantise bf16 activations X[m, k] per row to NVFP4, as the fixed format does
- * before each projection: per 16-element block s = E4M3(block amax / 6) (fp32,
+ * before each projection ("metrale_model_layers/layers/dense_ffn_fixed.rs",
+ * forward_fixed: nvfp4_proj_mx on bf16 rows): per 16-element block s = E4M3(block amax / 6) (fp32,
  * nearest even, saturating), code = E2M1(x / E4M3value(s)), no tensor scale;
  * all-zero block when s == 0.  codes uint8 [m, k/2], block_scales uint8
  * [m, k/16].  Exposed so callers can check the activation codes bit for bit. */
@@ -140,7 +143,9 @@ ffn_status ffn_nvfp4_weight_create(const void* codes, const void* block_scales,
                                    const float* global_scale, int64_t n, int64_t k,
                                    void* stream, ffn_nvfp4_weight** out);
 
-/* Fused gate+up handle of logical shape [2*inter, hidden]: rows [0, inter)
+/* Fused gate+up handle of logical shape [2*inter, hidden]
+ * ("metrale_model_layers/layers/dense_ffn_overlays.rs", set_fp8_gate_up_fused:
+ * one [2I, H] buffer whose halves are the gate and up weights): rows [0, inter)
  * are `gate`, rows [inter, 2*inter) are `up`, byte for byte, each keeping its
  * own tensor scale; built for the formats both parts serve (re-tiled from
  * their tiles; FFN_ERR_UNSUPPORTED if they share none).  `gate` and `up` must
@@ -167,7 +172,10 @@ ffn_status ffn_nvfp4_weight_info(const ffn_nvfp4_weight* w, unsigned* formats,
 ffn_status ffn_nvfp4_workspace_size(int64_t m, int64_t hidden, int64_t inter,
                                     ffn_act_format format, size_t* bytes);
 
-/* The FFN layer for m rows.
+/* The FFN layer for m rows ("metrale_model_layers/layers/dense_ffn_prefill.rs",
+ * forward_prefill_inner with its NVFP4 arm w4a16_prefill_gemm, for bf16
+ * activations; "metrale_model_layers/layers/dense_ffn_fixed.rs", forward_fixed,
+ * for the fixed format).
  *   x        [m, hidden] bf16
  *   gate_up  fused handle [2*inter, hidden] (ffn_nvfp4_weight_create_gate_up)
  *   down     handle [hidden, inter]
@@ -232,7 +240,9 @@ ffn_status ffn_nvfp4_forward_lora(const void* x, int64_t m, int64_t hidden, int6
                                   void* workspace, size_t workspace_bytes, void* stream);
 
 /* One projection y[m, n] = bf16(gs * sum_k x[m, k] * w[n, k]) for a plain
- * (not gate+up) handle of shape [n, k]; in FFN_ACT_NVFP4_FIXED x is quantised
+ * (not gate+up) handle of shape [n, k] (one call of the per-projection GEMM
+ * that "metrale_model_layers/layers/dense_ffn_prefill.rs", w4a16_prefill_gemm,
+ * dispatches, e.g. the down projection); in FFN_ACT_NVFP4_FIXED x is quantised
  * per row first.  Workspace: ffn_nvfp4_linear_workspace_size bytes. */
 ffn_status ffn_nvfp4_linear_workspace_size(int64_t m, int64_t n, int64_t k,
                                            ffn_act_format format, size_t* bytes);
