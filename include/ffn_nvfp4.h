@@ -288,7 +288,10 @@ ffn_status ffn_nvfp4_linear_noalloc(const void* x, int64_t m, const ffn_nvfp4_we
 typedef enum ffn_kernel_family {
   FFN_KERNEL_NONE = 0,       /* m == 0: nothing is launched                     */
   FFN_KERNEL_TC_W4A16 = 1,   /* tcgen05 kind::f16 MMA over dequantised weights  */
-  FFN_KERNEL_TC_W4A4 = 2,    /* tcgen05 block-scaled FP4 MMA (kind::mxf4nvf4)   */
+  FFN_KERNEL_TC_W4A4 = 2,    /* tcgen05 block-scaled FP4 MMA (kind::mxf4nvf4);
+                                one activation tile of 128 rows per CTA, or of
+                                16 rows for m <= 16, two CTAs per SM; the K
+                                split depends on (n, k) only                   */
   FFN_KERNEL_GEMV_W4A16 = 3, /* CUDA-core projection, bf16 activations          */
   FFN_KERNEL_GEMV_W4A4 = 4,  /* CUDA-core projection, fixed activation format   */
   FFN_KERNEL_TC_W4A16_PERSISTENT = 5, /* few-row FFN layer: persistent tcgen05

@@ -634,8 +634,7 @@ ffn_status ffn_nvfp4_projection_plan(int64_t m, int64_t n, int64_t k, ffn_act_fo
     *out = ffn_projection_plan{FFN_KERNEL_GEMV_W4A16, 0, 1, ffn::gemv_grid(ncols)};
   } else if (w4a4_path() == Path::kTc) {
     const ffn::TcPlan p = ffn::plan_w4a4(m, n, k, gate_up != 0, num_sms());
-    const int xt = ffn::w4a4_tiles_per_cta(p.xtiles);
-    *out = ffn_projection_plan{FFN_KERNEL_TC_W4A4, p.bn, p.splits, (p.xtiles + xt - 1) / xt * p.wtiles * p.splits};
+    *out = ffn_projection_plan{FFN_KERNEL_TC_W4A4, p.bn, p.splits, p.xtiles * p.wtiles * p.splits};
   } else {
     *out = ffn_projection_plan{FFN_KERNEL_GEMV_W4A4, 0, 1, ffn::gemv_grid(ncols)};
   }

@@ -103,11 +103,10 @@ PlanesPlan plan_planes(int64_t m, int64_t hidden, int64_t inter, int num_sms);
 cudaError_t launch_planes_ffn(const void* x, int64_t m, const TcWeight& gate_up, const TcWeight& down,
                               const PlanesPlan& p, const PlanesBuffers& b, void* out, cudaStream_t s);
 // Fixed-format (W4A4) projection on the block-scaled FP4 tensor core.  The
-// plan depends on (n, k) only (plus the number of 128-row activation tiles).
+// K split depends on (n, k) only; the activation tile (16 rows for m <= 16,
+// else 128) and the number of tiles on m, neither of which changes a result
+// bit.
 TcPlan plan_w4a4(int64_t m, int64_t n, int64_t k, bool gate_up, int num_sms);
-// Activation tiles of 128 rows each CTA of the W4A4 kernel multiplies with
-// one weight stage (1 or 2; changes no result bit).
-int w4a4_tiles_per_cta(int xtiles);
 size_t w4a4_sf_block_bytes(int64_t m, int64_t k);
 // With silu_mul, no K split and hq_codes/hq_sf given, the epilogue writes the
 // per-row NVFP4 quantisation of h (codes [m, n/4], blocked scales) instead

@@ -969,23 +969,29 @@ tc_w4a16_persistent_kernel(const __grid_constant__ CUtensorMap xmap, const PArgs
 //    256 elements, 128-byte swizzle), scale blocks (one 512-byte block per
 //    128 rows and 64 elements, written by the activation quantiser) by bulk
 //    copy, copied to TMEM as SFB;
-//  * the tile shape (128 weight rows x 128 activation rows), the K split and
-//    the K order depend only on (n, K), never on m, and every output column
-//    of an MMA depends only on its own activation row, so a row's result is
-//    the same whatever m is.
+//  * the K split and the K order depend only on (n, K), never on m, and every
+//    output column of an MMA depends only on its own activation row, so a
+//    row's result is the same whatever m is;
+//  * one activation tile per CTA, 128 rows (MMA N = 128, a 3-stage ring of
+//    36 KB stages) or 16 rows for m <= 16 (N = 16, 5 stages of 22.5 KB), and
+//    two CTAs per SM: one CTA's epilogue overlaps the other's main loop, the
+//    few-row grids stream every weight tile at once instead of in waves, and
+//    the next kernel's CTAs find room beside this one's as soon as one of
+//    them ends.
 // ---------------------------------------------------------------------------
-constexpr int kW4BN = 128;        // activation rows per tile (fixed)
+constexpr int kW4BN = 128;        // activation rows per tile
+constexpr int kW4BNSmall = 16;    // activation rows per tile for m <= 16
 constexpr int kW4Chunks = 4;      // 64-element chunks per stage
 
-// XT activation tiles per CTA share each weight stage (one MMA per tile and
-// chunk, an accumulator each): the weights cross L2 once per XT tiles.  Every
-// activation row is still the N column of a 128-row MMA with the same K
-// order, so XT changes no result bit.
-template <int XT>
+// XT activation tiles per CTA would share each weight stage (one MMA per tile
+// and chunk, an accumulator each; every activation row stays the N column of
+// an MMA with the same K order, so XT changes no result bit); the shapes in
+// use take one tile (XT = 1), which lets two CTAs share an SM.
+template <int XT, int BN, int S>
 struct W4Cfg {
-  static constexpr int kStages = XT == 1 ? 5 : 4;
+  static constexpr int kStages = S;
   static constexpr int kWBytes = kW4Chunks * kChunkBytes;  // 18432
-  static constexpr int kXBytes = kW4BN * 128;              // 16384 (128 rows x 256 elements)
+  static constexpr int kXBytes = BN * 128;                 // BN rows x 256 elements
   static constexpr int kSfbBytes = kW4Chunks * 512;        // 2048
   static constexpr int kStageBytes = kWBytes + XT * (kXBytes + kSfbBytes);
   static constexpr int kSmemEpi = kStages * kStageBytes;
@@ -995,10 +1001,13 @@ struct W4Cfg {
   // TMEM columns: XT accumulators, then per activation tile (one MMA-issuing
   // warp each) its own copy of the weight scales, then its activation scales
   static constexpr int kSlotCols = 4 * kW4Chunks * kStages;
-  static constexpr int kSfaCol = XT * kW4BN;
+  static constexpr int kSfaCol = XT * BN < 32 ? 32 : XT * BN;
   static constexpr int kSfbCol = kSfaCol + XT * kSlotCols;
-  static constexpr int kTmemCols = 512;
+  static constexpr int kTmemCols = kSfbCol + XT * kSlotCols <= 256 ? 256 : 512;
+  // two CTAs per SM when both fit (228 KB of shared memory, 512 TMEM columns)
+  static constexpr int kMinBlocks = (2 * (kSmemAlloc + 1024) <= 233472 && kTmemCols <= 256) ? 2 : 1;
   static_assert(kSfbCol + XT * kSlotCols <= kTmemCols, "TMEM budget");
+  static_assert(BN == kW4BN || XT == 1, "narrow tiles: one per CTA");
   static_assert(kStageBytes % 1024 == 0, "stage alignment");
   static_assert(kSmemAlloc <= 232448, "shared memory budget");
   static_assert(kSmemEpi >= 2 * 16384, "the two epilogue buffers alias the rings");
@@ -1007,14 +1016,13 @@ struct W4Cfg {
 struct W4Args {
   TcArgs t;
   const uint8_t* sfb;   // activation scale blocks [ceil(m/128)][kc][512]
-  int xtiles;           // activation tiles of 128 rows
+  int xtiles;           // activation tiles (of BN rows)
 };
 
-template <int EPI, int XT>
-__global__ void __launch_bounds__(256, 1)
+template <int EPI, int XT, int BN, int S>
+__global__ void __launch_bounds__(256, W4Cfg<XT, BN, S>::kMinBlocks)
 tc_w4a4_kernel(const __grid_constant__ CUtensorMap xmap, const W4Args w4) {
-  using C = W4Cfg<XT>;
-  constexpr int S = C::kStages;
+  using C = W4Cfg<XT, BN, S>;
   const TcArgs& a = w4.t;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -1083,7 +1091,8 @@ tc_w4a4_kernel(const __grid_constant__ CUtensorMap xmap, const W4Args w4) {
         }
         for (int t = 0; t < nxt; ++t) {
           uint8_t* xt = st + C::kWBytes + t * (C::kXBytes + C::kSfbBytes);
-          tma_load_2d(xt, &xmap, 32 * (kc0 + kW4Chunks * i), (xt0 + t) * kW4BN, &full[s]);
+          tma_load_2d(xt, &xmap, 32 * (kc0 + kW4Chunks * i), (xt0 + t) * BN, &full[s]);
+          // (scale blocks cover 128 rows; a narrow tile is the only one: m <= BN)
           bulk_load(xt + C::kXBytes,
                     w4.sfb + ((size_t)(xt0 + t) * a.kc_total + kc0 + kW4Chunks * i) * 512, nch * 512, &full[s]);
         }
@@ -1096,7 +1105,7 @@ tc_w4a4_kernel(const __grid_constant__ CUtensorMap xmap, const W4Args w4) {
     // tcgen05 instruction streams; one thread's issue rate is the limit),
     // each with its own copy of the weight scales
     const int t = warp == 1 ? 0 : 1;
-    const uint32_t idesc = idesc_mxf4nvf4(kTileRows, kW4BN);
+    const uint32_t idesc = idesc_mxf4nvf4(kTileRows, BN);
     const uint32_t sfa0 = tmem + C::kSfaCol + t * C::kSlotCols, sfb0 = tmem + C::kSfbCol + t * C::kSlotCols;
     for (int i = 0; i < nstage; ++i) {
       const int s = i % S;
@@ -1113,7 +1122,7 @@ tc_w4a4_kernel(const __grid_constant__ CUtensorMap xmap, const W4Args w4) {
       }
       for (int c = 0; c < nch; ++c) {
         const uint32_t slot = 4 * (s * kW4Chunks + c);
-        mma_mxf4nvf4(tmem + t * kW4BN, smem_desc_interleave(smem_u32(st + c * kChunkBytes), 2048, 128),
+        mma_mxf4nvf4(tmem + t * BN, smem_desc_interleave(smem_u32(st + c * kChunkBytes), 2048, 128),
                      smem_desc_sw128(smem_u32(xt)) + 2 * c, idesc, sfa0 + slot, sfb0 + slot, (i | c) != 0 ? 1u : 0u);
       }
       mma_commit(&empty[s]);
@@ -1131,7 +1140,7 @@ tc_w4a4_kernel(const __grid_constant__ CUtensorMap xmap, const W4Args w4) {
     griddep_wait();  // the previous kernel may still read this kernel's outputs
     if (done && !*abort_flag)
       for (int t = 0; t < nxt; ++t)
-        epilogue_tile<kW4BN, EPI, 2>(a, tmem + t * kW4BN, q, lane, g, epi + g * 16384, xt0 + t, wtile);
+        epilogue_tile<BN, EPI, 2>(a, tmem + t * BN, q, lane, g, epi + g * 16384, xt0 + t, wtile);
   }
   tc_fence_before();
   __syncthreads();
@@ -2324,13 +2333,12 @@ cudaError_t launch_tc_w4a16(const void* x, int64_t m, const TcWeight& w, bool si
                   : launch_bn<kEpiStore>(p.bn, map, a, grid, s);
 }
 
-int w4a4_tiles_per_cta(int xtiles) { return xtiles >= 2 ? 2 : 1; }
 
 TcPlan plan_w4a4(int64_t m, int64_t n, int64_t k, bool gate_up, int num_sms) {
-  // Everything but the number of activation tiles depends on (n, k) only.
+  // The K split depends on (n, k) only; the tile width and count on m.
   TcPlan p;
-  p.bn = kW4BN;
-  p.xtiles = (int)((m + kW4BN - 1) / kW4BN);
+  p.bn = m <= kW4BNSmall ? kW4BNSmall : kW4BN;
+  p.xtiles = (int)((m + p.bn - 1) / p.bn);
   p.wtiles = (int)(gate_up ? (n / 2 + 63) / 64 : (n + kTileRows - 1) / kTileRows);
   p.kc = (int)((k + kChunkK - 1) / kChunkK);
   p.n_pad = p.wtiles * kTileRows;
@@ -2358,7 +2366,7 @@ cudaError_t launch_tc_w4a4(const uint8_t* xcodes, const uint8_t* xsf_blocks, int
   {
     cuuint64_t dims[2] = {(cuuint64_t)(w.k / 2), (cuuint64_t)m};
     cuuint64_t strides[1] = {(cuuint64_t)(w.k / 2)};
-    cuuint32_t box[2] = {128, (cuuint32_t)(m < kW4BN ? m : kW4BN)};
+    cuuint32_t box[2] = {128, (cuuint32_t)(m < p.bn ? m : p.bn)};
     cuuint32_t estr[2] = {1, 1};
     if (enc(&map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t*>(xcodes), dims, strides, box,
             estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
@@ -2367,7 +2375,8 @@ cudaError_t launch_tc_w4a4(const uint8_t* xcodes, const uint8_t* xsf_blocks, int
   }
   W4Args a;
   a.xtiles = p.xtiles;
-  a.t.x_box_rows = (int)(m < kW4BN ? m : kW4BN);
+  a.t.x_box_rows = (int)(m < p.bn ? m : p.bn);
+  if (p.bn != kW4BN && (p.bn != kW4BNSmall || m > p.bn)) return cudaErrorInvalidValue;
   a.t.wt = w.tiled;
   a.t.gs = w.gs;
   a.t.m = (int)m;
@@ -2377,23 +2386,25 @@ cudaError_t launch_tc_w4a4(const uint8_t* xcodes, const uint8_t* xsf_blocks, int
   a.t.kc_per_split = p.kc_per_split;
   a.t.n_pad = p.n_pad;
   a.sfb = xsf_blocks;
-  const int xt = w4a4_tiles_per_cta(p.xtiles);
-  const dim3 grid((p.xtiles + xt - 1) / xt, p.wtiles, p.splits);
-  auto launch = [&](auto kern1, auto kern2, int) -> cudaError_t {
-    // set on every launch: the attribute belongs to the current device's context
-    const int smem = xt == 1 ? W4Cfg<1>::kSmemAlloc : W4Cfg<2>::kSmemAlloc;
-    cudaError_t e = xt == 1 ? cudaFuncSetAttribute(kern1, cudaFuncAttributeMaxDynamicSharedMemorySize, smem)
-                            : cudaFuncSetAttribute(kern2, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-    if (e != cudaSuccess) return e;
-    return xt == 1 ? launch_pdl(kern1, grid, dim3(256), smem, s, map, a)
-                   : launch_pdl(kern2, grid, dim3(256), smem, s, map, a);
+  const dim3 grid(p.xtiles, p.wtiles, p.splits);
+  using CWide = W4Cfg<1, kW4BN, 3>;
+  using CNarrow = W4Cfg<1, kW4BNSmall, 5>;
+  auto launch = [&](auto kern_wide, auto kern_narrow) -> cudaError_t {
+    // set on every launch: the attributes belong to the current device's context
+    auto go = [&](auto kern, int smem) -> cudaError_t {
+      cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+      if (e == cudaSuccess)
+        e = cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout, cudaSharedmemCarveoutMaxShared);
+      return e == cudaSuccess ? launch_pdl(kern, grid, dim3(256), smem, s, map, a) : e;
+    };
+    return p.bn == kW4BNSmall ? go(kern_narrow, CNarrow::kSmemAlloc) : go(kern_wide, CWide::kSmemAlloc);
   };
   cudaError_t e;
   if (p.splits > 1) {
     a.t.out = partials;
     {
       ProfScope prof(s, silu_mul ? "tc_w4a4_gate_up_partial" : "tc_w4a4_partial");
-      e = launch(tc_w4a4_kernel<kEpiPartial, 1>, tc_w4a4_kernel<kEpiPartial, 2>, kEpiPartial);
+      e = launch(tc_w4a4_kernel<kEpiPartial, 1, kW4BN, 3>, tc_w4a4_kernel<kEpiPartial, 1, kW4BNSmall, 5>);
     }
     if (e != cudaSuccess) return e;
     const int64_t total = m * a.t.n_out;
@@ -2411,11 +2422,11 @@ cudaError_t launch_tc_w4a4(const uint8_t* xcodes, const uint8_t* xsf_blocks, int
     a.t.q_sf = hq_sf;
     a.t.q_kc = (int)((a.t.n_out + kChunkK - 1) / kChunkK);
     ProfScope prof(s, "tc_w4a4_gate_up_silu_quant");
-    return launch(tc_w4a4_kernel<kEpiSiluMulQuant, 1>, tc_w4a4_kernel<kEpiSiluMulQuant, 2>, kEpiSiluMulQuant);
+    return launch(tc_w4a4_kernel<kEpiSiluMulQuant, 1, kW4BN, 3>, tc_w4a4_kernel<kEpiSiluMulQuant, 1, kW4BNSmall, 5>);
   }
   ProfScope prof(s, silu_mul ? "tc_w4a4_gate_up_silu" : "tc_w4a4");
-  return silu_mul ? launch(tc_w4a4_kernel<kEpiSiluMul, 1>, tc_w4a4_kernel<kEpiSiluMul, 2>, kEpiSiluMul)
-                  : launch(tc_w4a4_kernel<kEpiStore, 1>, tc_w4a4_kernel<kEpiStore, 2>, kEpiStore);
+  return silu_mul ? launch(tc_w4a4_kernel<kEpiSiluMul, 1, kW4BN, 3>, tc_w4a4_kernel<kEpiSiluMul, 1, kW4BNSmall, 5>)
+                  : launch(tc_w4a4_kernel<kEpiStore, 1, kW4BN, 3>, tc_w4a4_kernel<kEpiStore, 1, kW4BNSmall, 5>);
 }
 
 cudaError_t read_device_error(int* flags, bool clear) {
