@@ -110,15 +110,19 @@ def nvfp4_bytes(n, k):
 # --------------------------------------------------------------- clocks
 
 # DRAM traffic per launch (dram__bytes_read.sum + dram__bytes_write.sum) from
-# one ncu capture, keyed by (kernel, workload), with a fingerprint of the kernel
+# one ncu capture, keyed by (kernel, workload, m), with a fingerprint of the kernel
 # sources it was taken on (comments and whitespace ignored): reported only
 # while the sources are unchanged.
 KERNEL_SOURCES = ("csrc/tc_gemm.cu", "csrc/sm100.cuh", "csrc/common.cuh", "csrc/internal.h")
 TRAFFIC = {
-    ("tc_w4a16_gate_up_silu", "prefill"): {
-        "bytes": 148308480 + 128401664, "sources_sha1": "2610cbb5053b6413db136c565b839e635643644e"},
-    ("tc_planes_layer", "decode"): {
-        "bytes": 150508288 + 4229888, "sources_sha1": "2610cbb5053b6413db136c565b839e635643644e"},
+    ("tc_w4a16_gate_up_silu", "prefill", 4096): {
+        "bytes": 150610176 + 130894592, "sources_sha1": "8a93041e3bd8ed20dc33a186a7e2a2a15658e11c"},
+    ("tc_planes_layer", "decode", 1): {
+        "bytes": 150507008 + 4579584, "sources_sha1": "8a93041e3bd8ed20dc33a186a7e2a2a15658e11c"},
+    ("tc_w4a4_gate_up_silu_quant", "w4a4", 512): {
+        "bytes": 57844480 + 1723648, "sources_sha1": "8a93041e3bd8ed20dc33a186a7e2a2a15658e11c"},
+    ("tc_w4a4_gate_up_silu_quant", "w4a4", 1): {
+        "bytes": 56698368 + 9472, "sources_sha1": "8a93041e3bd8ed20dc33a186a7e2a2a15658e11c"},
 }
 
 def normalised_source(text):
@@ -143,8 +147,8 @@ def kernel_sources_sha1(read=None):
     return h.hexdigest()
 
 
-def measured_traffic(kname, workload):
-    t = TRAFFIC.get((kname, workload))
+def measured_traffic(kname, workload, m=None):
+    t = TRAFFIC.get((kname, workload, m))
     if t is None or t["sources_sha1"] != kernel_sources_sha1():
         return None
     return t["bytes"]
@@ -302,7 +306,7 @@ def roofline(wl, prof, peaks, peak_src, workload):
         unit = "GB/s"
     return {"kernel": kname, "bound": bound, "achieved": round(achieved, 2), "peak": peak,
             "peak_source": f"{peak_src} ({what})", "unit": unit, "frac": round(achieved / peak, 4),
-            "traffic": measured_traffic(kname, workload),
+            "traffic": measured_traffic(kname, workload, wl.m),
             "avg_launch_us": round(avg_s * 1e6, 2), "launches": launches}
 
 
