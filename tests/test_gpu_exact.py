@@ -106,6 +106,8 @@ W4A4_CASES = [
     (7, 256, 1024, None), (64, 640, 2048, None),
     # three activation tiles: CTAs of two tiles and a last CTA of one
     (300, 256, 512, None), (300, 128, 4096, 8),
+    # either side of the switch from 16-row to 128-row activation tiles
+    (16, 256, 1024, None), (17, 256, 1024, None),
 ]
 
 
@@ -113,6 +115,7 @@ W4A4_CASES = [
 def test_w4a4_exact_inputs_bit_exact(native, m, n, k, splits):
     plan = native.ffn_nvfp4_projection_plan(m, n, k, "nvfp4_fixed")
     assert plan["family"] == "tc_w4a4", plan
+    assert plan["tile_rows"] == (16 if m <= 16 else 128), plan
     if splits is not None:
         assert plan["k_splits"] == splits, plan
     rng = np.random.default_rng(2000 + m + n + k)

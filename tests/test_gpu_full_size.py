@@ -47,8 +47,10 @@ def w4a4(native):
 
 
 def test_w4a4_rows_bitwise_invariant_across_m(native, w4a4):
+    # m <= 16 takes 16-row activation tiles (MMA N = 16), larger m 128-row
+    # tiles: 16 and 17 sit on either side of that switch
     outs = {m: w4a4.forward("nvfp4_fixed", rows=m).view(torch.int16).cpu().numpy()
-            for m in (1, 7, 64, 512)}
+            for m in (1, 7, 16, 17, 64, 512)}
     for m, o in outs.items():
         assert np.array_equal(o, outs[512][:m]), f"rows of m={m} differ from m=512"
     # and the m=1 result again (same launch twice)
