@@ -1868,6 +1868,72 @@ __global__ void splitk_reduce_kernel(const float* __restrict__ P, int splits, in
   }
 }
 
+// The same reduction, four adjacent outputs per thread (16-byte partial loads,
+// one 8-byte store); each output's sum and epilogue are those above, in the
+// same order, so the results are identical.  Needs n_out and ldo divisible by
+// 4 (a group of four never crosses a 64-column gate/up block).
+template <bool kGateUp>
+__global__ void splitk_reduce4_kernel(const float* __restrict__ P, int splits, int m, int n_pad,
+                                      int n_out, const float* __restrict__ gs, float gs_mul,
+                                      uint16_t* __restrict__ out, int ldo, const LoraArgs lora) {
+  griddep_wait();  // the partial sums come from the previous kernel
+  griddep_launch_dependents();
+  const int nq = n_out / 4;
+  const int64_t idx = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;
+  if (idx >= (int64_t)m * nq) return;
+  const int r = (int)(idx / nq), n = 4 * (int)(idx % nq);
+  const size_t plane = (size_t)m * n_pad;
+  uint16_t o[4];
+  if (kGateUp) {
+    const int gcol = kTileRows * (n / 64) + (n % 64), ucol = gcol + 64;
+    float g[4] = {0.0f, 0.0f, 0.0f, 0.0f}, u[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+    for (int z = 0; z < splits; ++z) {
+      const float4 gv = *reinterpret_cast<const float4*>(P + z * plane + (size_t)r * n_pad + gcol);
+      const float4 uv = *reinterpret_cast<const float4*>(P + z * plane + (size_t)r * n_pad + ucol);
+      g[0] += gv.x; g[1] += gv.y; g[2] += gv.z; g[3] += gv.w;
+      u[0] += uv.x; u[1] += uv.y; u[2] += uv.z; u[3] += uv.w;
+    }
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const float gb = lora_add(bf16_round(gs[0] * gs_mul * g[i]), lora.b0, lora.off0, lora, r, n + i);
+      const float ub = lora_add(bf16_round(gs[1] * gs_mul * u[i]), lora.b1, lora.off1, lora, r, n + i);
+      o[i] = f32_to_bf16_bits(silu_fast(gb) * ub);
+    }
+  } else {
+    float acc[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+    for (int z = 0; z < splits; ++z) {
+      const float4 v = *reinterpret_cast<const float4*>(P + z * plane + (size_t)r * n_pad + n);
+      acc[0] += v.x; acc[1] += v.y; acc[2] += v.z; acc[3] += v.w;
+    }
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      float y = gs[0] * gs_mul * acc[i];
+      if (lora.b0) y = lora_add(bf16_round(y), lora.b0, lora.off0, lora, r, n + i);
+      o[i] = f32_to_bf16_bits(y);
+    }
+  }
+  *reinterpret_cast<uint2*>(out + (size_t)r * ldo + n) =
+      make_uint2((uint32_t)o[0] | ((uint32_t)o[1] << 16), (uint32_t)o[2] | ((uint32_t)o[3] << 16));
+}
+
+// Launch the split-K reduction (four outputs per thread when the shapes allow).
+cudaError_t launch_splitk_reduce(bool gate_up, const float* P, int splits, int64_t m, int n_pad, int n_out,
+                                 const float* gs, float gs_mul, uint16_t* y, int ldo, const LoraArgs& lora,
+                                 cudaStream_t s) {
+  if (n_out % 4 == 0 && ldo % 4 == 0) {
+    const dim3 rgrid((unsigned)((m * (n_out / 4) + 255) / 256));
+    return gate_up ? launch_pdl(splitk_reduce4_kernel<true>, rgrid, dim3(256), 0, s, P, splits, (int)m, n_pad,
+                                n_out, gs, gs_mul, y, ldo, lora)
+                   : launch_pdl(splitk_reduce4_kernel<false>, rgrid, dim3(256), 0, s, P, splits, (int)m, n_pad,
+                                n_out, gs, gs_mul, y, ldo, lora);
+  }
+  const dim3 rgrid((unsigned)((m * n_out + 255) / 256));
+  return gate_up ? launch_pdl(splitk_reduce_kernel<true>, rgrid, dim3(256), 0, s, P, splits, (int)m, n_pad, n_out,
+                              gs, gs_mul, y, ldo, lora)
+                 : launch_pdl(splitk_reduce_kernel<false>, rgrid, dim3(256), 0, s, P, splits, (int)m, n_pad, n_out,
+                              gs, gs_mul, y, ldo, lora);
+}
+
 // Re-tile a canonical NVFP4 weight (codes [n, k/2], scales [n, k/16]) into the
 // per-(128-row tile, 64-element chunk) layout the kernel streams.  For a fused
 // gate+up weight (half = inter), tile t holds gate rows [64t, 64t+64) followed
@@ -2316,16 +2382,9 @@ cudaError_t launch_tc_w4a16(const void* x, int64_t m, const TcWeight& w, bool si
       e = launch_bn<kEpiPartial>(p.bn, map, a, grid, s);
     }
     if (e != cudaSuccess) return e;
-    const int64_t total = m * a.n_out;
     ProfScope prof(s, silu_mul ? "splitk_reduce_silu_mul" : "splitk_reduce");
-    const dim3 rgrid((unsigned)((total + 255) / 256));
-    const float* P = static_cast<const float*>(partials);
-    return silu_mul ? launch_pdl(splitk_reduce_kernel<true>, rgrid, dim3(256), 0, s, P, p.splits,
-                                 (int)m, p.n_pad, a.n_out, w.gs, kW4A16Unscale,
-                                 static_cast<uint16_t*>(y), a.ldo, lora)
-                    : launch_pdl(splitk_reduce_kernel<false>, rgrid, dim3(256), 0, s, P, p.splits,
-                                 (int)m, p.n_pad, a.n_out, w.gs, kW4A16Unscale,
-                                 static_cast<uint16_t*>(y), a.ldo, lora);
+    return launch_splitk_reduce(silu_mul, static_cast<const float*>(partials), p.splits, m, p.n_pad, a.n_out,
+                                w.gs, kW4A16Unscale, static_cast<uint16_t*>(y), a.ldo, lora, s);
   }
   a.out = y;
   ProfScope prof(s, silu_mul ? "tc_w4a16_gate_up_silu" : "tc_w4a16");
@@ -2407,14 +2466,9 @@ cudaError_t launch_tc_w4a4(const uint8_t* xcodes, const uint8_t* xsf_blocks, int
       e = launch(tc_w4a4_kernel<kEpiPartial, 1, kW4BN, 3>, tc_w4a4_kernel<kEpiPartial, 1, kW4BNSmall, 5>);
     }
     if (e != cudaSuccess) return e;
-    const int64_t total = m * a.t.n_out;
     ProfScope prof(s, silu_mul ? "splitk_reduce_silu_mul" : "splitk_reduce");
-    const dim3 rgrid((unsigned)((total + 255) / 256));
-    const float* P = static_cast<const float*>(partials);
-    return silu_mul ? launch_pdl(splitk_reduce_kernel<true>, rgrid, dim3(256), 0, s, P, p.splits, (int)m,
-                                 p.n_pad, a.t.n_out, w.gs, 1.0f, static_cast<uint16_t*>(y), a.t.ldo, LoraArgs())
-                    : launch_pdl(splitk_reduce_kernel<false>, rgrid, dim3(256), 0, s, P, p.splits, (int)m,
-                                 p.n_pad, a.t.n_out, w.gs, 1.0f, static_cast<uint16_t*>(y), a.t.ldo, LoraArgs());
+    return launch_splitk_reduce(silu_mul, static_cast<const float*>(partials), p.splits, m, p.n_pad, a.t.n_out,
+                                w.gs, 1.0f, static_cast<uint16_t*>(y), a.t.ldo, LoraArgs(), s);
   }
   a.t.out = y;
   if (silu_mul && hq_codes && hq_sf) {
