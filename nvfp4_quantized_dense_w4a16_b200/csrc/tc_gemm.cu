@@ -2137,8 +2137,9 @@ cudaError_t launch_layer(LArgs a, int max_grid, int num_sms, cudaStream_t s) {
   if (e == cudaSuccess) e = cudaGetDevice(&dev);
   if (e == cudaSuccess) e = cudaDeviceGetAttribute(&smem_sm, cudaDevAttrMaxSharedMemoryPerMultiprocessor, dev);
   if (e != cudaSuccess) return e;
-  // registers: __launch_bounds__(256, 2) keeps two CTAs within the register
-  // file; threads: 512 of 2048; shared memory (1 KB per CTA reserved):
+  // registers: __launch_bounds__(kLayerThreads, 2) keeps two CTAs within the
+  // register file; threads: 576 of 2048; shared memory (1 KB per CTA
+  // reserved; two CTAs of the 4-stage ring leave about 40 KB of an SM free):
   const int occupancy = 2 * (C::kSmemAlloc + 1024) <= smem_sm ? 2 : 1;
   const int grid = min(max_grid, occupancy * num_sms);
   if (grid < 1) return cudaErrorInvalidConfiguration;
