@@ -86,6 +86,16 @@ def test_traffic_reported_only_for_the_captured_sources():
     assert bench.measured_traffic("no_such_kernel", "prefill") is None
 
 
+def test_traffic_is_keyed_by_kernel_workload_and_rows(monkeypatch):
+    monkeypatch.setattr(bench, "kernel_sources_sha1", lambda read=None: "abc")
+    monkeypatch.setattr(bench, "TRAFFIC", {("k", "w4a4", 512): {"bytes": 123, "sources_sha1": "abc"},
+                                           ("k", "w4a4", 1): {"bytes": 7, "sources_sha1": "old"}})
+    assert bench.measured_traffic("k", "w4a4", 512) == 123
+    assert bench.measured_traffic("k", "w4a4", 64) is None      # another m: not captured
+    assert bench.measured_traffic("k", "w4a4", 1) is None       # captured on other sources
+    assert bench.measured_traffic("k", "prefill", 512) is None
+
+
 def test_roofline_bound_uses_each_formats_own_peak(layers):
     peaks = {"hbm_gbs": 6557.8, "bf16_tflops": 1671.7, "bf16_tflops_sustained": 1402.4}
     assert bench.tensor_peak(peaks, "bf16")[0] == 1671.7
